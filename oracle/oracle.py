@@ -1,0 +1,143 @@
+"""Python access to the C reference oracle (``ternary_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY.  Imported by ``tests/``, by ``__graft_entry__.smoke``
+and by the CPU-baseline leg of ``bench.py``; never by the product package.
+This module only marshals numpy arrays into the C functions; every step of
+the arithmetic lives in ``ternary_oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ternary_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_CFLAGS = ["-O1", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+           "-fexcess-precision=standard", "-shared", "-fPIC"]
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library next to its source."""
+    if force or not os.path.exists(_LIB) or (
+            os.path.getmtime(_LIB) < os.path.getmtime(_SRC)):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *_CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _bind(lib):
+    i64, p = ctypes.c_int64, ctypes.c_void_p
+    lib.orc_mean_abs.restype = ctypes.c_double
+    lib.orc_mean_abs.argtypes = [p, i64, i64]
+    lib.orc_ternarize.restype = ctypes.c_int
+    lib.orc_ternarize.argtypes = [p, i64, i64, p, p]
+    lib.orc_quantize_act.restype = None
+    lib.orc_quantize_act.argtypes = [p, i64, i64, p, p]
+    lib.orc_ternary_acc.restype = ctypes.c_int
+    lib.orc_ternary_acc.argtypes = [p, i64, i64, p, i64, p]
+    lib.orc_rescale.restype = None
+    lib.orc_rescale.argtypes = [p, i64, i64, p, ctypes.c_double, p]
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def use_library(path):
+    """Point this module at another build of the oracle source (the pin
+    tests use it to run the pins against deliberately broken copies).
+    Returns the previously bound library; pass it back to restore."""
+    global _lib
+    prev = _load()
+    _lib = path if isinstance(path, ctypes.CDLL) else _bind(ctypes.CDLL(path))
+    return prev
+
+
+def compile_variant(src_text: str, out_path: str) -> str:
+    """Compile a (modified) copy of the oracle source with the same flags."""
+    c_path = out_path + ".c"
+    with open(c_path, "w") as f:
+        f.write(src_text)
+    subprocess.run(["gcc", *_CFLAGS, "-o", out_path, c_path, "-lm"], check=True)
+    return out_path
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data
+
+
+def mean_abs(W) -> float:
+    W, pw = _c(W, np.float32)
+    N, K = W.shape
+    return float(_load().orc_mean_abs(pw, N, K))
+
+
+def ternarize(W):
+    """Return (codes int8 [N,K], mean float).  Raises on non-finite W."""
+    W, pw = _c(W, np.float32)
+    N, K = W.shape
+    codes = np.empty((N, K), np.int8)
+    mean = ctypes.c_double()
+    rc = _load().orc_ternarize(pw, N, K, ctypes.addressof(mean),
+                               codes.ctypes.data)
+    if rc != 0:
+        raise ValueError("non-finite value in W")
+    return codes, mean.value
+
+
+def quantize_act(x):
+    """Return (q int8 [M,K], amax float32 [M])."""
+    x, px = _c(x, np.float32)
+    M, K = x.shape
+    q = np.empty((M, K), np.int8)
+    amax = np.empty(M, np.float32)
+    _load().orc_quantize_act(px, M, K, q.ctypes.data, amax.ctypes.data)
+    return q, amax
+
+
+def ternary_acc(codes, q):
+    """Return acc int32 [M,N] = q @ codes.T (raises on int32 overflow)."""
+    codes, pc = _c(codes, np.int8)
+    q, pq = _c(q, np.int8)
+    N, K = codes.shape
+    M, K2 = q.shape
+    assert K == K2
+    acc = np.empty((M, N), np.int32)
+    if _load().orc_ternary_acc(pc, N, K, pq, M, acc.ctypes.data) != 0:
+        raise OverflowError("accumulator does not fit int32")
+    return acc
+
+
+def rescale(acc, amax, mean: float):
+    """Return y float64 [M,N] = acc * (amax/127) * mean."""
+    acc, pa = _c(acc, np.int32)
+    amax, pm = _c(amax, np.float32)
+    M, N = acc.shape
+    y = np.empty((M, N), np.float64)
+    _load().orc_rescale(pa, M, N, pm, float(mean), y.ctypes.data)
+    return y
+
+
+def ternary_linear(x, codes, mean: float):
+    """Whole layer on ternary codes: returns dict(q, amax, acc, y)."""
+    q, amax = quantize_act(x)
+    acc = ternary_acc(codes, q)
+    y = rescale(acc, amax, mean)
+    return {"q": q, "amax": amax, "acc": acc, "y": y}

@@ -1,0 +1,159 @@
+/*
+ * ternary_oracle.c — reference oracle for the ternary-weight linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is plain, slow, single-threaded C
+ * that restates what the method computes, for the parity tests, the smoke
+ * check and the CPU-baseline leg of the benchmark.  Nothing in the product
+ * path may include, link or call it, and it shares no code, header, table or
+ * helper with the CUDA implementation.
+ *
+ * What it computes (sources are the pages on VibeVoice-ASR-BitNet):
+ *   - Per-tensor ternarisation of a projection matrix W [N x K]:
+ *       s = 1 / mean|W| over the whole tensor, codes = round(W * s) clipped
+ *       to {-1, 0, +1}.  ("VibeVoice-ASR-BitNet-ONNX" model page,
+ *       "Quantization" table, row "LM projections (196 mats)": I2_S ternary,
+ *       per-tensor s = 1/mean|W|; "The Paper Says ARM Support" post, section
+ *       "What the model is trying to do": every weight becomes -1, 0 or +1.)
+ *   - Per-token int8 activation quantisation by absmax, an int32 (here
+ *       int64-checked) ternary dot product, and the rescale by absmax/127 and
+ *       1/s.  The pages only say the engine uses fused INT8 operations
+ *       (xujun.org article, section on heterogeneous quantisation; aitrends
+ *       summary, "Technical features"); the formula below is the plainest
+ *       reading of absmax int8 quantisation.
+ *   - The dot product itself is a plain sum of code * q: ternary weights turn
+ *       the multiply into add/subtract (xujun.org article, heterogeneous
+ *       quantisation section).
+ *
+ * Readings taken where the pages are silent (each one is listed in the
+ * design notes of the repository):
+ *   R1  rounding of W*s and of x*scale is round-half-to-even (IEEE rint).
+ *   R2  mean|W| is accumulated in fp64 in a fixed order: each row summed
+ *       sequentially over k, then the row sums summed sequentially over n;
+ *       the total is divided by N*K.
+ *   R3  mean|W| is floored at 1e-5 (an all-zero W then gives all-zero codes).
+ *   R4  the activation scale is computed in fp32: amax = max|x| (exact),
+ *       scale = 127.0f / amax (IEEE single division), q = rint(x * scale) in
+ *       single precision, clamped to [-128, 127].  A row with amax == 0 gives
+ *       q == 0 and y == 0.
+ *   R5  y = acc * (amax / 127) * mean|W|, evaluated here in fp64.
+ *
+ * Build: gcc -O1 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC
+ * (contraction off so that x * scale is a single IEEE multiply).
+ */
+#include <math.h>
+#include <stdint.h>
+
+#define ORC_MEAN_FLOOR 1e-5
+
+/* R2 + R3: mean of |W| over the whole [N x K] tensor. */
+double orc_mean_abs(const float *W, int64_t N, int64_t K)
+{
+    double total = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+        double row = 0.0;
+        for (int64_t k = 0; k < K; ++k)
+            row += fabs((double)W[n * K + k]);
+        total += row;
+    }
+    double mean = total / (double)(N * K);
+    if (mean < ORC_MEAN_FLOOR)
+        mean = ORC_MEAN_FLOOR;
+    return mean;
+}
+
+/* Ternarise W with s = 1/mean|W|.  Writes codes[n*K+k] in {-1,0,1} and the
+ * mean to *mean_out.  Returns 0, or 1 if W holds a non-finite value (codes
+ * are then left unwritten). */
+int orc_ternarize(const float *W, int64_t N, int64_t K, double *mean_out,
+                  int8_t *codes)
+{
+    for (int64_t i = 0; i < N * K; ++i)
+        if (!isfinite(W[i]))
+            return 1;
+    double mean = orc_mean_abs(W, N, K);
+    double s = 1.0 / mean;
+    for (int64_t i = 0; i < N * K; ++i) {
+        double r = rint((double)W[i] * s);
+        if (r > 1.0)
+            r = 1.0;
+        if (r < -1.0)
+            r = -1.0;
+        codes[i] = (int8_t)r;
+    }
+    *mean_out = mean;
+    return 0;
+}
+
+/* R4: per-token absmax int8 quantisation of x [M x K]. */
+void orc_quantize_act(const float *x, int64_t M, int64_t K, int8_t *q,
+                      float *amax)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        const float *row = x + m * K;
+        float a = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = fabsf(row[k]);
+            if (v > a)
+                a = v;
+        }
+        amax[m] = a;
+        if (a == 0.0f) {
+            for (int64_t k = 0; k < K; ++k)
+                q[m * K + k] = 0;
+            continue;
+        }
+        float scale = 127.0f / a;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = row[k] * scale;
+            float r = rintf(v);
+            if (r > 127.0f)
+                r = 127.0f;
+            if (r < -128.0f)
+                r = -128.0f;
+            q[m * K + k] = (int8_t)r;
+        }
+    }
+}
+
+/* acc[m*N+n] = sum_k codes[n*K+k] * q[m*K+k].  Summed in int64; returns 0,
+ * or 1 if a sum does not fit int32 (acc is still written, truncated). */
+int orc_ternary_acc(const int8_t *codes, int64_t N, int64_t K,
+                    const int8_t *q, int64_t M, int32_t *acc)
+{
+    int overflow = 0;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t sum = 0;
+            for (int64_t k = 0; k < K; ++k)
+                sum += (int64_t)codes[n * K + k] * (int64_t)q[m * K + k];
+            if (sum > INT32_MAX || sum < INT32_MIN)
+                overflow = 1;
+            acc[m * N + n] = (int32_t)sum;
+        }
+    }
+    return overflow;
+}
+
+/* R5: y[m*N+n] = acc[m*N+n] * (amax[m] / 127) * mean, in fp64. */
+void orc_rescale(const int32_t *acc, int64_t M, int64_t N, const float *amax,
+                 double mean, double *y)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        double a = (double)amax[m] / 127.0;
+        for (int64_t n = 0; n < N; ++n)
+            y[m * N + n] = (double)acc[m * N + n] * a * mean;
+    }
+}
+
+/* The whole layer on already-ternarised codes: quantise x, accumulate,
+ * rescale.  Any of q_out / amax_out / acc_out may be scratch supplied by the
+ * caller; all are written.  Returns the overflow flag of orc_ternary_acc. */
+int orc_ternary_linear(const float *x, int64_t M, const int8_t *codes,
+                       int64_t N, int64_t K, double mean, int8_t *q_out,
+                       float *amax_out, int32_t *acc_out, double *y_out)
+{
+    orc_quantize_act(x, M, K, q_out, amax_out);
+    int ovf = orc_ternary_acc(codes, N, K, q_out, M, acc_out);
+    orc_rescale(acc_out, M, N, amax_out, mean, y_out);
+    return ovf;
+}
