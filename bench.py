@@ -1,0 +1,351 @@
+"""Benchmark of the ternary-weight decoder projections on B200.
+
+Default workload: the full decode sweep — 28 layers x 7 projections = 196
+ternary matrices of a Qwen2.5-1.5B-shaped decoder (q/o 1536x1536, k/v
+256x1536, gate/up 8960x1536, down 1536x8960; 1,310,195,712 weights,
+327,548,928 bytes of 2-bit codes), one token (M = 1), seeded synthetic
+weights N(0, 0.02^2) and activations N(0, 1) with 1% outlier channels x20.
+A step is one pass of the whole hot path over every projection: fused
+activation quantisation, ternary product, rescale (one persistent launch).
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own
+replica of the sweep on its own token (data-parallel decode; no collective
+on the data path), value = all ranks' tokens / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "196-matrix ternary decode sweep tokens/s & weight GB/s (% of HBM roofline)"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--m", type=int, default=1, help="tokens per step (decode: 1..32)")
+    ap.add_argument("--layers", type=int, default=28)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", FALLBACK_HBM_GBS), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def sweep_bytes(shapes, M):
+    codes = sum((-(-N // 16) * 16) * K // 4 for (_, _, _, N, K) in shapes)
+    algo_codes = sum(N * K // 4 for (_, _, _, N, K) in shapes)
+    xin = sum(M * K * 4 for (_, _, _, N, K) in shapes)
+    yout = sum(M * N * 4 for (_, _, _, N, K) in shapes)
+    return algo_codes + xin + yout, algo_codes, codes
+
+
+class ClockSampler:
+    """Polls SM clock, power and throttle reasons through NVML while running."""
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.stop_ev = [], set(), threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.nv, self.err = None, str(e)
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksThrottleReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksThrottleReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksThrottleReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksThrottleReasonSwPowerCap", 0x4),
+        }
+        while not self.stop_ev.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append(mhz)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self.stop_ev.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.nv:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def build_workload(api, torch, dev, M, layers, rank):
+    """Generate, upload and ternarise the sweep; return descriptors and buffers."""
+    from ternary_weight_decoder_b200 import synth
+    shapes = synth.sweep_shapes(layers)
+    x_off, y_off, xo, yo = [], [], 0, 0
+    for (_, _, _, N, K) in shapes:
+        x_off.append(xo)
+        y_off.append(yo)
+        xo += M * K
+        yo += M * N
+    x_host = torch.empty(xo, dtype=torch.float32).pin_memory()
+    xn = x_host.numpy()
+    descs = []
+    x_all = torch.empty(xo, dtype=torch.float32, device=dev)
+    y_all = torch.empty(yo, dtype=torch.float32, device=dev)
+    for i, (l, p, name, N, K) in enumerate(shapes):
+        W = synth.weights(l, p, N, K)
+        Wd = torch.from_numpy(W).to(dev)
+        packed, mean_abs, wscale = api.ternarize_pack(Wd)
+        del Wd
+        # each rank decodes its own token stream
+        xn[x_off[i]:x_off[i] + M * K] = synth.activations(l + 1000 * rank, p, M, K).ravel()
+        descs.append(dict(x=x_all[x_off[i]:x_off[i] + M * K].view(M, K), packed=packed,
+                          wscale=wscale, y=y_all[y_off[i]:y_off[i] + M * N].view(M, N),
+                          N=N, K=K))
+    api.check()
+    x_all.copy_(x_host)
+    torch.cuda.synchronize()
+    return shapes, descs, x_host, x_all, y_all
+
+
+def cpu_oracle_sample(M, budget_s=12.0, layers=28):
+    """Time the reference oracle on host cores over whole projections of the
+    sweep until about budget_s of timed work; return tokens/s scaled by the
+    weight count."""
+    from oracle import oracle as orc
+    from ternary_weight_decoder_b200 import synth
+    shapes = synth.sweep_shapes(layers)
+    total_w = sum(N * K for (_, _, _, N, K) in shapes)
+    timed, done_w, used = 0.0, 0, []
+    for (l, p, name, N, K) in shapes:
+        W = synth.weights(l, p, N, K)
+        x = synth.activations(l, p, M, K)
+        codes, mean = orc.ternarize(W)
+        t0 = time.perf_counter()
+        orc.ternary_linear(x, codes, mean)
+        timed += time.perf_counter() - t0
+        done_w += N * K
+        used.append(f"L{l}.{name}")
+        if timed >= budget_s:
+            break
+    sweep_s = timed * total_w / done_w
+    return {"value": M / sweep_s, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": (f"{len(used)} of {len(shapes)} projections ({used[0]}..{used[-1]}, "
+                       f"{done_w / total_w:.3f} of the weights) at M={M}, "
+                       f"{timed:.1f} s timed, scaled to the full sweep by weight count")}
+
+
+def run_reference(args):
+    """The oracle as it stands, on host cores, on the same metric and config."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import oracle as orc
+    from ternary_weight_decoder_b200 import synth
+    M = args.m
+    shapes = synth.sweep_shapes(args.layers)
+    total_w = sum(N * K for (_, _, _, N, K) in shapes)
+    # per-step sample: leading rows of each projection of layer 0, sized so
+    # that warm-up + steps take about 60 s in total (at most ~2 s a step)
+    per_step_s = min(2.0, 60.0 / max(1, args.steps + args.warmup))
+    calib = []
+    for (l, p, name, N, K) in shapes[:7]:
+        W = synth.weights(l, p, N, K)
+        codes, mean = orc.ternarize(W)
+        x = synth.activations(l, p, M, K)
+        calib.append((codes, mean, x, N, K))
+    t0 = time.perf_counter()
+    for codes, mean, x, N, K in calib:
+        orc.ternary_linear(x, codes[:16], mean)
+    per_row_s = (time.perf_counter() - t0) / (16 * len(calib))
+    rows = max(1, int(per_step_s / (per_row_s * len(calib))))
+    sample = [(c[:min(rows, N)], m, x) for (c, m, x, N, K) in calib]
+    sample_w = sum(c.size for c, _, _ in sample)
+    for _ in range(args.warmup):
+        for c, m, x in sample:
+            orc.ternary_linear(x, c, m)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for c, m, x in sample:
+            orc.ternary_linear(x, c, m)
+    el = time.perf_counter() - t0
+    step_s = el / args.steps
+    value = M / (step_s * total_w / sample_w)
+    samp = (f"per step: first {rows} rows of each of layer 0's 7 projections "
+            f"({sample_w} weights, M={M}), scaled to the {len(shapes)}-projection sweep by "
+            f"weight count")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8xternary->int32, f32 in/out", "data": "synthetic",
+        "config": {"workload": f"decode_sweep_196x_M{M}", "M": M,
+                   "projections": len(shapes)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": samp},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    from ternary_weight_decoder_b200 import build
+    build.build()
+    from ternary_weight_decoder_b200 import api
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    M = args.m
+    shapes, descs, x_host, x_all, y_all = build_workload(api, torch, dev, M, args.layers, rank)
+    table = api.SweepTable(descs, M, device=dev)
+    algo_bytes, algo_codes, _ = sweep_bytes(shapes, M)
+    launches_per_step = 1 if M <= 8 else -(-M // 8)  # refined below from the library plan
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        api.decoder_projection_sweep(table)
+    api.check()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            api.decoder_projection_sweep(table)
+        e1.record(stream)
+        barrier()
+    api.check()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    tokens = M * world * args.steps
+    value = tokens / (ms / 1e3)
+
+    # dominant kernel: the sweep launch itself (one launch per step at M <= 8)
+    hbm, src = peaks()
+    achieved = algo_bytes / (ms_per_step / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": None,
+                "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured"
+                else "fallback 6650 GB/s",
+                "algorithmic_bytes_per_launch": algo_bytes,
+                "weight_bytes_per_launch": algo_codes,
+                "weight_gbs": algo_codes / (ms_per_step / 1e3) / 1e9}
+
+    e2e = None
+    if not args.no_e2e:
+        y_host = torch.empty(y_all.numel(), dtype=torch.float32).pin_memory()
+        k2 = max(3, min(args.steps, 2000))
+        for _ in range(3):
+            x_all.copy_(x_host, non_blocking=True)
+            api.decoder_projection_sweep(table)
+            y_host.copy_(y_all, non_blocking=True)
+            stream.synchronize()
+        barrier()
+        t0 = time.perf_counter()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(k2):
+            x_all.copy_(x_host, non_blocking=True)
+            api.decoder_projection_sweep(table)
+            y_host.copy_(y_all, non_blocking=True)
+            stream.synchronize()   # the host reads every step's result
+        f1.record(stream)
+        barrier()
+        wall = time.perf_counter() - t0
+        ems = f0.elapsed_time(f1)
+        if dist is not None:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": M * world * k2 / (ems / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": x_all.numel() * 4, "d2h_bytes_per_step": y_all.numel() * 4,
+               "steps": k2, "ms_per_step": ems / k2, "host_wall_ms_per_step": wall * 1e3 / k2}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_oracle_sample(M, layers=args.layers)
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8xternary->int32, f32 in/out", "data": "synthetic",
+        "config": {"workload": f"decode_sweep_196x_M{M}" if args.layers == 28
+                   else f"decode_sweep_{7 * args.layers}x_M{M}",
+                   "M": M, "projections": len(shapes), "layers": args.layers,
+                   "parallelism": f"dp{world} (independent replicas, no collective)",
+                   "l2": f"inputs {algo_bytes / 1e6:.0f} MB > 126 MB L2; no flush"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }))
+
+
+if __name__ == "__main__":
+    main()

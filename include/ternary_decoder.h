@@ -1,0 +1,223 @@
+/*
+ * ternary_decoder.h — C ABI of the B200 ternary-weight linear layer.
+ *
+ * The layer is the 1.58-bit ("BitNet") projection of the VibeVoice-ASR-BitNet
+ * LM decoder: every projection matrix W [N x K] is ternarised per tensor with
+ * s = 1/mean|W| to codes in {-1, 0, +1} ("VibeVoice-ASR-BitNet-ONNX" model
+ * page, "Quantization" table, row "LM projections (196 mats)"), activations
+ * are quantised per token to int8 by absmax, multiplied with the codes in
+ * integer arithmetic (ternary weights turn the multiply into add/subtract:
+ * xujun.org article, heterogeneous-quantisation section) and rescaled by
+ * absmax/127 and 1/s.  A Qwen2.5-1.5B-shaped decoder has 28 layers x 7
+ * projections = 196 such matrices (the same Quantization table).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Matrices are row-major.  W is [N x K] (PyTorch Linear layout), x is
+ *    [M x K], y = x W^T is [M x N].  Indices and sizes are int64_t.
+ *  - Unless stated otherwise every pointer is a DEVICE pointer to memory the
+ *    caller allocated and owns; the library allocates nothing that outlives a
+ *    call.  Scratch memory is passed in as `ws` of `ws_bytes`, sized by the
+ *    matching *_workspace_bytes query.
+ *  - Work is enqueued on the caller's stream and the call returns without
+ *    waiting.  Argument errors are detected on the host and returned at once;
+ *    errors found by a kernel (non-finite weights, a timed-out wait) are
+ *    recorded in a per-device error word and returned by tw_check().
+ *  - Every device pointer must be 16-byte aligned.  K must be a positive
+ *    multiple of 128 (the pages' ternary file format packs 128 weights per
+ *    unit: "The Paper Says ARM Support" post, "Postscript two").
+ *  - Return value: TW_OK or one of the TW_ERR_* codes; tw_last_error() gives
+ *    a message for the last failing call on the calling host thread.
+ *
+ * Packed code layout (this library's own design)
+ * ----------------------------------------------
+ * Codes are stored as c + 1 in {0, 1, 2} in two bits (pattern 3 is invalid),
+ * sixteen consecutive-k codes of one row per 32-bit word: the code of
+ * k0 + 4*s + b sits at bit 8*b + 2*s, so (word >> 2*s) & 0x03030303 yields
+ * four consecutive codes as bytes.  Rows are grouped in blocks of 16 (N is
+ * padded up to a multiple of 16 with code 0); a tile is 16 rows x 128 k =
+ * 512 bytes; tiles are stored row-block-major (all K/128 tiles of rows
+ * 16r..16r+15 are contiguous).  Inside a tile, 32-bit word 4*l + j (l = 4g + t,
+ * g in 0..7, t in 0..3, j in 0..3) holds row g + 8*(j & 1) and
+ * k = 64*(j >> 1) + 16*t .. +15, so each 16-byte lane slot of a tile is what
+ * one lane of a warp needs for two m16n8k32 integer MMA fragments.
+ */
+#ifndef TERNARY_DECODER_H
+#define TERNARY_DECODER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TW_API __attribute__((visibility("default")))
+#else
+#define TW_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream; identical to cudaStream_t.  NULL is the legacy default. */
+typedef struct CUstream_st *tw_stream_t;
+
+enum {
+    TW_OK = 0,
+    TW_ERR_NULL = 1,       /* a required pointer is NULL                    */
+    TW_ERR_SHAPE = 2,      /* N < 1, M < 1, K < 1, K % 128 != 0, or too big */
+    TW_ERR_ALIGN = 3,      /* a pointer is not 16-byte aligned              */
+    TW_ERR_BUFSIZE = 4,    /* a buffer or workspace is smaller than needed  */
+    TW_ERR_NONFINITE = 5,  /* W holds Inf or NaN (reported by tw_check)     */
+    TW_ERR_CUDA = 6,       /* a CUDA runtime call failed                    */
+    TW_ERR_TIMEOUT = 7,    /* a bounded device-side wait expired (tw_check) */
+    TW_ERR_CORRUPT = 8,    /* a table or packed buffer is malformed         */
+    TW_ERR_UNSUPPORTED = 9 /* no sm_100 device, or a mode not built         */
+};
+
+/* Bytes of packed codes for an [N x K] matrix: ceil(N/16)*16 * K / 4. */
+TW_API size_t tw_packed_bytes(int64_t N, int64_t K);
+
+/* Scratch needed by tw_ternarize_pack: one fp64 row sum per row plus a
+ * little header (8*N + 256 bytes, rounded up to 256). */
+TW_API size_t tw_ternarize_workspace_bytes(int64_t N, int64_t K);
+
+/*
+ * Ternarise W [N x K] fp32 per tensor and pack the codes.
+ * Defines: mean = sum|W| / (N*K) accumulated in fp64 in a fixed order (each
+ * row summed over k in order, then the row sums over n in order), floored at
+ * 1e-5; s = 1/mean; code = clip(rint(W * s), -1, 1) evaluated in fp64 with
+ * round-half-to-even.  ("VibeVoice-ASR-BitNet-ONNX" model page, Quantization
+ * table: per-tensor s = 1/mean|W|.)
+ *   W         [N x K] fp32, read only.
+ *   packed    output, packed_bytes >= tw_packed_bytes(N, K); layout above.
+ *   mean_abs  output, one double: mean|W| (= 1/s).  May be NULL.
+ *   wscale    output, one float: (float)mean, the per-tensor dequant factor
+ *             consumed by tw_ternary_linear.  Required.
+ *   ws        scratch of ws_bytes >= tw_ternarize_workspace_bytes(N, K).
+ * A non-finite W sets TW_ERR_NONFINITE in the device error word (the
+ * outputs are then unspecified).
+ */
+TW_API int tw_ternarize_pack(const float *W, int64_t N, int64_t K, void *packed,
+                      size_t packed_bytes, double *mean_abs, float *wscale,
+                      void *ws, size_t ws_bytes, tw_stream_t stream);
+
+/*
+ * Debug / parity: unpack codes to int8 {-1, 0, 1} row-major [N x K].
+ * invalid_count (device, one int32, may be NULL) receives the number of
+ * 2-bit fields holding the invalid pattern 3 (those codes are written as 0).
+ */
+TW_API int tw_unpack_codes(const void *packed, int64_t N, int64_t K, int8_t *codes,
+                    int32_t *invalid_count, tw_stream_t stream);
+
+/*
+ * Per-token int8 activation quantisation of x [M x K] fp32 by absmax.
+ *   amax[m]  = max_k |x[m,k]|                     (fp32, exact)
+ *   scale    = 127.0f / amax[m]                   (IEEE fp32 division)
+ *   xq[m,k]  = clamp(rint(x[m,k] * scale), -128, 127)   (fp32 multiply,
+ *              round-half-to-even); a row with amax == 0 gives xq == 0.
+ *   qsum[m]  = sum_k xq[m,k]  (optional, may be NULL; the prefill entry
+ *              points use it to fold the +1 code offset back out).
+ * The pages name only "fused INT8" operations (xujun.org article,
+ * heterogeneous-quantisation section); this is the plainest absmax reading.
+ * Non-finite x gives unspecified results.
+ */
+TW_API int tw_quantize_act(const float *x, int64_t M, int64_t K, int8_t *xq,
+                    float *amax, int32_t *qsum, tw_stream_t stream);
+
+/* Scratch needed by tw_ternary_linear / tw_ternary_linear_q for this shape
+ * (0 for the decode path M <= 32). */
+TW_API size_t tw_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * y = rescale(quantize(x) * codes^T): the whole layer on one matrix.
+ *   acc[m,n] = sum_k code[n,k] * xq[m,k]          (exact int32)
+ *   y[m,n]   = ((float)acc * (amax[m] / 127.0f)) * wscale   (fp32)
+ * x [M x K] fp32; packed/wscale from tw_ternarize_pack; y [M x N] fp32
+ * output; acc_out [M x N] int32 output or NULL.  M <= 32 runs the fused
+ * act-quant + decode kernel; larger M quantises into ws and runs the
+ * tensor-core prefill kernel.
+ */
+TW_API int tw_ternary_linear(const float *x, int64_t M, int64_t N, int64_t K,
+                      const void *packed, const float *wscale, float *y,
+                      int32_t *acc_out, void *ws, size_t ws_bytes,
+                      tw_stream_t stream);
+
+/*
+ * Same product on activations already quantised by tw_quantize_act:
+ * xq [M x K] int8, amax [M] fp32, qsum [M] int32 (required).
+ */
+TW_API int tw_ternary_linear_q(const int8_t *xq, const float *amax,
+                        const int32_t *qsum, int64_t M, int64_t N, int64_t K,
+                        const void *packed, const float *wscale, float *y,
+                        int32_t *acc_out, void *ws, size_t ws_bytes,
+                        tw_stream_t stream);
+
+/*
+ * One projection of a decoder sweep.  All pointers are device pointers.
+ * Decode sweeps (M <= 32) read x; prefill sweeps (M > 32) read xq, amax and
+ * qsum (from tw_quantize_act) and ignore x.
+ */
+typedef struct tw_proj_desc {
+    const float *x;        /* [M x K] fp32 activations (decode)            */
+    const int8_t *xq;      /* [M x K] int8 activations (prefill)           */
+    const float *amax;     /* [M] absmax that goes with xq (prefill)       */
+    const int32_t *qsum;   /* [M] row sums of xq (prefill)                 */
+    const void *packed;    /* packed codes of W [N x K]                    */
+    const float *wscale;   /* one float, mean|W|                           */
+    float *y;              /* [M x N] fp32 output                          */
+    int32_t *acc_out;      /* [M x N] int32 output, or NULL                */
+    int64_t N, K;
+} tw_proj_desc;
+
+/* Bytes of the encoded sweep table for `count` projections. */
+TW_API size_t tw_sweep_table_bytes(int count);
+
+/*
+ * HOST-ONLY.  Validate `count` descriptors (host array) for a sweep over M
+ * tokens and encode them into `table` (host memory, table_bytes >=
+ * tw_sweep_table_bytes(count)).  The caller copies the table to device
+ * memory (64-byte aligned) and passes that copy to
+ * tw_decoder_projection_sweep; the table stays valid for as long as the
+ * buffers it names do.  For M > 32 it embeds TMA descriptors of each xq and
+ * therefore needs the CUDA driver.
+ */
+TW_API int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M,
+                          void *table, size_t table_bytes);
+
+/* Scratch needed by tw_decoder_projection_sweep for an encoded HOST table. */
+TW_API size_t tw_sweep_workspace_bytes(const void *table_host);
+
+/*
+ * Run the layer over every projection of an encoded table: one persistent
+ * launch for decode (M <= 32; two or more only when M*K of the widest
+ * projection does not fit shared memory and the tokens are split into
+ * groups), one grouped tensor-core launch for prefill.
+ *   table_host  the host table written by tw_sweep_table_encode (read for the
+ *               launch configuration: count, M, sizes);
+ *   table_dev   the caller's device copy of the same bytes (64-byte aligned),
+ *               which the kernels read.
+ * The 196 projections of the synthetic decoder sweep share no data: each
+ * has its own x and y.
+ */
+TW_API int tw_decoder_projection_sweep(const void *table_host, const void *table_dev,
+                                void *ws, size_t ws_bytes, tw_stream_t stream);
+
+/* Wait for `stream`, then return and clear the device error word of the
+ * current device (TW_OK if no kernel reported an error). */
+TW_API int tw_check(tw_stream_t stream);
+
+/* Message of the last failing call on this host thread ("" if none). */
+TW_API const char *tw_last_error(void);
+
+/*
+ * Self-test of the bounded-wait machinery: launch one block that waits on a
+ * barrier nothing ever completes, giving up after timeout_ns; the kernel
+ * then records TW_ERR_TIMEOUT, which tw_check() returns.  Faults nothing.
+ */
+TW_API int tw_debug_wait_timeout(uint64_t timeout_ns, tw_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TERNARY_DECODER_H */

@@ -1,0 +1,221 @@
+"""Thin Python binding of ``libternary_decoder.so`` (argument marshalling only).
+
+Every function here checks tensor properties, passes raw pointers and the
+current CUDA stream to the C entry point of the same name (``tw_`` prefix in
+C) and raises ``TernaryError`` on a non-zero status.  All arithmetic runs in
+the library's CUDA kernels; there is no fallback: importing this module
+fails loudly when the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libternary_decoder.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m ternary_weight_decoder_b200.build` "
+        "(or __graft_entry__.build()); there is no CPU fallback")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+TW_OK = 0
+STATUS = {0: "TW_OK", 1: "TW_ERR_NULL", 2: "TW_ERR_SHAPE", 3: "TW_ERR_ALIGN",
+          4: "TW_ERR_BUFSIZE", 5: "TW_ERR_NONFINITE", 6: "TW_ERR_CUDA",
+          7: "TW_ERR_TIMEOUT", 8: "TW_ERR_CORRUPT", 9: "TW_ERR_UNSUPPORTED"}
+
+
+class TernaryError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+_i64, _sz, _p, _int = ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int
+
+
+def _sig(name, res, args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = args
+    return f
+
+
+tw_packed_bytes = _sig("tw_packed_bytes", _sz, [_i64, _i64])
+tw_ternarize_workspace_bytes = _sig("tw_ternarize_workspace_bytes", _sz, [_i64, _i64])
+tw_ternarize_pack = _sig("tw_ternarize_pack", _int,
+                         [_p, _i64, _i64, _p, _sz, _p, _p, _p, _sz, _p])
+tw_unpack_codes = _sig("tw_unpack_codes", _int, [_p, _i64, _i64, _p, _p, _p])
+tw_quantize_act = _sig("tw_quantize_act", _int, [_p, _i64, _i64, _p, _p, _p, _p])
+tw_linear_workspace_bytes = _sig("tw_linear_workspace_bytes", _sz, [_i64, _i64, _i64])
+tw_ternary_linear = _sig("tw_ternary_linear", _int,
+                         [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p, _sz, _p])
+tw_ternary_linear_q = _sig("tw_ternary_linear_q", _int,
+                           [_p, _p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p, _sz, _p])
+tw_sweep_table_bytes = _sig("tw_sweep_table_bytes", _sz, [_int])
+tw_sweep_table_encode = _sig("tw_sweep_table_encode", _int, [_p, _int, _i64, _p, _sz])
+tw_sweep_workspace_bytes = _sig("tw_sweep_workspace_bytes", _sz, [_p])
+tw_decoder_projection_sweep = _sig("tw_decoder_projection_sweep", _int, [_p, _p, _p, _sz, _p])
+tw_check = _sig("tw_check", _int, [_p])
+tw_last_error = _sig("tw_last_error", ctypes.c_char_p, [])
+tw_debug_wait_timeout = _sig("tw_debug_wait_timeout", _int, [ctypes.c_uint64, _p])
+
+
+class ProjDesc(ctypes.Structure):
+    """Mirror of ``tw_proj_desc``."""
+    _fields_ = [("x", _p), ("xq", _p), ("amax", _p), ("qsum", _p), ("packed", _p),
+                ("wscale", _p), ("y", _p), ("acc_out", _p), ("N", _i64), ("K", _i64)]
+
+
+def _raise(status: int):
+    if status != TW_OK:
+        raise TernaryError(status, tw_last_error().decode(errors="replace"))
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, name, device=True):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def check(stream=None):
+    """Synchronise and raise if a kernel recorded an error."""
+    _raise(tw_check(_stream(stream)))
+
+
+def packed_bytes(N: int, K: int) -> int:
+    return int(tw_packed_bytes(N, K))
+
+
+def ternarize_pack(W: torch.Tensor, stream=None):
+    """W [N, K] fp32 (CUDA) -> (packed uint8, mean_abs float64[1], wscale float32[1])."""
+    _need(W, torch.float32, "W")
+    N, K = W.shape
+    dev = W.device
+    packed = torch.empty(max(packed_bytes(N, K), 16), dtype=torch.uint8, device=dev)
+    mean_abs = torch.empty(2, dtype=torch.float64, device=dev)
+    wscale = torch.empty(4, dtype=torch.float32, device=dev)
+    wsb = int(tw_ternarize_workspace_bytes(N, K))
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    _raise(tw_ternarize_pack(_ptr(W), N, K, _ptr(packed), packed.numel(), _ptr(mean_abs),
+                             _ptr(wscale), _ptr(ws), wsb, _stream(stream)))
+    return packed, mean_abs[:1], wscale[:1]
+
+
+def unpack_codes(packed: torch.Tensor, N: int, K: int, stream=None):
+    """-> (codes int8 [N, K], invalid_count int32[1])."""
+    _need(packed, torch.uint8, "packed")
+    codes = torch.empty((N, K), dtype=torch.int8, device=packed.device)
+    invalid = torch.zeros(4, dtype=torch.int32, device=packed.device)
+    _raise(tw_unpack_codes(_ptr(packed), N, K, _ptr(codes), _ptr(invalid), _stream(stream)))
+    return codes, invalid[:1]
+
+
+def quantize_act(x: torch.Tensor, stream=None):
+    """x [M, K] fp32 -> (xq int8 [M, K], amax fp32 [M], qsum int32 [M])."""
+    _need(x, torch.float32, "x")
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    amax = torch.empty(M, dtype=torch.float32, device=x.device)
+    qsum = torch.empty(M, dtype=torch.int32, device=x.device)
+    _raise(tw_quantize_act(_ptr(x), M, K, _ptr(xq), _ptr(amax), _ptr(qsum), _stream(stream)))
+    return xq, amax, qsum
+
+
+def linear_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(tw_linear_workspace_bytes(M, N, K))
+
+
+def ternary_linear(x: torch.Tensor, packed: torch.Tensor, wscale: torch.Tensor, N: int,
+                   y: torch.Tensor | None = None, acc_out: torch.Tensor | None = None,
+                   ws: torch.Tensor | None = None, stream=None):
+    """y [M, N] fp32 = the ternary layer on x [M, K] fp32; acc_out optional int32 [M, N]."""
+    _need(x, torch.float32, "x")
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    wsb = linear_workspace_bytes(M, N, K)
+    if ws is None and wsb:
+        ws = torch.empty(wsb, dtype=torch.uint8, device=x.device)
+    _raise(tw_ternary_linear(_ptr(x), M, N, K, _ptr(packed), _ptr(wscale), _ptr(y),
+                             _ptr(acc_out), _ptr(ws), ws.numel() if ws is not None else 0,
+                             _stream(stream)))
+    return y
+
+
+def ternary_linear_q(xq, amax, qsum, packed, wscale, N: int, y=None, acc_out=None, ws=None,
+                     stream=None):
+    """y [M, N] fp32 from pre-quantised xq [M, K] int8, amax [M], qsum [M]."""
+    _need(xq, torch.int8, "xq")
+    M, K = xq.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=xq.device)
+    wsb = linear_workspace_bytes(M, N, K)
+    if ws is None and wsb:
+        ws = torch.empty(wsb, dtype=torch.uint8, device=xq.device)
+    _raise(tw_ternary_linear_q(_ptr(xq), _ptr(amax), _ptr(qsum), M, N, K, _ptr(packed),
+                               _ptr(wscale), _ptr(y), _ptr(acc_out), _ptr(ws),
+                               ws.numel() if ws is not None else 0, _stream(stream)))
+    return y
+
+
+def _dp(d, key):
+    """Device address of d[key]: a tensor, a raw int address, or None."""
+    v = d.get(key)
+    if v is None:
+        return None
+    return v if isinstance(v, int) else v.data_ptr()
+
+
+class SweepTable:
+    """An encoded sweep over many projections: the host bytes written by
+    ``tw_sweep_table_encode`` and their device copy.  Keep the tensors named
+    by the descriptors alive for as long as the table is used."""
+
+    def __init__(self, descs: Sequence[dict], M: int, device=None):
+        n = len(descs)
+        arr = (ProjDesc * n)()
+        for i, d in enumerate(descs):
+            arr[i] = ProjDesc(
+                x=_dp(d, "x"), xq=_dp(d, "xq"), amax=_dp(d, "amax"), qsum=_dp(d, "qsum"),
+                packed=_dp(d, "packed"), wscale=_dp(d, "wscale"), y=_dp(d, "y"),
+                acc_out=_dp(d, "acc_out"), N=int(d["N"]), K=int(d["K"]))
+        nbytes = int(tw_sweep_table_bytes(n))
+        self.host = torch.empty(nbytes, dtype=torch.uint8).pin_memory() \
+            if torch.cuda.is_available() else torch.empty(nbytes, dtype=torch.uint8)
+        _raise(tw_sweep_table_encode(arr, n, M, _ptr(self.host), nbytes))
+        self.count, self.M = n, M
+        self.device = None
+        if device is not None:
+            self.device = self.host.to(device, non_blocking=False)
+        wsb = int(tw_sweep_workspace_bytes(_ptr(self.host)))
+        self.ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=device) \
+            if device is not None else None
+        self.ws_bytes = wsb
+
+
+def decoder_projection_sweep(table: SweepTable, stream=None):
+    """Run every projection of ``table`` (one persistent launch for decode)."""
+    _raise(tw_decoder_projection_sweep(_ptr(table.host), _ptr(table.device), _ptr(table.ws),
+                                       table.ws_bytes, _stream(stream)))
+
+
+def debug_wait_timeout(timeout_ns: int, stream=None):
+    _raise(tw_debug_wait_timeout(timeout_ns, _stream(stream)))

@@ -1,0 +1,365 @@
+// tw_api.cu — the C ABI: argument checks, status codes, the per-device error
+// word, sweep-table encoding and dispatch to the kernel families.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "tw_device.cuh"
+#include "tw_internal.h"
+
+namespace {
+
+__device__ uint32_t g_tw_err;  // per-device error word (EFLAG_* bits)
+
+thread_local char t_last_error[512] = "";
+constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s limit of an ordinary wait
+
+int fail(int code, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(TW_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Address of g_tw_err on the current device (looked up once per device).
+int err_word(uint32_t **out)
+{
+    static std::mutex mu;
+    static uint32_t *cache[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64)
+        return fail(TW_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lk(mu);
+    if (!cache[dev]) {
+        int major = 0;
+        e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        if (major != 10)
+            return fail(TW_ERR_UNSUPPORTED, "device %d is sm_%d0, this library is built for sm_100a",
+                        dev, major);
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_tw_err);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+        cache[dev] = static_cast<uint32_t *>(p);
+    }
+    *out = cache[dev];
+    return TW_OK;
+}
+
+int check_shape(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 1 || N < 1 || K < 1)
+        return fail(TW_ERR_SHAPE, "shape M=%lld N=%lld K=%lld: all must be >= 1", (long long)M,
+                    (long long)N, (long long)K);
+    if (K % tw::kTileK)
+        return fail(TW_ERR_SHAPE, "K=%lld is not a multiple of 128", (long long)K);
+    if (N > (1 << 24) || K > (1 << 24) || M > (1 << 24))
+        return fail(TW_ERR_SHAPE, "shape M=%lld N=%lld K=%lld exceeds 2^24", (long long)M,
+                    (long long)N, (long long)K);
+    return TW_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t tw_packed_bytes(int64_t N, int64_t K)
+{
+    if (N < 1 || K < 1)
+        return 0;
+    return (size_t)(tw::ceil_div(N, tw::kTileRows) * tw::kTileRows) * (size_t)K / 4;
+}
+
+size_t tw_ternarize_workspace_bytes(int64_t N, int64_t K)
+{
+    (void)K;
+    if (N < 1)
+        return 0;
+    return (size_t)((256 + 8 * N + 255) / 256 * 256);
+}
+
+const char *tw_last_error(void) { return t_last_error; }
+
+int tw_ternarize_pack(const float *W, int64_t N, int64_t K, void *packed, size_t packed_bytes,
+                      double *mean_abs, float *wscale, void *ws, size_t ws_bytes,
+                      tw_stream_t stream)
+{
+    t_last_error[0] = 0;
+    if (!W || !packed || !wscale || !ws)
+        return fail(TW_ERR_NULL, "tw_ternarize_pack: W, packed, wscale and ws are required");
+    if (int rc = check_shape(1, N, K))
+        return rc;
+    if (!aligned16(W) || !aligned16(packed) || !aligned16(ws) || !aligned16(wscale) ||
+        (mean_abs && !aligned16(mean_abs)))
+        return fail(TW_ERR_ALIGN, "tw_ternarize_pack: pointers must be 16-byte aligned");
+    if (packed_bytes < tw_packed_bytes(N, K))
+        return fail(TW_ERR_BUFSIZE, "packed buffer %zu < %zu bytes", packed_bytes,
+                    tw_packed_bytes(N, K));
+    if (ws_bytes < tw_ternarize_workspace_bytes(N, K))
+        return fail(TW_ERR_BUFSIZE, "workspace %zu < %zu bytes", ws_bytes,
+                    tw_ternarize_workspace_bytes(N, K));
+    uint32_t *err = nullptr;
+    if (int rc = err_word(&err))
+        return rc;
+    cudaError_t e = tw::launch_ternarize(W, N, K, static_cast<uint8_t *>(packed), mean_abs,
+                                         wscale, ws, err, stream);
+    return e == cudaSuccess ? TW_OK : cuda_fail(e, "ternarize launch");
+}
+
+int tw_unpack_codes(const void *packed, int64_t N, int64_t K, int8_t *codes,
+                    int32_t *invalid_count, tw_stream_t stream)
+{
+    t_last_error[0] = 0;
+    if (!packed || !codes)
+        return fail(TW_ERR_NULL, "tw_unpack_codes: packed and codes are required");
+    if (int rc = check_shape(1, N, K))
+        return rc;
+    if (!aligned16(packed) || !aligned16(codes) || (invalid_count && !aligned16(invalid_count)))
+        return fail(TW_ERR_ALIGN, "tw_unpack_codes: pointers must be 16-byte aligned");
+    uint32_t *err = nullptr;
+    if (int rc = err_word(&err))
+        return rc;
+    cudaError_t e = tw::launch_unpack(static_cast<const uint8_t *>(packed), N, K, codes,
+                                      invalid_count, stream);
+    return e == cudaSuccess ? TW_OK : cuda_fail(e, "unpack launch");
+}
+
+int tw_quantize_act(const float *x, int64_t M, int64_t K, int8_t *xq, float *amax, int32_t *qsum,
+                    tw_stream_t stream)
+{
+    t_last_error[0] = 0;
+    if (!x || !xq || !amax)
+        return fail(TW_ERR_NULL, "tw_quantize_act: x, xq and amax are required");
+    if (int rc = check_shape(M, 1, K))
+        return rc;
+    if (!aligned16(x) || !aligned16(xq) || !aligned16(amax) || (qsum && !aligned16(qsum)))
+        return fail(TW_ERR_ALIGN, "tw_quantize_act: pointers must be 16-byte aligned");
+    uint32_t *err = nullptr;
+    if (int rc = err_word(&err))
+        return rc;
+    cudaError_t e = tw::launch_quantize(x, M, K, xq, amax, qsum, stream);
+    return e == cudaSuccess ? TW_OK : cuda_fail(e, "quantize launch");
+}
+
+size_t tw_linear_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    (void)N;
+    if (M <= tw::kDecodeMaxM)
+        return 0;
+    const size_t xq = (size_t)((M * K + 255) / 256 * 256);
+    const size_t vec = (size_t)((M * 4 + 255) / 256 * 256);
+    return xq + 2 * vec + 256;
+}
+
+int tw_ternary_linear(const float *x, int64_t M, int64_t N, int64_t K, const void *packed,
+                      const float *wscale, float *y, int32_t *acc_out, void *ws, size_t ws_bytes,
+                      tw_stream_t stream)
+{
+    t_last_error[0] = 0;
+    if (!x || !packed || !wscale || !y)
+        return fail(TW_ERR_NULL, "tw_ternary_linear: x, packed, wscale and y are required");
+    if (int rc = check_shape(M, N, K))
+        return rc;
+    if (!aligned16(x) || !aligned16(packed) || !aligned16(wscale) || !aligned16(y) ||
+        (acc_out && !aligned16(acc_out)))
+        return fail(TW_ERR_ALIGN, "tw_ternary_linear: pointers must be 16-byte aligned");
+    if (ws_bytes < tw_linear_workspace_bytes(M, N, K) || (ws_bytes && !ws))
+        return fail(TW_ERR_BUFSIZE, "workspace %zu < %zu bytes", ws_bytes,
+                    tw_linear_workspace_bytes(M, N, K));
+    uint32_t *err = nullptr;
+    if (int rc = err_word(&err))
+        return rc;
+    if (M <= tw::kDecodeMaxM) {
+        if (K > tw::kDecodeMaxK)
+            return fail(TW_ERR_SHAPE, "decode path supports K <= %lld", (long long)tw::kDecodeMaxK);
+        tw::DescRecord r;
+        memset(&r, 0, sizeof(r));
+        r.x = x;
+        r.packed = static_cast<const uint8_t *>(packed);
+        r.wscale = wscale;
+        r.y = y;
+        r.acc_out = acc_out;
+        r.N = N;
+        r.K = K;
+        tw::DecodeLaunch L{};
+        L.table = nullptr;
+        L.single = &r;
+        L.count = 1;
+        L.M = M;
+        L.total_rb = tw::ceil_div(N, tw::kTileRows);
+        L.total_tiles = L.total_rb * (K / tw::kTileK);
+        L.max_K = K;
+        cudaError_t e = tw::launch_decode(L, err, kWaitNs, stream);
+        return e == cudaSuccess ? TW_OK : cuda_fail(e, "decode launch");
+    }
+    return fail(TW_ERR_UNSUPPORTED, "prefill path (M > 32) is not built yet");
+}
+
+int tw_ternary_linear_q(const int8_t *xq, const float *amax, const int32_t *qsum, int64_t M,
+                        int64_t N, int64_t K, const void *packed, const float *wscale, float *y,
+                        int32_t *acc_out, void *ws, size_t ws_bytes, tw_stream_t stream)
+{
+    t_last_error[0] = 0;
+    (void)xq; (void)amax; (void)qsum; (void)M; (void)N; (void)K; (void)packed; (void)wscale;
+    (void)y; (void)acc_out; (void)ws; (void)ws_bytes; (void)stream;
+    return fail(TW_ERR_UNSUPPORTED, "prefill path (M > 32) is not built yet");
+}
+
+size_t tw_sweep_table_bytes(int count)
+{
+    if (count < 1)
+        return 0;
+    return sizeof(tw::TableHeader) + (size_t)count * sizeof(tw::DescRecord);
+}
+
+int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void *table,
+                          size_t table_bytes)
+{
+    t_last_error[0] = 0;
+    if (!descs || !table)
+        return fail(TW_ERR_NULL, "tw_sweep_table_encode: descs and table are required");
+    if (count < 1)
+        return fail(TW_ERR_SHAPE, "count=%d must be >= 1", count);
+    if (table_bytes < tw_sweep_table_bytes(count))
+        return fail(TW_ERR_BUFSIZE, "table buffer %zu < %zu bytes", table_bytes,
+                    tw_sweep_table_bytes(count));
+    if (M < 1 || M > (1 << 24))
+        return fail(TW_ERR_SHAPE, "M=%lld out of range", (long long)M);
+    const bool decode = M <= tw::kDecodeMaxM;
+    if (!decode)
+        return fail(TW_ERR_UNSUPPORTED, "prefill sweep (M > 32) is not built yet");
+    auto *hdr = static_cast<tw::TableHeader *>(table);
+    auto *recs = reinterpret_cast<tw::DescRecord *>(hdr + 1);
+    memset(table, 0, tw_sweep_table_bytes(count));
+    int64_t rb = 0, tiles = 0, max_K = 0, sum_K = 0;
+    for (int d = 0; d < count; ++d) {
+        const tw_proj_desc &s = descs[d];
+        if (int rc = check_shape(M, s.N, s.K))
+            return fail(rc, "descriptor %d: %s", d, t_last_error);
+        if (decode && s.K > tw::kDecodeMaxK)
+            return fail(TW_ERR_SHAPE, "descriptor %d: decode path supports K <= %lld", d,
+                        (long long)tw::kDecodeMaxK);
+        if (!s.packed || !s.wscale || !s.y || (decode && !s.x))
+            return fail(TW_ERR_NULL, "descriptor %d: x, packed, wscale and y are required", d);
+        if (!aligned16(s.packed) || !aligned16(s.wscale) || !aligned16(s.y) ||
+            (s.x && !aligned16(s.x)) || (s.acc_out && !aligned16(s.acc_out)))
+            return fail(TW_ERR_ALIGN, "descriptor %d: pointers must be 16-byte aligned", d);
+        tw::DescRecord &r = recs[d];
+        r.x = s.x;
+        r.xq = s.xq;
+        r.amax = s.amax;
+        r.qsum = s.qsum;
+        r.packed = static_cast<const uint8_t *>(s.packed);
+        r.wscale = s.wscale;
+        r.y = s.y;
+        r.acc_out = s.acc_out;
+        r.N = s.N;
+        r.K = s.K;
+        r.rb_begin = rb;
+        r.tile_begin = tiles;
+        const int64_t nrb = tw::ceil_div(s.N, tw::kTileRows);
+        rb += nrb;
+        tiles += nrb * (s.K / tw::kTileK);
+        max_K = s.K > max_K ? s.K : max_K;
+        sum_K += s.K;
+    }
+    hdr->magic = tw::kTableMagic;
+    hdr->count = count;
+    hdr->M = M;
+    hdr->total_rb = rb;
+    hdr->total_tiles = tiles;
+    hdr->max_K = max_K;
+    hdr->sum_K = sum_K;
+    return TW_OK;
+}
+
+size_t tw_sweep_workspace_bytes(const void *table_host)
+{
+    (void)table_host;
+    return 0;
+}
+
+int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, void *ws,
+                                size_t ws_bytes, tw_stream_t stream)
+{
+    t_last_error[0] = 0;
+    (void)ws;
+    (void)ws_bytes;
+    if (!table_host || !table_dev)
+        return fail(TW_ERR_NULL, "tw_decoder_projection_sweep: host and device tables required");
+    if ((reinterpret_cast<uintptr_t>(table_dev) & 63u) != 0)
+        return fail(TW_ERR_ALIGN, "device table must be 64-byte aligned");
+    const auto *hdr = static_cast<const tw::TableHeader *>(table_host);
+    if (hdr->magic != tw::kTableMagic || hdr->count < 1)
+        return fail(TW_ERR_CORRUPT, "host table was not produced by tw_sweep_table_encode");
+    uint32_t *err = nullptr;
+    if (int rc = err_word(&err))
+        return rc;
+    if (hdr->M > tw::kDecodeMaxM)
+        return fail(TW_ERR_UNSUPPORTED, "prefill sweep (M > 32) is not built yet");
+    tw::DecodeLaunch L{};
+    L.table = reinterpret_cast<const tw::DescRecord *>(
+        static_cast<const tw::TableHeader *>(table_dev) + 1);
+    L.single = nullptr;
+    L.count = hdr->count;
+    L.M = hdr->M;
+    L.total_rb = hdr->total_rb;
+    L.total_tiles = hdr->total_tiles;
+    L.max_K = hdr->max_K;
+    cudaError_t e = tw::launch_decode(L, err, kWaitNs, stream);
+    return e == cudaSuccess ? TW_OK : cuda_fail(e, "sweep launch");
+}
+
+int tw_check(tw_stream_t stream)
+{
+    t_last_error[0] = 0;
+    uint32_t *err = nullptr;
+    if (int rc = err_word(&err))
+        return rc;
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaStreamSynchronize");
+    uint32_t v = 0;
+    e = cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "reading the error word");
+    if (!v)
+        return TW_OK;
+    const uint32_t zero = 0;
+    e = cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "clearing the error word");
+    if (v & tw::EFLAG_TIMEOUT)
+        return fail(TW_ERR_TIMEOUT, "a device-side wait timed out (error word 0x%x)", v);
+    if (v & tw::EFLAG_NONFINITE)
+        return fail(TW_ERR_NONFINITE, "non-finite weight found (error word 0x%x)", v);
+    return fail(TW_ERR_CORRUPT, "kernel reported a malformed descriptor (error word 0x%x)", v);
+}
+
+int tw_debug_wait_timeout(uint64_t timeout_ns, tw_stream_t stream)
+{
+    t_last_error[0] = 0;
+    uint32_t *err = nullptr;
+    if (int rc = err_word(&err))
+        return rc;
+    cudaError_t e = tw::launch_wait_probe(err, timeout_ns, stream);
+    return e == cudaSuccess ? TW_OK : cuda_fail(e, "wait probe launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,257 @@
+"""Parity of the CUDA path (through the C ABI) with the reference oracle.
+
+Codes, packed bytes, int8 activations, amax, sum(q) and int32 accumulators
+must be bit-exact; fp32 outputs within 1e-6 relative of the fp64 oracle.
+Sizes span several tiles plus ragged tails; every output buffer is poisoned
+before the call so an unwritten element shows up (the NaN fingerprint of a
+missing remainder-row path, "The Paper Says ARM Support" post, round three).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import oracle as orc
+from tests import gpu_util as G
+from tests.conftest import ROOT
+from ternary_weight_decoder_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+POISON_I32 = np.int32(-2**31)
+
+
+@pytest.fixture(scope="module")
+def dev():
+    return G.torch_dev()
+
+
+@pytest.fixture(scope="module")
+def api():
+    return G.api()
+
+
+def _weights(N, K, seed, sigma=0.02):
+    return synth.weights(seed, 17, N, K, sigma)
+
+
+def _acts(M, K, seed, outliers=True):
+    return synth.activations(seed, 23, M, K, outliers)
+
+
+# ------------------------------------------------------------ ternarise
+@pytest.mark.parametrize("N,K", [(16, 128), (37, 256), (256, 1536), (1536, 1536),
+                                 (100, 8960), (1, 128)])
+def test_ternarize_pack_bit_exact(dev, api, N, K):
+    W = _weights(N, K, N + K)
+    packed, mean_abs, wscale = G.ternarize_gpu(W, dev)
+    codes, _ = G.check_packed_against_oracle(W, packed, mean_abs, wscale, N, K)
+    got, invalid = api.unpack_codes(packed, N, K)
+    api.check()
+    assert (got.cpu().numpy() == codes).all()
+    assert int(invalid.cpu()[0]) == 0
+
+
+def test_ternarize_hand_case(dev, api, golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "hand_4x8.json")))
+    W = np.tile(np.array(g["W"], np.float32), (1, 16))          # K = 128, mean unchanged
+    packed, mean_abs, wscale = G.ternarize_gpu(W, dev)
+    assert float(mean_abs.cpu()[0]) == g["mean_abs"]
+    codes, _ = api.unpack_codes(packed, 4, 128)
+    assert (codes.cpu().numpy() == np.tile(np.array(g["codes"], np.int8), (1, 16))).all()
+    x = np.tile(np.array(g["x"], np.float32), (1, 16))
+    acc = G.to_dev(np.full((1, 4), POISON_I32), dev)
+    y = api.ternary_linear(G.to_dev(x, dev), packed, wscale, 4, acc_out=acc)
+    api.check()
+    assert acc.cpu().numpy().tolist() == [[16 * v for v in g["acc"][0]]]
+    assert y.cpu().numpy().tolist() == [[16.0 * v for v in g["y"][0]]]
+
+
+def test_ternarize_zero_weights(dev, api):
+    W = np.zeros((20, 256), np.float32)
+    packed, mean_abs, wscale = G.ternarize_gpu(W, dev)
+    assert float(mean_abs.cpu()[0]) == 1e-5
+    codes, _ = api.unpack_codes(packed, 20, 256)
+    assert not codes.cpu().numpy().any()
+    y = api.ternary_linear(G.to_dev(_acts(3, 256, 1), dev), packed, wscale, 20)
+    api.check()
+    assert not y.cpu().numpy().any()
+
+
+def test_ternarize_nonfinite_reported(dev, api):
+    W = _weights(16, 128, 5)
+    W[3, 7] = np.inf
+    api.ternarize_pack(G.to_dev(W, dev))
+    with pytest.raises(api.TernaryError) as e:
+        api.check()
+    assert e.value.status == 5
+    api.check()  # the error word was cleared
+
+
+# ------------------------------------------------------------ act quant
+@pytest.mark.parametrize("M,K", [(1, 1536), (5, 8960), (33, 128), (300, 256)])
+def test_quantize_act_bit_exact(dev, api, M, K):
+    x = _acts(M, K, M * 7 + K)
+    x[min(2, M - 1)] = 0.0  # an all-zero token
+    xq, amax, qsum = api.quantize_act(G.to_dev(x, dev))
+    api.check()
+    q, a = orc.quantize_act(x)
+    assert (xq.cpu().numpy() == q).all()
+    assert (amax.cpu().numpy() == a).all()
+    assert (qsum.cpu().numpy() == q.astype(np.int64).sum(axis=1)).all()
+
+
+# ------------------------------------------------------------ decode linear
+def _run_linear(api, dev, W, x, N):
+    import torch
+    packed, mean_abs, wscale = G.ternarize_gpu(W, dev)
+    M = x.shape[0]
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+    acc = torch.full((M, N), int(POISON_I32), dtype=torch.int32, device=dev)
+    api.ternary_linear(G.to_dev(x, dev), packed, wscale, N, y=y, acc_out=acc)
+    api.check()
+    return y.cpu().numpy(), acc.cpu().numpy()
+
+
+@pytest.mark.parametrize("M", list(range(1, 34)))
+def test_decode_linear_m_tails(dev, api, M):
+    if M > 32:
+        pytest.skip("M > 32 is the prefill path")
+    N, K = 80, 640   # 5 row blocks, 5 k tiles (a partial 8-tile chunk)
+    W = _weights(N, K, 100 + M)
+    x = _acts(M, K, 200 + M)
+    y, acc = _run_linear(api, dev, W, x, N)
+    codes, mean = orc.ternarize(W)
+    ref = orc.ternary_linear(x, codes, mean)
+    assert (acc == ref["acc"]).all()
+    G.assert_y_close(y, ref["y"], f"M={M}")
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1536, 1536), (1, 256, 1536), (1, 1536, 8960),
+                                   (4, 8960, 1536), (8, 37, 1152), (16, 1536, 8960),
+                                   (32, 1536, 8960), (32, 300, 1536), (3, 1, 128)])
+def test_decode_linear_shapes(dev, api, M, N, K):
+    W = _weights(N, K, M + N + K)
+    x = _acts(M, K, M * 3 + K)
+    y, acc = _run_linear(api, dev, W, x, N)
+    codes, mean = orc.ternarize(W)
+    ref = orc.ternary_linear(x, codes, mean)
+    assert (acc == ref["acc"]).all()
+    G.assert_y_close(y, ref["y"], f"{M}x{N}x{K}")
+
+
+def test_decode_zero_token_row(dev, api):
+    N, K = 64, 256
+    W = _weights(N, K, 9)
+    x = _acts(3, K, 9)
+    x[1] = 0.0
+    y, acc = _run_linear(api, dev, W, x, N)
+    assert not acc[1].any() and not y[1].any()
+
+
+def test_decode_k_permutation_detector(dev, api):
+    """A joint permutation of K leaves acc unchanged; swapping the two
+    64-halves of every 128-block of W alone changes it (a 64-vs-128 block
+    mis-read, "The Paper Says ARM Support" post, postscript two)."""
+    N, K, M = 48, 512, 4
+    W = _weights(N, K, 31)
+    x = _acts(M, K, 32)
+    _, acc = _run_linear(api, dev, W, x, N)
+    perm = np.random.default_rng(0).permutation(K)
+    _, acc_p = _run_linear(api, dev, np.ascontiguousarray(W[:, perm]),
+                           np.ascontiguousarray(x[:, perm]), N)
+    assert (acc_p == acc).all()
+    blk = np.arange(K).reshape(-1, 2, 64)[:, ::-1, :].ravel()
+    _, acc_s = _run_linear(api, dev, np.ascontiguousarray(W[:, blk]), x, N)
+    assert (acc_s != acc).any()
+
+
+# ------------------------------------------------------------ sweep
+def _sweep_case(api, dev, layers, M, seed_base=0):
+    import torch
+    descs, keep, refs = [], [], []
+    for (l, p, name, N, K) in synth.sweep_shapes(layers):
+        W = synth.weights(l + seed_base, p, N, K)
+        x = synth.activations(l + seed_base, p, M, K)
+        packed, mean_abs, wscale = G.ternarize_gpu(W, dev)
+        xd = G.to_dev(x, dev)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+        acc = torch.full((M, N), int(POISON_I32), dtype=torch.int32, device=dev)
+        descs.append(dict(x=xd, packed=packed, wscale=wscale, y=y, acc_out=acc, N=N, K=K))
+        keep.append((W, x))
+    table = api.SweepTable(descs, M, device=dev)
+    api.decoder_projection_sweep(table)
+    api.check()
+    return descs, keep
+
+
+@pytest.mark.parametrize("M", [1, 4, 8, 16, 32])
+def test_sweep_one_layer(dev, api, M):
+    descs, keep = _sweep_case(api, dev, 1, M, seed_base=M)
+    for d, (W, x) in zip(descs, keep):
+        codes, mean = orc.ternarize(W)
+        ref = orc.ternary_linear(x, codes, mean)
+        assert (d["acc_out"].cpu().numpy() == ref["acc"]).all(), (M, d["N"], d["K"])
+        G.assert_y_close(d["y"].cpu().numpy(), ref["y"], f"M={M} N={d['N']} K={d['K']}")
+
+
+def test_sweep_two_layers_m1(dev, api):
+    descs, keep = _sweep_case(api, dev, 2, 1, seed_base=50)
+    for d, (W, x) in zip(descs, keep):
+        codes, mean = orc.ternarize(W)
+        ref = orc.ternary_linear(x, codes, mean)
+        assert (d["acc_out"].cpu().numpy() == ref["acc"]).all()
+        G.assert_y_close(d["y"].cpu().numpy(), ref["y"])
+
+
+def test_sweep_ragged_small_projections(dev, api):
+    """Many tiny projections (fewer row blocks than CTAs, ragged N)."""
+    import torch
+    M = 3
+    rng = np.random.default_rng(5)
+    shapes = [(int(rng.integers(1, 70)), 128 * int(rng.integers(1, 6))) for _ in range(40)]
+    descs, keep = [], []
+    for i, (N, K) in enumerate(shapes):
+        W = _weights(N, K, 1000 + i)
+        x = _acts(M, K, 2000 + i)
+        packed, _, wscale = G.ternarize_gpu(W, dev)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+        acc = torch.full((M, N), int(POISON_I32), dtype=torch.int32, device=dev)
+        descs.append(dict(x=G.to_dev(x, dev), packed=packed, wscale=wscale, y=y, acc_out=acc,
+                          N=N, K=K))
+        keep.append((W, x))
+    table = api.SweepTable(descs, M, device=dev)
+    api.decoder_projection_sweep(table)
+    api.check()
+    for d, (W, x) in zip(descs, keep):
+        codes, mean = orc.ternarize(W)
+        ref = orc.ternary_linear(x, codes, mean)
+        assert (d["acc_out"].cpu().numpy() == ref["acc"]).all()
+        G.assert_y_close(d["y"].cpu().numpy(), ref["y"])
+
+
+# ------------------------------------------------------------ errors
+def test_wait_timeout_is_reported(dev, api):
+    api.debug_wait_timeout(2_000_000)   # 2 ms; nothing ever arrives
+    with pytest.raises(api.TernaryError) as e:
+        api.check()
+    assert e.value.status == 7
+    api.check()
+
+
+def test_argument_errors(dev, api):
+    import torch
+    x = torch.zeros((2, 128), dtype=torch.float32, device=dev)
+    packed, _, wscale = G.ternarize_gpu(_weights(16, 128, 1), dev)
+    with pytest.raises(api.TernaryError) as e:
+        api.ternary_linear(torch.zeros((2, 100), dtype=torch.float32, device=dev), packed,
+                           wscale, 16)
+    assert e.value.status == 2
+    flat = torch.zeros(2 * 128 + 1, dtype=torch.float32, device=dev)
+    with pytest.raises(api.TernaryError) as e:
+        api.ternary_linear(flat[1:].view(2, 128), packed, wscale, 16)
+    assert e.value.status == 3
+    y = api.ternary_linear(x, packed, wscale, 16)
+    api.check()
+    assert not y.cpu().numpy().any()
