@@ -124,8 +124,9 @@ TW_API int tw_unpack_codes(const void *packed, int64_t N, int64_t K, int8_t *cod
 TW_API int tw_quantize_act(const float *x, int64_t M, int64_t K, int8_t *xq,
                     float *amax, int32_t *qsum, tw_stream_t stream);
 
-/* Scratch needed by tw_ternary_linear / tw_ternary_linear_q for this shape
- * (0 for the decode path M <= 32). */
+/* Scratch needed by tw_ternary_linear for this shape: the int8 rows plus
+ * per-token scales (M <= 32: round128(M*K) + 256 bytes; larger M:
+ * M*K + 8*M bytes rounded up).  tw_ternary_linear_q needs none. */
 TW_API size_t tw_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
@@ -201,6 +202,10 @@ TW_API size_t tw_sweep_workspace_bytes(const void *table_host);
  */
 TW_API int tw_decoder_projection_sweep(const void *table_host, const void *table_dev,
                                 void *ws, size_t ws_bytes, tw_stream_t stream);
+
+/* HOST-ONLY.  Number of kernel launches one tw_decoder_projection_sweep call
+ * on this encoded table makes (0 for a malformed table). */
+TW_API int tw_sweep_launches(const void *table_host);
 
 /* Wait for `stream`, then return and clear the device error word of the
  * current device (TW_OK if no kernel reported an error). */

@@ -61,6 +61,7 @@ tw_sweep_table_bytes = _sig("tw_sweep_table_bytes", _sz, [_int])
 tw_sweep_table_encode = _sig("tw_sweep_table_encode", _int, [_p, _int, _i64, _p, _sz])
 tw_sweep_workspace_bytes = _sig("tw_sweep_workspace_bytes", _sz, [_p])
 tw_decoder_projection_sweep = _sig("tw_decoder_projection_sweep", _int, [_p, _p, _p, _sz, _p])
+tw_sweep_launches = _sig("tw_sweep_launches", _int, [_p])
 tw_check = _sig("tw_check", _int, [_p])
 tw_last_error = _sig("tw_last_error", ctypes.c_char_p, [])
 tw_debug_wait_timeout = _sig("tw_debug_wait_timeout", _int, [ctypes.c_uint64, _p])
@@ -206,6 +207,7 @@ class SweepTable:
         if device is not None:
             self.device = self.host.to(device, non_blocking=False)
         wsb = int(tw_sweep_workspace_bytes(_ptr(self.host)))
+        self.launches = int(tw_sweep_launches(_ptr(self.host)))
         self.ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=device) \
             if device is not None else None
         self.ws_bytes = wsb

@@ -75,7 +75,43 @@ int check_shape(int64_t M, int64_t N, int64_t K)
     return TW_OK;
 }
 
+size_t round256(int64_t b) { return (size_t)((b + 255) / 256 * 256); }
+
+// One projection on the tensor-core prefill path (any M >= 1).
+int run_prefill_single(const int8_t *xq, const float *amax, const int32_t *qsum, int64_t M,
+                       int64_t N, int64_t K, const void *packed, const float *wscale, float *y,
+                       int32_t *acc_out, uint32_t *err, cudaStream_t stream)
+{
+    tw::DescRecord r;
+    memset(&r, 0, sizeof(r));
+    r.xq = xq;
+    r.amax = amax;
+    r.qsum = qsum;
+    r.packed = static_cast<const uint8_t *>(packed);
+    r.wscale = wscale;
+    r.y = y;
+    r.acc_out = acc_out;
+    r.N = N;
+    r.K = K;
+    int rc = tw::encode_xq_tmap(xq, M, K, r.tmap_xq);
+    if (rc)
+        return fail(TW_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", rc);
+    tw::PrefillLaunch L{};
+    L.table = nullptr;
+    L.single = &r;
+    L.count = 1;
+    L.M = M;
+    L.total_ptiles = tw::prefill_tiles(M, N);
+    cudaError_t e = tw::launch_prefill(L, err, kWaitNs, stream);
+    return e == cudaSuccess ? TW_OK : cuda_fail(e, "prefill launch");
+}
+
 }  // namespace
+
+namespace tw {
+int error_word(uint32_t **out) { return err_word(out); }
+int record_error(int code, const char *msg) { return fail(code, "%s", msg); }
+}  // namespace tw
 
 extern "C" {
 
@@ -161,10 +197,8 @@ size_t tw_linear_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {
     (void)N;
     if (M <= tw::kDecodeMaxM)
-        return 0;
-    const size_t xq = (size_t)((M * K + 255) / 256 * 256);
-    const size_t vec = (size_t)((M * 4 + 255) / 256 * 256);
-    return xq + 2 * vec + 256;
+        return (size_t)(tw::round128(M * K) + 256);
+    return round256(M * K) + 2 * round256(M * 4);
 }
 
 int tw_ternary_linear(const float *x, int64_t M, int64_t N, int64_t K, const void *packed,
@@ -197,6 +231,7 @@ int tw_ternary_linear(const float *x, int64_t M, int64_t N, int64_t K, const voi
         r.acc_out = acc_out;
         r.N = N;
         r.K = K;
+        r.ws_xq_off = 0;
         tw::DecodeLaunch L{};
         L.table = nullptr;
         L.single = &r;
@@ -205,10 +240,19 @@ int tw_ternary_linear(const float *x, int64_t M, int64_t N, int64_t K, const voi
         L.total_rb = tw::ceil_div(N, tw::kTileRows);
         L.total_tiles = L.total_rb * (K / tw::kTileK);
         L.max_K = K;
+        L.ws = static_cast<uint8_t *>(ws);
+        L.ws_sa_off = tw::round128(M * K);
         cudaError_t e = tw::launch_decode(L, err, kWaitNs, stream);
         return e == cudaSuccess ? TW_OK : cuda_fail(e, "decode launch");
     }
-    return fail(TW_ERR_UNSUPPORTED, "prefill path (M > 32) is not built yet");
+    // Prefill: quantise into the workspace, then the tensor-core GEMM.
+    int8_t *xq = static_cast<int8_t *>(ws);
+    float *amax = reinterpret_cast<float *>(static_cast<char *>(ws) + round256(M * K));
+    int32_t *qsum = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(amax) + round256(M * 4));
+    cudaError_t e = tw::launch_quantize(x, M, K, xq, amax, qsum, stream);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "quantize launch");
+    return run_prefill_single(xq, amax, qsum, M, N, K, packed, wscale, y, acc_out, err, stream);
 }
 
 int tw_ternary_linear_q(const int8_t *xq, const float *amax, const int32_t *qsum, int64_t M,
@@ -216,9 +260,20 @@ int tw_ternary_linear_q(const int8_t *xq, const float *amax, const int32_t *qsum
                         int32_t *acc_out, void *ws, size_t ws_bytes, tw_stream_t stream)
 {
     t_last_error[0] = 0;
-    (void)xq; (void)amax; (void)qsum; (void)M; (void)N; (void)K; (void)packed; (void)wscale;
-    (void)y; (void)acc_out; (void)ws; (void)ws_bytes; (void)stream;
-    return fail(TW_ERR_UNSUPPORTED, "prefill path (M > 32) is not built yet");
+    (void)ws;
+    (void)ws_bytes;
+    if (!xq || !amax || !qsum || !packed || !wscale || !y)
+        return fail(TW_ERR_NULL,
+                    "tw_ternary_linear_q: xq, amax, qsum, packed, wscale and y are required");
+    if (int rc = check_shape(M, N, K))
+        return rc;
+    if (!aligned16(xq) || !aligned16(amax) || !aligned16(qsum) || !aligned16(packed) ||
+        !aligned16(wscale) || !aligned16(y) || (acc_out && !aligned16(acc_out)))
+        return fail(TW_ERR_ALIGN, "tw_ternary_linear_q: pointers must be 16-byte aligned");
+    uint32_t *err = nullptr;
+    if (int rc = err_word(&err))
+        return rc;
+    return run_prefill_single(xq, amax, qsum, M, N, K, packed, wscale, y, acc_out, err, stream);
 }
 
 size_t tw_sweep_table_bytes(int count)
@@ -242,12 +297,10 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
     if (M < 1 || M > (1 << 24))
         return fail(TW_ERR_SHAPE, "M=%lld out of range", (long long)M);
     const bool decode = M <= tw::kDecodeMaxM;
-    if (!decode)
-        return fail(TW_ERR_UNSUPPORTED, "prefill sweep (M > 32) is not built yet");
     auto *hdr = static_cast<tw::TableHeader *>(table);
     auto *recs = reinterpret_cast<tw::DescRecord *>(hdr + 1);
     memset(table, 0, tw_sweep_table_bytes(count));
-    int64_t rb = 0, tiles = 0, max_K = 0, sum_K = 0;
+    int64_t rb = 0, tiles = 0, ptiles = 0, max_K = 0, sum_K = 0, ws_off = 0;
     for (int d = 0; d < count; ++d) {
         const tw_proj_desc &s = descs[d];
         if (int rc = check_shape(M, s.N, s.K))
@@ -257,8 +310,12 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
                         (long long)tw::kDecodeMaxK);
         if (!s.packed || !s.wscale || !s.y || (decode && !s.x))
             return fail(TW_ERR_NULL, "descriptor %d: x, packed, wscale and y are required", d);
+        if (!decode && (!s.xq || !s.amax || !s.qsum))
+            return fail(TW_ERR_NULL, "descriptor %d: prefill needs xq, amax and qsum", d);
         if (!aligned16(s.packed) || !aligned16(s.wscale) || !aligned16(s.y) ||
-            (s.x && !aligned16(s.x)) || (s.acc_out && !aligned16(s.acc_out)))
+            (s.x && !aligned16(s.x)) || (s.acc_out && !aligned16(s.acc_out)) ||
+            (s.xq && !aligned16(s.xq)) || (s.amax && !aligned16(s.amax)) ||
+            (s.qsum && !aligned16(s.qsum)))
             return fail(TW_ERR_ALIGN, "descriptor %d: pointers must be 16-byte aligned", d);
         tw::DescRecord &r = recs[d];
         r.x = s.x;
@@ -273,6 +330,18 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
         r.K = s.K;
         r.rb_begin = rb;
         r.tile_begin = tiles;
+        r.ptile_begin = ptiles;
+        if (!decode) {
+            int rc = tw::encode_xq_tmap(s.xq, M, s.K, r.tmap_xq);
+            if (rc)
+                return fail(TW_ERR_CUDA, "descriptor %d: cuTensorMapEncodeTiled failed (%d)", d,
+                            rc);
+        }
+        ptiles += tw::prefill_tiles(M, s.N);
+        if (decode) {
+            r.ws_xq_off = ws_off;
+            ws_off += tw::round128(M * s.K);
+        }
         const int64_t nrb = tw::ceil_div(s.N, tw::kTileRows);
         rb += nrb;
         tiles += nrb * (s.K / tw::kTileK);
@@ -284,6 +353,8 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
     hdr->M = M;
     hdr->total_rb = rb;
     hdr->total_tiles = tiles;
+    hdr->total_ptiles = ptiles;
+    hdr->ws_bytes = decode ? ws_off + 256 * (int64_t)count : 0;
     hdr->max_K = max_K;
     hdr->sum_K = sum_K;
     return TW_OK;
@@ -291,16 +362,16 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
 
 size_t tw_sweep_workspace_bytes(const void *table_host)
 {
-    (void)table_host;
-    return 0;
+    const auto *hdr = static_cast<const tw::TableHeader *>(table_host);
+    if (!hdr || hdr->magic != tw::kTableMagic)
+        return 0;
+    return (size_t)hdr->ws_bytes;
 }
 
 int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, void *ws,
                                 size_t ws_bytes, tw_stream_t stream)
 {
     t_last_error[0] = 0;
-    (void)ws;
-    (void)ws_bytes;
     if (!table_host || !table_dev)
         return fail(TW_ERR_NULL, "tw_decoder_projection_sweep: host and device tables required");
     if ((reinterpret_cast<uintptr_t>(table_dev) & 63u) != 0)
@@ -311,8 +382,22 @@ int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, v
     uint32_t *err = nullptr;
     if (int rc = err_word(&err))
         return rc;
-    if (hdr->M > tw::kDecodeMaxM)
-        return fail(TW_ERR_UNSUPPORTED, "prefill sweep (M > 32) is not built yet");
+    if (hdr->M > tw::kDecodeMaxM) {
+        tw::PrefillLaunch P{};
+        P.table = reinterpret_cast<const tw::DescRecord *>(
+            static_cast<const tw::TableHeader *>(table_dev) + 1);
+        P.single = nullptr;
+        P.count = hdr->count;
+        P.M = hdr->M;
+        P.total_ptiles = hdr->total_ptiles;
+        cudaError_t e = tw::launch_prefill(P, err, kWaitNs, stream);
+        return e == cudaSuccess ? TW_OK : cuda_fail(e, "prefill sweep launch");
+    }
+    if (ws_bytes < (size_t)hdr->ws_bytes || !ws)
+        return fail(TW_ERR_BUFSIZE, "sweep workspace %zu < %lld bytes", ws_bytes,
+                    (long long)hdr->ws_bytes);
+    if (!aligned16(ws))
+        return fail(TW_ERR_ALIGN, "sweep workspace must be 16-byte aligned");
     tw::DecodeLaunch L{};
     L.table = reinterpret_cast<const tw::DescRecord *>(
         static_cast<const tw::TableHeader *>(table_dev) + 1);
@@ -322,8 +407,20 @@ int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, v
     L.total_rb = hdr->total_rb;
     L.total_tiles = hdr->total_tiles;
     L.max_K = hdr->max_K;
+    L.ws = static_cast<uint8_t *>(ws);
+    L.ws_sa_off = hdr->ws_bytes - 256 * (int64_t)hdr->count;
     cudaError_t e = tw::launch_decode(L, err, kWaitNs, stream);
     return e == cudaSuccess ? TW_OK : cuda_fail(e, "sweep launch");
+}
+
+int tw_sweep_launches(const void *table_host)
+{
+    const auto *hdr = static_cast<const tw::TableHeader *>(table_host);
+    if (!hdr || hdr->magic != tw::kTableMagic)
+        return 0;
+    if (hdr->M > tw::kDecodeMaxM)
+        return 1;
+    return tw::decode_launches(hdr->M, hdr->max_K);
 }
 
 int tw_check(tw_stream_t stream)

@@ -1,5 +1,5 @@
-// tw_decode.cu — fused activation-quantisation + ternary GEMV for decode
-// (M <= 32 tokens), as one persistent launch over any number of projections.
+// tw_decode.cu — activation quantisation + ternary GEMV for decode (M <= 32
+// tokens), as two launches over any number of projections.
 //
 // What it computes, per projection: q = absmax int8 quantisation of each
 // token row of x, acc = q * codes^T in exact integer arithmetic, and
@@ -9,21 +9,27 @@
 // bounds decode: "The Paper Says ARM Support" post, "What the model is
 // trying to do".)
 //
-// Structure (one CTA per SM, 9 warps):
+// Launch 1 (k_quant_rows): one block per (projection, token) quantises the
+// row, held in registers (one HBM round trip), into int8 scratch together
+// with amax/127 and sum(q).  It lets launch 2 start at once (programmatic
+// dependent launch), so the weight stream below overlaps it.
+//
+// Launch 2 (k_decode), one CTA per SM, 9 warps:
 //   * The grid splits the concatenated 16-row blocks of all projections into
 //     equal shares of packed bytes; each CTA streams its share once.
-//   * Warp 8 (activation warp) quantises, for every projection the CTA
-//     touches, the token rows of x into an int8 shared-memory buffer (double
-//     buffered when it fits) together with amax/127 and sum(q) per token.
-//   * Warps 0..7 (consumer warps) each own every 8th row block of the share.
-//     Each keeps a private ring of 4 KB slots filled by 1-D bulk copies (the
-//     TMA engine) that it issues itself, several chunks ahead, so the packed
-//     codes stream from HBM independently of the arithmetic.
-//   * Codes are decoded in registers: (word >> 2s) & 0x03030303 gives four
-//     codes + 1 as bytes, which are fed straight into m16n8k32 int8 MMAs
-//     (weights are the 16-row side, tokens the 8-column side).  The +1
-//     offset is removed at the end with the per-token sum(q):
-//     sum (c+1) q - sum q = sum c q, exactly.
+//   * Warps 0..7 (consumer warps) each own every 8th row block of the share
+//     and keep a private ring of 4 KB slots that they fill with 1-D bulk
+//     copies (the TMA engine) several chunks ahead, so the codes stream from
+//     HBM independently of the arithmetic.
+//   * Warp 8 (activation warp) waits for launch 1, then bulk-copies each
+//     projection's int8 rows, amax/127 and sum(q) into one of up to four
+//     shared-memory buffers ahead of the consumers.
+//   * Codes are decoded in registers with one AND per register:
+//     word & (0x03030303 << 2s) holds four codes + 1 of consecutive k,
+//     scaled by 4^s, as unsigned bytes; they feed m16n8k32 u8 x s8 MMAs
+//     (weights are the 16-row side, tokens the 8-column side), one
+//     accumulator per s.  At the end acc = sum_s (acc_s >> 2s) - sum(q),
+//     exact: sum (c+1) q - sum q = sum c q.
 //   * Every wait is bounded; a timeout sets the device error word, stops the
 //     block and drains the copies still in flight before the block exits.
 #include <cstring>
@@ -38,20 +44,34 @@ constexpr int kNC = 8;                      // consumer warps
 constexpr int kThreads = (kNC + 1) * 32;    // + activation warp
 constexpr int kCT = 8;                      // tiles per ring chunk
 constexpr int kChunk = kCT * kTileBytes;    // 4 KB
+constexpr int kMaxXB = 4;                   // activation buffers
 constexpr int kSmemLimit = 227 * 1024;
-constexpr int kMiscBytes = 2048;            // barriers, token info, plan
+constexpr int kMiscBytes = 2048 + 256 * kMaxXB;  // barriers, token info, plan
 constexpr uint64_t kDrainNs = 1000000000ull;
+constexpr int kQThreads = 256;
+constexpr int kQRegs = 12;                  // float4 per thread kept in registers
 
 struct DecodeParams {
     const DescRecord *table;  // null: use `single`
     DescRecord single;
     int count;
+    int M;
     int m0, mg;               // token group [m0, m0 + mg)
-    int xb;                   // activation buffers (1 or 2)
+    int xb;                   // activation buffers (1..4)
     int xs;                   // activation row stride in shared memory
     int slots;                // ring slots per consumer warp
     int64_t total_rb, total_tiles;
+    const uint8_t *ws;        // quantised activations (launch 1 output)
+    int64_t ws_sa_off;        // offset of the per-projection amax/127, sum(q)
     WaitCtl ctl;
+};
+
+struct QuantParams {
+    const DescRecord *table;
+    DescRecord single;
+    int count, M;
+    uint8_t *ws;
+    int64_t ws_sa_off;
 };
 
 struct Plan {
@@ -60,13 +80,112 @@ struct Plan {
     int abort_flag;
 };
 
-__device__ __forceinline__ const DescRecord &rec(const DecodeParams &p, int d)
+template <class P>
+__device__ __forceinline__ const DescRecord &rec(const P &p, int d)
 {
     return p.table ? p.table[d] : p.single;
 }
 
 __device__ __forceinline__ int64_t rb_count(const DescRecord &r) { return (r.N + 15) >> 4; }
 
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ----------------------------------------------------------------- launch 1
+__device__ __forceinline__ uint32_t quant4(float4 v, float scale, bool zero, int &sum)
+{
+    int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+    if (!zero) {
+        q0 = min(max(__float2int_rn(__fmul_rn(v.x, scale)), -128), 127);
+        q1 = min(max(__float2int_rn(__fmul_rn(v.y, scale)), -128), 127);
+        q2 = min(max(__float2int_rn(__fmul_rn(v.z, scale)), -128), 127);
+        q3 = min(max(__float2int_rn(__fmul_rn(v.w, scale)), -128), 127);
+    }
+    sum += q0 + q1 + q2 + q3;
+    return (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) | ((uint32_t)(q2 & 0xff) << 16) |
+           ((uint32_t)(q3 & 0xff) << 24);
+}
+
+__device__ __forceinline__ float amax4(float4 v)
+{
+    return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+}
+
+// Block (d, m): quantise token row m of projection d.  amax = max|x|,
+// scale = 127/amax (IEEE fp32), q = clamp(rint(x*scale), -128, 127).
+__global__ void __launch_bounds__(kQThreads) k_quant_rows(const __grid_constant__ QuantParams p)
+{
+    pdl_launch_dependents();
+    __shared__ float red_f[kQThreads / 32];
+    __shared__ int red_i[kQThreads / 32];
+    const int d = blockIdx.x / p.M, m = blockIdx.x % p.M;
+    const DescRecord &r = rec(p, d);
+    const int64_t K4 = r.K / 4;
+    const float4 *row = reinterpret_cast<const float4 *>(r.x + (int64_t)m * r.K);
+    uint32_t *qrow = reinterpret_cast<uint32_t *>(p.ws + r.ws_xq_off + (int64_t)m * r.K);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool in_regs = K4 <= (int64_t)kQRegs * kQThreads;
+
+    float4 v[kQRegs];
+    float a = 0.f;
+    if (in_regs) {
+#pragma unroll
+        for (int i = 0; i < kQRegs; ++i) {
+            const int64_t idx = tid + (int64_t)i * kQThreads;
+            v[i] = idx < K4 ? __ldg(row + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < kQRegs; ++i)
+            a = fmaxf(a, amax4(v[i]));
+    } else {
+        for (int64_t i = tid; i < K4; i += kQThreads)
+            a = fmaxf(a, amax4(__ldg(row + i)));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if (lane == 0)
+        red_f[warp] = a;
+    __syncthreads();
+    a = red_f[0];
+#pragma unroll
+    for (int w = 1; w < kQThreads / 32; ++w)
+        a = fmaxf(a, red_f[w]);
+
+    const bool zero = (a == 0.f);
+    const float scale = zero ? 0.f : __fdiv_rn(127.f, a);
+    int sum = 0;
+    if (in_regs) {
+#pragma unroll
+        for (int i = 0; i < kQRegs; ++i) {
+            const int64_t idx = tid + (int64_t)i * kQThreads;
+            if (idx < K4)
+                qrow[idx] = quant4(v[i], scale, zero, sum);
+        }
+    } else {
+        for (int64_t i = tid; i < K4; i += kQThreads)
+            qrow[i] = quant4(__ldg(row + i), scale, zero, sum);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0)
+        red_i[warp] = sum;
+    __syncthreads();
+    if (tid == 0) {
+        int s = 0;
+        for (int w = 0; w < kQThreads / 32; ++w)
+            s += red_i[w];
+        uint8_t *info = p.ws + p.ws_sa_off + 256 * (int64_t)d;
+        reinterpret_cast<float *>(info)[m] = __fdiv_rn(a, 127.f);
+        reinterpret_cast<int *>(info + 128)[m] = s;
+    }
+}
+
+// ----------------------------------------------------------------- launch 2
 // First row block owned by CTA i of G: the first block whose first tile is
 // at or after tile floor(total_tiles * i / G).
 __device__ int64_t share_boundary(const DecodeParams &p, int i, int G)
@@ -160,52 +279,43 @@ __device__ __forceinline__ void issue_chunk(const DecodeParams &p, const ChunkIt
     bulk_g2s(dst, src, (uint32_t)(n * kTileBytes), bar);
 }
 
-__device__ __forceinline__ uint32_t quant4(float4 v, float scale, bool zero, int &sum)
+// D(16x8, s32) += A(16x32, u8, row) * B(32x8, s8, col).
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1)
 {
-    int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
-    if (!zero) {
-        q0 = min(max(__float2int_rn(__fmul_rn(v.x, scale)), -128), 127);
-        q1 = min(max(__float2int_rn(__fmul_rn(v.y, scale)), -128), 127);
-        q2 = min(max(__float2int_rn(__fmul_rn(v.z, scale)), -128), 127);
-        q3 = min(max(__float2int_rn(__fmul_rn(v.w, scale)), -128), 127);
-    }
-    sum += q0 + q1 + q2 + q3;
-    return (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) | ((uint32_t)(q2 & 0xff) << 16) |
-           ((uint32_t)(q3 & 0xff) << 24);
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Activation warp: quantise token rows [m0, m0+mg) of projection d into
-// buffer b (row stride xs), amax/127 into sa[tok], sum(q) into qs[tok].
-__device__ void quantise_rows(const DecodeParams &p, int d, uint8_t *xbuf, float *sa, int *qs,
-                              int lane)
+__device__ __forceinline__ uint32_t comp(const uint4 &v, int s)
 {
-    const DescRecord &r = rec(p, d);
-    const int64_t K = r.K, K4 = K / 4;
-    for (int tok = 0; tok < p.mg; ++tok) {
-        const float4 *row = reinterpret_cast<const float4 *>(r.x + (int64_t)(p.m0 + tok) * K);
-        float a = 0.f;
-#pragma unroll 4
-        for (int64_t i = lane; i < K4; i += 32) {
-            const float4 v = __ldg(row + i);
-            a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-        }
+    return s == 0 ? v.x : s == 1 ? v.y : s == 2 ? v.z : v.w;
+}
+
+// One 16x128 tile.  Lane slot a holds 4 words: rows g and g+8 at k 16t.. and
+// 64+16t..; (word & (3 << 2s per byte)) are the codes + 1 of k = 16t+4s+b
+// (resp. 64+16t+4s+b), times 4^s.  MMA s pairs them with the token bytes at
+// the same k: component s of the 16-byte loads at xrow + koff (+ 64).
+template <int NT>
+__device__ __forceinline__ void tile_mma(int (&acc)[NT][4][4], const uint4 &a,
+                                         const uint32_t (&xrow)[NT], uint32_t koff)
+{
+    uint4 b0[NT], b1[NT];
 #pragma unroll
-        for (int o = 16; o; o >>= 1)
-            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        const bool zero = (a == 0.f);
-        const float scale = zero ? 0.f : __fdiv_rn(127.f, a);
-        uint32_t *dst = reinterpret_cast<uint32_t *>(xbuf + (int64_t)tok * p.xs);
-        int sum = 0;
-#pragma unroll 4
-        for (int64_t i = lane; i < K4; i += 32)
-            dst[i] = quant4(__ldg(row + i), scale, zero, sum);
+    for (int nt = 0; nt < NT; ++nt) {
+        b0[nt] = lds128(xrow[nt] + koff);
+        b1[nt] = lds128(xrow[nt] + koff + 64);
+    }
 #pragma unroll
-        for (int o = 16; o; o >>= 1)
-            sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) {
-            sa[tok] = __fdiv_rn(a, 127.f);
-            qs[tok] = sum;
-        }
+    for (int s = 0; s < 4; ++s) {
+        const uint32_t mk = 0x03030303u << (2 * s);
+        const uint32_t a0 = a.x & mk, a1 = a.y & mk, a2 = a.z & mk, a3 = a.w & mk;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            mma_u8s8(acc[nt][s], a0, a1, a2, a3, comp(b0[nt], s), comp(b1[nt], s));
     }
 }
 
@@ -215,25 +325,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    // Layout: rings | zero row (at 64 mod 128) | activation buffers (rows at
+    // 0 mod 128, stride xs = 64 mod 128) | token info | barriers | plan.
     const int ring_bytes = kNC * p.slots * kChunk;
     uint8_t *ring = smem;
-    uint8_t *xbase = smem + ring_bytes;
+    uint8_t *zero_row = smem + ring_bytes + 64;
+    uint8_t *xbase = smem + ring_bytes + 64 + p.xs;  // = ring + K + 128: 0 mod 128
     const int xbuf_bytes = p.mg * p.xs;
-    uint8_t *misc = xbase + p.xb * xbuf_bytes;
-    float *sa = reinterpret_cast<float *>(misc);             // [2][32]
-    int *qs = reinterpret_cast<int *>(misc + 256);           // [2][32]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(misc + 512);
-    // bars: ring_full[kNC*slots], x_full[2], x_empty[2]
-    Plan *plan = reinterpret_cast<Plan *>(misc + 512 + 8 * (kNC * p.slots + 4));
+    uint8_t *misc = xbase + p.xb * xbuf_bytes + 128;
+    misc += (128 - (smem_u32(misc) & 127)) & 127;
+    uint8_t *info = misc;                                    // [xb][256]: sa[32], qs[32]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(misc + 256 * kMaxXB);
+    // bars: ring_full[kNC*slots], x_full[kMaxXB], x_empty[kMaxXB]
+    Plan *plan = reinterpret_cast<Plan *>(misc + 256 * kMaxXB + 8 * (kNC * p.slots + 2 * kMaxXB));
     const uint32_t bar_ring = smem_u32(bars);
     const uint32_t bar_xfull = bar_ring + 8 * kNC * p.slots;
-    const uint32_t bar_xempty = bar_xfull + 16;
+    const uint32_t bar_xempty = bar_xfull + 8 * kMaxXB;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNC * p.slots; ++i)
             mbar_init(bar_ring + 8 * i, 1);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar_xfull + 8 * b, 32);
+        for (int b = 0; b < kMaxXB; ++b) {
+            mbar_init(bar_xfull + 8 * b, 1);
             mbar_init(bar_xempty + 8 * b, kNC * 32);
         }
         fence_barrier_init();
@@ -249,21 +362,39 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             plan->d_hi = -1;
         }
     }
+    for (int i = threadIdx.x; i < p.xs / 16; i += kThreads)
+        reinterpret_cast<uint4 *>(zero_row)[i] = make_uint4(0, 0, 0, 0);
     __syncthreads();
     const Plan pl = *plan;
     volatile int *abort_flag = &plan->abort_flag;
 
     if (warp == kNC) {
         // ------------------------------------------------ activation warp
-        for (int d = pl.d_lo; d <= pl.d_hi; ++d) {
-            const int seg = d - pl.d_lo, b = seg % p.xb;
-            if (seg >= p.xb &&
-                !mbar_wait(bar_xempty + 8 * b, ((seg / p.xb) - 1) & 1, p.ctl, abort_flag))
-                return;
-            quantise_rows(p, d, xbase + b * xbuf_bytes, sa + 32 * b, qs + 32 * b, lane);
-            __syncwarp();
-            mbar_arrive(bar_xfull + 8 * b);
+        if (lane == 0) {
+            pdl_wait();  // launch 1 has finished writing the int8 rows
+            for (int d = pl.d_lo; d <= pl.d_hi; ++d) {
+                const int seg = d - pl.d_lo, b = seg % p.xb;
+                if (seg >= p.xb &&
+                    !mbar_wait(bar_xempty + 8 * b, ((seg / p.xb) - 1) & 1, p.ctl, abort_flag))
+                    break;
+                const DescRecord &r = rec(p, d);
+                const uint32_t bx = bar_xfull + 8 * b;
+                const uint32_t dst = smem_u32(xbase + b * xbuf_bytes);
+                mbar_arrive_expect_tx(bx, (uint32_t)(p.mg * r.K + 256));
+                for (int tok = 0; tok < p.mg; ++tok)
+                    bulk_g2s(dst + tok * p.xs, p.ws + r.ws_xq_off + (int64_t)(p.m0 + tok) * r.K,
+                             (uint32_t)r.K, bx);
+                bulk_g2s(smem_u32(info + 256 * b), p.ws + p.ws_sa_off + 256 * (int64_t)d, 256, bx);
+            }
+            // Drain: the activation copies of the last buffers land before exit.
+            WaitCtl drain = p.ctl;
+            drain.timeout_ns = kDrainNs;
+            const int nseg = pl.d_hi - pl.d_lo + 1;
+            for (int seg = nseg - p.xb; seg < nseg; ++seg)
+                if (seg >= 0)
+                    mbar_wait(bar_xfull + 8 * (seg % p.xb), (seg / p.xb) & 1, drain, nullptr);
         }
+        __syncwarp();
         return;
     }
 
@@ -271,23 +402,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     const int g = lane >> 2, t = lane & 3;
     const uint32_t ring_w = smem_u32(ring) + warp * p.slots * kChunk;
     const uint32_t bar_w = bar_ring + 8 * warp * p.slots;
-    const uint32_t xbase_s = smem_u32(xbase);
+    const uint32_t zero_s = smem_u32(zero_row);
 
     ChunkIter cons, prod;
     cons.init(p, pl, warp);
     prod = cons;
     int issued = 0, consumed = 0;
-    if (lane == 0) {
-        for (int s = 0; s < p.slots && prod.valid; ++s) {
+    for (int s = 0; s < p.slots && prod.valid; ++s) {
+        if (lane == 0)
             issue_chunk(p, prod, ring_w + s * kChunk, bar_w + 8 * s);
-            prod.next(p);
-            ++issued;
-        }
-    } else {
-        for (int s = 0; s < p.slots && prod.valid; ++s) {
-            prod.next(p);
-            ++issued;
-        }
+        prod.next(p);
+        ++issued;
     }
 
     bool ok = true;
@@ -299,17 +424,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         }
         const DescRecord &r = rec(p, d);
         const float wscale = __ldg(r.wscale);
-        const uint32_t xrow = xbase_s + b * xbuf_bytes;
+        const float *sa = reinterpret_cast<const float *>(info + 256 * b);
+        const int *qs = reinterpret_cast<const int *>(info + 256 * b + 128);
+        uint32_t xrow[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int tok = 8 * nt + g;
+            xrow[nt] = (tok < p.mg ? smem_u32(xbase + b * xbuf_bytes + tok * p.xs) : zero_s) +
+                       16 * t;
+        }
 
         while (cons.valid && cons.d == d) {
-            int acc[2][NT][4];
+            int acc[NT][4][4];
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+                for (int s = 0; s < 4; ++s)
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        acc[h][nt][i] = 0;
+                        acc[nt][s][i] = 0;
             const int64_t rb = cons.rb;
             const int nch = cons.nch, KT = cons.KT;  // cons moves on after the last chunk
             for (int kc = 0; kc < nch; ++kc) {
@@ -321,32 +454,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                 const int kt0 = kc * kCT;
                 const int n = min(kCT, KT - kt0);
                 const uint32_t src = ring_w + slot * kChunk + lane * 16;
-                for (int i = 0; i < n; ++i) {
-                    const uint4 a = lds128(src + i * kTileBytes);
-                    const uint32_t xk = xrow + (kt0 + i) * kTileK + 16 * t;
+                const uint32_t kbase = (uint32_t)kt0 * kTileK;
+                if (n == kCT) {
+                    uint4 a[kCT];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t w0 = h ? a.z : a.x;  // row g
-                        const uint32_t w1 = h ? a.w : a.y;  // row g + 8
-                        uint4 bx[NT];
+                    for (int i = 0; i < kCT; ++i)
+                        a[i] = lds128(src + i * kTileBytes);
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            const int tok = 8 * nt + g;
-                            bx[nt] = tok < p.mg ? lds128(xk + tok * p.xs + 64 * h)
-                                                : make_uint4(0, 0, 0, 0);
-                        }
-                        const uint32_t m3 = 0x03030303u;
-                        const uint32_t a00 = w0 & m3, a01 = w1 & m3;
-                        const uint32_t a02 = (w0 >> 2) & m3, a03 = (w1 >> 2) & m3;
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-                            mma_s8_16832(acc[0][nt], a00, a01, a02, a03, bx[nt].x, bx[nt].y);
-                        const uint32_t a10 = (w0 >> 4) & m3, a11 = (w1 >> 4) & m3;
-                        const uint32_t a12 = (w0 >> 6) & m3, a13 = (w1 >> 6) & m3;
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-                            mma_s8_16832(acc[1][nt], a10, a11, a12, a13, bx[nt].z, bx[nt].w);
-                    }
+                    for (int i = 0; i < kCT; ++i)
+                        tile_mma<NT>(acc, a[i], xrow, kbase + i * kTileK);
+                } else {
+                    for (int i = 0; i < n; ++i)
+                        tile_mma<NT>(acc, lds128(src + i * kTileBytes), xrow, kbase + i * kTileK);
                 }
                 __syncwarp();
                 ++consumed;
@@ -371,9 +490,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                     const int tok = 8 * nt + 2 * t + (i & 1);
                     const int64_t row = rl * kTileRows + g + 8 * (i >> 1);
                     if (tok < p.mg && row < r.N) {
-                        const int v = acc[0][nt][i] + acc[1][nt][i] - qs[32 * b + tok];
-                        const int64_t o = (int64_t)(p.m0 + tok) * r.N + row;
-                        r.y[o] = __fmul_rn(__fmul_rn((float)v, sa[32 * b + tok]), wscale);
+                        const int m = p.m0 + tok;  // sa/qs hold all M tokens
+                        const int v = acc[nt][0][i] + (acc[nt][1][i] >> 2) +
+                                      (acc[nt][2][i] >> 4) + (acc[nt][3][i] >> 6) - qs[m];
+                        const int64_t o = (int64_t)m * r.N + row;
+                        r.y[o] = __fmul_rn(__fmul_rn((float)v, sa[m]), wscale);
                         if (r.acc_out)
                             r.acc_out[o] = v;
                     }
@@ -413,11 +534,54 @@ cudaError_t launch_nt(const DecodeParams &p, int grid, int smem, cudaStream_t st
                                          smem);
     if (e != cudaSuccess)
         return e;
-    k_decode<NT><<<grid, kThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    // Programmatic dependent launch: may start while k_quant_rows runs.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_decode<NT>, p);
+}
+
+// Bytes of dynamic shared memory of k_decode for this plan.
+int64_t smem_bytes(int slots, int mg, int xb, int64_t max_K)
+{
+    const int64_t xs = max_K + 64;
+    return 1024 + (int64_t)kNC * slots * kChunk + xs + 128 + (int64_t)xb * mg * xs + 256 +
+           kMiscBytes;
+}
+
+// Largest token group (and its ring depth) that fits shared memory.
+bool plan_groups(int M, int64_t max_K, int *mg_out, int *slots_out)
+{
+    int mg = M;
+    while (true) {
+        for (int s = 4; s >= 2; --s)
+            if (smem_bytes(s, mg, 1, max_K) <= kSmemLimit) {
+                *mg_out = mg;
+                *slots_out = s;
+                return true;
+            }
+        if (mg == 1)
+            return false;
+        mg = mg > 8 ? mg - 8 : mg - 1;
+    }
 }
 
 }  // namespace
+
+int decode_launches(int64_t M, int64_t max_K)
+{
+    int mg = 1, slots = 2;
+    if (!plan_groups((int)M, max_K, &mg, &slots))
+        return 0;
+    return 1 + (int)((M + mg - 1) / mg);  // quantise + one decode launch per group
+}
 
 cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout_ns,
                           cudaStream_t stream)
@@ -428,6 +592,28 @@ cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess)
         return e;
+    const int M = (int)L.M;
+    int mg = 1, slots = 2;
+    if (!plan_groups(M, L.max_K, &mg, &slots))
+        return cudaErrorInvalidValue;
+    int xb = 1;
+    while (xb < kMaxXB && smem_bytes(slots, mg, xb + 1, L.max_K) <= kSmemLimit)
+        ++xb;
+
+    // Launch 1: quantise every (projection, token) row.
+    QuantParams q;
+    memset(&q, 0, sizeof(q));
+    q.table = L.table;
+    if (L.single)
+        q.single = *L.single;
+    q.count = L.count;
+    q.M = M;
+    q.ws = L.ws;
+    q.ws_sa_off = L.ws_sa_off;
+    k_quant_rows<<<(unsigned)(L.count * (int64_t)M), kQThreads, 0, stream>>>(q);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
 
     DecodeParams p;
     memset(&p, 0, sizeof(p));
@@ -435,36 +621,18 @@ cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout
     if (L.single)
         p.single = *L.single;
     p.count = L.count;
+    p.M = M;
     p.total_rb = L.total_rb;
     p.total_tiles = L.total_tiles;
     p.xs = (int)(L.max_K + 64);
+    p.ws = L.ws;
+    p.ws_sa_off = L.ws_sa_off;
     p.ctl.err = err;
     p.ctl.timeout_ns = timeout_ns;
-
-    // Shared-memory plan: ring, then 1 or 2 activation buffers of mg rows.
-    const int M = (int)L.M;
-    auto fits = [&](int s, int m, int b) {
-        return 1024 + kNC * s * kChunk + b * m * p.xs + kMiscBytes <= kSmemLimit;
-    };
-    // Largest token group that fits with a ring of 4 (else 3, else 2)
-    // slots per warp; a second activation buffer only when it also fits.
-    int slots = 0, mg = M, xb = 1;
-    while (true) {
-        for (int s = 4; s >= 2 && !slots; --s)
-            if (fits(s, mg, 1))
-                slots = s;
-        if (slots)
-            break;
-        if (mg == 1)
-            return cudaErrorInvalidValue;
-        mg = mg > 8 ? mg - 8 : mg - 1;
-    }
-    if (fits(slots, mg, 2))
-        xb = 2;
     p.slots = slots;
     p.xb = xb;
-    const int smem = 1024 + kNC * slots * kChunk + xb * mg * p.xs + kMiscBytes;
-    int64_t grid64 = L.total_rb < sms ? L.total_rb : sms;
+    const int smem = (int)smem_bytes(slots, mg, xb, L.max_K);
+    const int64_t grid64 = L.total_rb < sms ? L.total_rb : sms;
     const int grid = (int)(grid64 < 1 ? 1 : grid64);
 
     for (int m0 = 0; m0 < M; m0 += mg) {

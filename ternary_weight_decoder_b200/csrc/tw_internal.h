@@ -32,7 +32,8 @@ struct alignas(64) DescRecord {
     int64_t rb_begin;    // first 16-row block of this projection in the sweep
     int64_t tile_begin;  // first 16x128 code tile of this projection
     int64_t ptile_begin; // first prefill output tile of this projection
-    int64_t reserved[3];
+    int64_t ws_xq_off;   // decode: offset of this projection's int8 rows in ws
+    int64_t reserved[2];
     alignas(64) uint8_t tmap_xq[128];  // CUtensorMap of xq (prefill only)
 };
 static_assert(sizeof(DescRecord) == 256, "record size");
@@ -46,7 +47,7 @@ struct alignas(64) TableHeader {
     int64_t total_ptiles;
     int64_t max_K;
     int64_t sum_K;
-    int64_t reserved[1];
+    int64_t ws_bytes;    // decode: scratch for the quantised activations
 };
 static_assert(sizeof(TableHeader) == 64, "header size");
 
@@ -68,10 +69,38 @@ struct DecodeLaunch {
     int64_t M;
     int64_t total_rb, total_tiles, max_K;
     const DescRecord *single; // host copy of a one-record sweep (table == null)
+    uint8_t *ws;              // scratch: int8 rows at each record's ws_xq_off,
+    int64_t ws_sa_off;        // then 256 bytes of amax/127, sum(q) per record
 };
+// Kernel launches one decode call makes for M tokens (quantise + groups).
+int decode_launches(int64_t M, int64_t max_K);
+// Decode scratch: per projection its M int8 rows (128-byte aligned), then
+// per projection 256 bytes: 32 floats amax/127 and 32 ints sum(q).
+inline int64_t round128(int64_t b) { return (b + 127) / 128 * 128; }
 cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout_ns,
                           cudaStream_t stream);
 
+struct PrefillLaunch {
+    const DescRecord *table;  // device records (or null: use `single`)
+    int count;
+    int64_t M;
+    int64_t total_ptiles;
+    const DescRecord *single; // host record incl. its TMA descriptor
+};
+cudaError_t launch_prefill(const PrefillLaunch &L, uint32_t *err, uint64_t timeout_ns,
+                           cudaStream_t stream);
+// Output tiles of one projection on the prefill path (128 x 256 each).
+int64_t prefill_tiles(int64_t M, int64_t N);
+// Encode the TMA descriptor of xq [M x K] int8 into out128 (128 bytes).
+// Returns 0, -1 when the driver entry point is unavailable, or a CUresult.
+int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, void *out128);
+
 cudaError_t launch_wait_probe(uint32_t *err, uint64_t timeout_ns, cudaStream_t stream);
+
+// Address of the per-device error word on the current device (TW_OK or a
+// TW_ERR_* status; the message is kept for tw_last_error()).
+int error_word(uint32_t **out);
+// Record a message for tw_last_error() and return `code`.
+int record_error(int code, const char *msg);
 
 }  // namespace tw

@@ -1,0 +1,471 @@
+// tw_prefill.cu — ternary GEMM for prefill (M > 32 tokens) on the 5th-
+// generation tensor cores (tcgen05, int8, int32 accumulators in TMEM).
+//
+// D[m, n] = sum_k xq[m, k] * (code[n, k] + 1) runs as tcgen05.mma kind::i8
+// (A = int8 activations, K-major, loaded by TMA with 128-byte swizzle;
+// B = codes + 1 expanded from the 2-bit layout into int8 in shared memory by
+// eight expansion warps), then the epilogue removes the +1 offset with the
+// per-token sum(q) and rescales:
+//   acc = D - qsum[m],   y = ((float)acc * (amax[m] / 127)) * mean|W|.
+// (Per-tensor ternary weights, s = 1/mean|W|: "VibeVoice-ASR-BitNet-ONNX"
+// model page, Quantization table.  The prefill length is the audio frame
+// count plus the prompt, one frame per 3200 samples of 24 kHz audio: same
+// page, "Layout".)
+//
+// Tile: 128 tokens x 256 weight rows, K in stages of 128 (one swizzle atom),
+// four MMAs of K = 32 per stage.  Persistent: one CTA per SM walks the
+// output tiles of every projection (all token tiles of a weight tile run
+// back to back across the grid, so the weight codes stream from HBM once
+// and the activations stay in L2).  Two TMEM accumulators let the epilogue
+// of one tile overlap the main loop of the next.
+//
+// Warps: 0 TMA producer, 1 MMA issuer (and TMEM owner), 2..5 epilogue
+// (TMEM lane quarters 2, 3, 0, 1), 6..13 code expansion.  Every wait is
+// bounded; on a timeout the block stops, drains its copies and MMAs, frees
+// its TMEM and returns.
+#include <cstring>
+#include <cuda.h>
+
+#include "tw_device.cuh"
+#include "tw_internal.h"
+
+namespace tw {
+namespace {
+
+constexpr int kBM = 128;                 // tokens per tile (MMA M)
+constexpr int kBN = 256;                 // weight rows per tile (MMA N)
+constexpr int kBK = 128;                 // k per stage
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK;       // 16 KB
+constexpr int kBBytes = kBN * kBK;       // 32 KB
+constexpr int kCodeBytes = kBN / kTileRows * kTileBytes;  // 16 tiles = 8 KB
+constexpr int kStageBytes = kABytes + kBBytes + kCodeBytes;
+constexpr int kNumExp = 8;               // expansion warps
+constexpr int kThreads = (6 + kNumExp) * 32;
+constexpr int kTmemCols = 512;           // two 256-column accumulators
+constexpr uint64_t kDrainNs = 1000000000ull;
+
+struct PrefillParams {
+    const DescRecord *table;  // null: use `single`
+    DescRecord single;
+    int count;
+    int64_t M;
+    int64_t total_ptiles;
+    WaitCtl ctl;
+};
+
+__device__ __forceinline__ const DescRecord &prec(const PrefillParams &p, int d)
+{
+    return p.table ? p.table[d] : p.single;
+}
+
+// Output tile t -> projection d, token tile mi, weight tile nj.  Inside a
+// projection the token tiles of one weight tile are consecutive.
+struct TileCoord {
+    int d;
+    int64_t mi, nj;
+};
+
+__device__ TileCoord tile_coord(const PrefillParams &p, int64_t t)
+{
+    int lo = 0, hi = p.count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prec(p, mid).ptile_begin <= t)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    const int64_t tm = (p.M + kBM - 1) / kBM;
+    const int64_t local = t - prec(p, lo).ptile_begin;
+    return TileCoord{lo, local % tm, local / tm};
+}
+
+// ------------------------------------------------------------- tcgen05 PTX
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(dst_smem), "r"(ncols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::i8, int32 accumulate.
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on `bar` when every MMA issued so far by this thread has completed.
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(bar) : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i gets row (lane base + i).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+          "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 2-D TMA load of one box into shared memory (no multicast).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int32_t x, int32_t y,
+                                            uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle,
+// 8-row groups 1024 bytes apart (SBO), leading offset unused (1).
+__device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr)
+{
+    uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;   // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;   // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: int8 x int8 -> int32, both K-major, M = 128, N = 256.
+constexpr uint32_t kIdesc = (2u << 4)            // D format: s32
+                            | (1u << 7)          // A: signed int8
+                            | (1u << 10)         // B: signed int8
+                            | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+
+struct SmemLayout {
+    uint32_t base;  // 1024-aligned shared address of stage 0
+    __device__ uint32_t a(int s) const { return base + s * kStageBytes; }
+    __device__ uint32_t b(int s) const { return base + s * kStageBytes + kABytes; }
+    __device__ uint32_t codes(int s) const { return base + s * kStageBytes + kABytes + kBBytes; }
+};
+
+__global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__ PrefillParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gen_base = smem_raw + (base - raw);
+    SmemLayout L{base};
+    uint8_t *misc = gen_base + kStages * kStageBytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(misc);
+    // barriers: load_full[S], exp_full[S], empty[S], tmem_full[2], tmem_empty[2], drain
+    const uint32_t bar0 = smem_u32(bars);
+    const uint32_t b_load = bar0, b_exp = bar0 + 8 * kStages, b_empty = bar0 + 16 * kStages;
+    const uint32_t b_tfull = bar0 + 24 * kStages, b_tempty = b_tfull + 16;
+    const uint32_t b_drain = b_tempty + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 512);
+    int *abort_flag_p = reinterpret_cast<int *>(misc + 520);
+    volatile int *abort_flag = abort_flag_p;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(b_load + 8 * s, 1);
+            mbar_init(b_exp + 8 * s, kNumExp * 32);
+            mbar_init(b_empty + 8 * s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(b_tfull + 8 * a, 1);
+            mbar_init(b_tempty + 8 * a, 4 * 32);
+        }
+        mbar_init(b_drain, 1);
+        *abort_flag_p = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1)
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int64_t G = gridDim.x;
+    const int64_t ntiles = p.total_ptiles;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            int64_t it = 0;
+            for (int64_t t = blockIdx.x; t < ntiles && !*abort_flag; t += G) {
+                const TileCoord c = tile_coord(p, t);
+                const DescRecord &r = prec(p, c.d);
+                const int64_t KT = r.K / kBK;
+                const int64_t nrb = (r.N + kTileRows - 1) / kTileRows;
+                const int64_t rb0 = c.nj * (kBN / kTileRows);
+                const int nct = (int)min((int64_t)(kBN / kTileRows), nrb - rb0);
+                const uint32_t bytes = kABytes + nct * kTileBytes;
+                for (int64_t kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = (int)(it % kStages);
+                    if (it >= kStages &&
+                        !mbar_wait(b_empty + 8 * s, (uint32_t)((it / kStages - 1) & 1), p.ctl,
+                                   abort_flag))
+                        break;
+                    mbar_arrive_expect_tx(b_load + 8 * s, bytes);
+                    tma_load_2d(L.a(s), r.tmap_xq, (int32_t)(kt * kBK), (int32_t)(c.mi * kBM),
+                                b_load + 8 * s);
+                    for (int i = 0; i < nct; ++i)
+                        bulk_g2s(L.codes(s) + i * kTileBytes,
+                                 r.packed + ((rb0 + i) * KT + kt) * kTileBytes, kTileBytes,
+                                 b_load + 8 * s);
+                }
+            }
+            // Drain: the last (up to) kStages loads must land before exit.
+            WaitCtl drain = p.ctl;
+            drain.timeout_ns = kDrainNs;
+            for (int64_t j = it - kStages; j < it; ++j)
+                if (j >= 0)
+                    mbar_wait(b_load + 8 * (int)(j % kStages), (uint32_t)((j / kStages) & 1), drain,
+                              nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int64_t it = 0, tt = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < ntiles && ok; t += G, ++tt) {
+                const TileCoord c = tile_coord(p, t);
+                const int64_t KT = prec(p, c.d).K / kBK;
+                const int ab = (int)(tt & 1);
+                if (tt >= 2 && !mbar_wait(b_tempty + 8 * ab, (uint32_t)((tt / 2 - 1) & 1), p.ctl,
+                                          abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(ab * kBN);
+                for (int64_t kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = (int)(it % kStages);
+                    const uint32_t par = (uint32_t)((it / kStages) & 1);
+                    if (!mbar_wait(b_load + 8 * s, par, p.ctl, abort_flag) ||
+                        !mbar_wait(b_exp + 8 * s, par, p.ctl, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sdesc_k_sw128(L.a(s));
+                    const uint64_t bd = sdesc_k_sw128(L.b(s));
+#pragma unroll
+                    for (int j = 0; j < kBK / 32; ++j)  // +32 bytes of K = +2 in the address field
+                        mma_i8(d_tmem, ad + 2 * j, bd + 2 * j, kIdesc, (kt > 0 || j > 0) ? 1u : 0u);
+                    mma_commit(b_empty + 8 * s);
+                }
+                if (!ok)
+                    break;
+                mma_commit(b_tfull + 8 * ab);
+            }
+            // All MMAs issued by this thread complete before TMEM is freed.
+            mma_commit(b_drain);
+            WaitCtl drain = p.ctl;
+            drain.timeout_ns = kDrainNs;
+            mbar_wait(b_drain, 0, drain, nullptr);
+        }
+        __syncwarp();
+    } else if (warp < 6) {
+        // ------------------------------------------------------ epilogue
+        const int quarter = warp & 3;                 // TMEM lanes 32q..32q+31
+        int64_t tt = 0;
+        for (int64_t t = blockIdx.x; t < ntiles; t += G, ++tt) {
+            const TileCoord c = tile_coord(p, t);
+            const DescRecord &r = prec(p, c.d);
+            const int ab = (int)(tt & 1);
+            if (!mbar_wait(b_tfull + 8 * ab, (uint32_t)((tt / 2) & 1), p.ctl, abort_flag))
+                break;
+            tc_fence_after();
+            const int64_t m = c.mi * kBM + quarter * 32 + lane;
+            const bool row_ok = m < p.M;
+            const float sa = row_ok ? __fdiv_rn(__ldg(r.amax + m), 127.f) : 0.f;
+            const int qs = row_ok ? __ldg(r.qsum + m) : 0;
+            const float wscale = __ldg(r.wscale);
+            const int64_t n0 = c.nj * kBN;
+            for (int cc = 0; cc < kBN / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * kBN + cc * 32), v);
+                if (!row_ok)
+                    continue;
+                const int64_t nb = n0 + cc * 32;
+                float *yrow = r.y + m * r.N;
+                int32_t *arow = r.acc_out ? r.acc_out + m * r.N : nullptr;
+                if (nb + 32 <= r.N && (r.N & 3) == 0) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        int a4[4];
+                        float f4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            a4[e] = (int)v[4 * q + e] - qs;
+                            f4[e] = __fmul_rn(__fmul_rn((float)a4[e], sa), wscale);
+                        }
+                        *reinterpret_cast<float4 *>(yrow + nb + 4 * q) =
+                            make_float4(f4[0], f4[1], f4[2], f4[3]);
+                        if (arow)
+                            *reinterpret_cast<int4 *>(arow + nb + 4 * q) =
+                                make_int4(a4[0], a4[1], a4[2], a4[3]);
+                    }
+                } else {
+                    for (int e = 0; e < 32 && nb + e < r.N; ++e) {
+                        const int a = (int)v[e] - qs;
+                        yrow[nb + e] = __fmul_rn(__fmul_rn((float)a, sa), wscale);
+                        if (arow)
+                            arow[nb + e] = a;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(b_tempty + 8 * ab);
+        }
+    } else {
+        // ------------------------------------------------------ expansion
+        const int e = threadIdx.x - 6 * 32;           // 0..255
+        int64_t it = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < ntiles && ok; t += G) {
+            const TileCoord c = tile_coord(p, t);
+            const int64_t KT = prec(p, c.d).K / kBK;
+            for (int64_t kt = 0; kt < KT; ++kt, ++it) {
+                const int s = (int)(it % kStages);
+                if (!mbar_wait(b_load + 8 * s, (uint32_t)((it / kStages) & 1), p.ctl, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                // Two 16-byte lane slots per thread: slot q = e + 256*h is lane
+                // l = q % 32 of code tile q / 32 (rows 16*(q/32) .. +15).
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int q = e + 256 * h;
+                    const int tile = q >> 5, l = q & 31;
+                    const int g = l >> 2, tq = l & 3;
+                    const uint4 w = lds128(L.codes(s) + tile * kTileBytes + l * 16);
+                    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = (jj + 2 * (g & 1)) & 3;   // staggered: no bank conflicts
+                        const uint32_t wd = words[j];
+                        const int row = tile * kTileRows + g + 8 * (j & 1);
+                        const int chunk = 4 * (j >> 1) + tq;      // 16-byte chunk of the 128 B row
+                        const uint32_t dst = L.b(s) + row * 128 + ((chunk ^ (row & 7)) << 4);
+                        const uint32_t m3 = 0x03030303u;
+                        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst),
+                                     "r"(wd & m3), "r"((wd >> 2) & m3), "r"((wd >> 4) & m3),
+                                     "r"((wd >> 6) & m3)
+                                     : "memory");
+                    }
+                }
+                fence_proxy_async_smem();  // make the B tile visible to the tensor cores
+                mbar_arrive(b_exp + 8 * s);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, void *out128)
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !f)
+            return -1;
+        fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    CUtensorMap m;
+    memset(&m, 0, sizeof(m));
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)K};
+    const cuuint32_t box[2] = {kBK, kBM};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(xq), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return (int)r;
+    static_assert(sizeof(CUtensorMap) == 128, "tensor map size");
+    memcpy(out128, &m, sizeof(m));
+    return 0;
+}
+
+int64_t prefill_tiles(int64_t M, int64_t N)
+{
+    return ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
+}
+
+cudaError_t launch_prefill(const PrefillLaunch &L, uint32_t *err, uint64_t timeout_ns,
+                           cudaStream_t stream)
+{
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess)
+        return e;
+    PrefillParams p;
+    memset(&p, 0, sizeof(p));
+    p.table = L.table;
+    if (L.single)
+        p.single = *L.single;
+    p.count = L.count;
+    p.M = L.M;
+    p.total_ptiles = L.total_ptiles;
+    p.ctl.err = err;
+    p.ctl.timeout_ns = timeout_ns;
+    const int smem = kStages * kStageBytes + 1024 /*align*/ + 1024 /*misc*/;
+    e = cudaFuncSetAttribute(k_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+        return e;
+    const int64_t grid = L.total_ptiles < sms ? L.total_ptiles : sms;
+    k_prefill<<<(unsigned)(grid < 1 ? 1 : grid), kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace tw

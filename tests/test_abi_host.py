@@ -47,7 +47,8 @@ def test_size_queries(lib):
     assert api.packed_bytes(0, 128) == 0
     assert api.tw_ternarize_workspace_bytes(1536, 1536) % 256 == 0
     assert api.tw_ternarize_workspace_bytes(1536, 1536) >= 256 + 8 * 1536
-    assert api.linear_workspace_bytes(32, 1536, 1536) == 0
+    assert api.linear_workspace_bytes(32, 1536, 1536) == 32 * 1536 + 256
+    assert api.linear_workspace_bytes(1, 8960, 8960) == 8960 + 256
     assert api.linear_workspace_bytes(256, 1536, 1536) >= 256 * 1536 + 2 * 256 * 4
 
 
@@ -64,10 +65,11 @@ def _descs(shapes, base=0x10000):
 REC = np.dtype([("x", "<u8"), ("xq", "<u8"), ("amax", "<u8"), ("qsum", "<u8"),
                 ("packed", "<u8"), ("wscale", "<u8"), ("y", "<u8"), ("acc_out", "<u8"),
                 ("N", "<i8"), ("K", "<i8"), ("rb_begin", "<i8"), ("tile_begin", "<i8"),
-                ("ptile_begin", "<i8"), ("res", "<i8", 3), ("tmap", "u1", 128)])
+                ("ptile_begin", "<i8"), ("ws_xq_off", "<i8"), ("res", "<i8", 2),
+                ("tmap", "u1", 128)])
 HDR = np.dtype([("magic", "<u4"), ("count", "<i4"), ("M", "<i8"), ("total_rb", "<i8"),
                 ("total_tiles", "<i8"), ("total_ptiles", "<i8"), ("max_K", "<i8"),
-                ("sum_K", "<i8"), ("res", "<i8")])
+                ("sum_K", "<i8"), ("ws_bytes", "<i8")])
 
 
 def test_table_encode_prefix_sums(lib):
@@ -89,6 +91,11 @@ def test_table_encode_prefix_sums(lib):
     assert hdr["total_rb"] == sum(nrb) and hdr["total_tiles"] == sum(ntiles)
     assert hdr["max_K"] == 8960 and hdr["sum_K"] == 1536 * 2 + 256 + 8960
     assert recs["N"].tolist() == [s[0] for s in shapes]
+    xq = [-(-K // 128) * 128 for N, K in shapes]   # M = 1 rows, 128-byte aligned
+    assert recs["ws_xq_off"].tolist() == np.concatenate([[0], np.cumsum(xq)[:-1]]).tolist()
+    assert hdr["ws_bytes"] == sum(xq) + 256 * len(shapes)
+    assert api.tw_sweep_workspace_bytes(buf.ctypes.data) == hdr["ws_bytes"]
+    assert api.tw_sweep_launches(buf.ctypes.data) == 2   # quantise + one decode launch
 
 
 @pytest.mark.parametrize("bad,status", [

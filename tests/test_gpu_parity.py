@@ -115,9 +115,8 @@ def _run_linear(api, dev, W, x, N):
 
 
 @pytest.mark.parametrize("M", list(range(1, 34)))
-def test_decode_linear_m_tails(dev, api, M):
-    if M > 32:
-        pytest.skip("M > 32 is the prefill path")
+def test_linear_m_tails(dev, api, M):
+    """M = 1..32 run the decode kernel, M = 33 the tensor-core prefill."""
     N, K = 80, 640   # 5 row blocks, 5 k tiles (a partial 8-tile chunk)
     W = _weights(N, K, 100 + M)
     x = _acts(M, K, 200 + M)
@@ -167,6 +166,41 @@ def test_decode_k_permutation_detector(dev, api):
     assert (acc_s != acc).any()
 
 
+# ------------------------------------------------------------ prefill linear
+@pytest.mark.parametrize("M,N,K", [(33, 80, 640), (128, 256, 128), (129, 257, 256),
+                                   (255, 1536, 1536), (256, 1536, 1536), (257, 300, 1152),
+                                   (1024, 256, 1536), (300, 8960, 1536), (64, 1536, 8960),
+                                   (40, 1, 128), (200, 30, 384)])
+def test_prefill_linear_shapes(dev, api, M, N, K):
+    W = _weights(N, K, 7 * M + N + K)
+    x = _acts(M, K, 11 * M + K)
+    y, acc = _run_linear(api, dev, W, x, N)
+    codes, mean = orc.ternarize(W)
+    ref = orc.ternary_linear(x, codes, mean)
+    assert (acc == ref["acc"]).all(), f"{M}x{N}x{K}: {(acc != ref['acc']).sum()} accumulators off"
+    G.assert_y_close(y, ref["y"], f"{M}x{N}x{K}")
+
+
+def test_prefill_linear_q_and_zero_rows(dev, api):
+    """Pre-quantised entry point; an all-zero token row gives zeros."""
+    import torch
+    M, N, K = 150, 512, 1024
+    W = _weights(N, K, 77)
+    x = _acts(M, K, 78)
+    x[5] = 0.0
+    packed, _, wscale = G.ternarize_gpu(W, dev)
+    xq, amax, qsum = api.quantize_act(G.to_dev(x, dev))
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+    acc = torch.full((M, N), int(POISON_I32), dtype=torch.int32, device=dev)
+    api.ternary_linear_q(xq, amax, qsum, packed, wscale, N, y=y, acc_out=acc)
+    api.check()
+    codes, mean = orc.ternarize(W)
+    ref = orc.ternary_linear(x, codes, mean)
+    assert (acc.cpu().numpy() == ref["acc"]).all()
+    G.assert_y_close(y.cpu().numpy(), ref["y"])
+    assert not y.cpu().numpy()[5].any()
+
+
 # ------------------------------------------------------------ sweep
 def _sweep_case(api, dev, layers, M, seed_base=0):
     import torch
@@ -178,7 +212,10 @@ def _sweep_case(api, dev, layers, M, seed_base=0):
         xd = G.to_dev(x, dev)
         y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
         acc = torch.full((M, N), int(POISON_I32), dtype=torch.int32, device=dev)
-        descs.append(dict(x=xd, packed=packed, wscale=wscale, y=y, acc_out=acc, N=N, K=K))
+        d = dict(x=xd, packed=packed, wscale=wscale, y=y, acc_out=acc, N=N, K=K)
+        if M > 32:   # prefill sweeps take pre-quantised activations
+            d["xq"], d["amax"], d["qsum"] = api.quantize_act(xd)
+        descs.append(d)
         keep.append((W, x))
     table = api.SweepTable(descs, M, device=dev)
     api.decoder_projection_sweep(table)
@@ -186,7 +223,7 @@ def _sweep_case(api, dev, layers, M, seed_base=0):
     return descs, keep
 
 
-@pytest.mark.parametrize("M", [1, 4, 8, 16, 32])
+@pytest.mark.parametrize("M", [1, 4, 8, 16, 32, 33, 256])
 def test_sweep_one_layer(dev, api, M):
     descs, keep = _sweep_case(api, dev, 1, M, seed_base=M)
     for d, (W, x) in zip(descs, keep):
