@@ -102,6 +102,30 @@ TW_API int tw_ternarize_pack(const float *W, int64_t N, int64_t K, void *packed,
                       void *ws, size_t ws_bytes, tw_stream_t stream);
 
 /*
+ * tw_ternarize_pack without scratch arguments, for callers that cannot
+ * allocate device memory when they need a matrix packed (for example a
+ * plugin inside a host framework that owns the device-memory budget and
+ * gives its plugins no allocator, or a loop that must not call cudaMalloc
+ * because it may synchronise the device).  The pages have no counterpart of
+ * this entry point; it exists only for such callers.
+ *
+ * Same results as tw_ternarize_pack.  Its scratch (256 + 8*N bytes) lives
+ * in a fixed device array inside the library, sized for N <= TW_NOALLOC_MAX_N
+ * rows; every GPU that loads the library keeps that array (262,400 bytes)
+ * until the process exits.  Larger N returns TW_ERR_SHAPE.  The first call
+ * on a device looks the array's device address up (cudaGetSymbolAddress);
+ * make that first call before any stream capture.  All calls on a device
+ * share the one array, so calls that may run at the same time on the GPU
+ * (different streams, no ordering between them) race and corrupt each
+ * other's results; order them on one stream.  Allocates no memory.
+ */
+#define TW_NOALLOC_MAX_N 32768
+TW_API int tw_ternarize_pack_noalloc(const float *W, int64_t N, int64_t K,
+                                     void *packed, size_t packed_bytes,
+                                     double *mean_abs, float *wscale,
+                                     tw_stream_t stream);
+
+/*
  * Debug / parity: unpack codes to int8 {-1, 0, 1} row-major [N x K].
  * invalid_count (device, one int32, may be NULL) receives the number of
  * 2-bit fields holding the invalid pattern 3 (those codes are written as 0).

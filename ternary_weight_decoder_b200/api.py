@@ -50,6 +50,9 @@ tw_packed_bytes = _sig("tw_packed_bytes", _sz, [_i64, _i64])
 tw_ternarize_workspace_bytes = _sig("tw_ternarize_workspace_bytes", _sz, [_i64, _i64])
 tw_ternarize_pack = _sig("tw_ternarize_pack", _int,
                          [_p, _i64, _i64, _p, _sz, _p, _p, _p, _sz, _p])
+tw_ternarize_pack_noalloc = _sig("tw_ternarize_pack_noalloc", _int,
+                                 [_p, _i64, _i64, _p, _sz, _p, _p, _p])
+NOALLOC_MAX_N = 32768
 tw_unpack_codes = _sig("tw_unpack_codes", _int, [_p, _i64, _i64, _p, _p, _p])
 tw_quantize_act = _sig("tw_quantize_act", _int, [_p, _i64, _i64, _p, _p, _p, _p])
 tw_linear_workspace_bytes = _sig("tw_linear_workspace_bytes", _sz, [_i64, _i64, _i64])
@@ -117,6 +120,25 @@ def ternarize_pack(W: torch.Tensor, stream=None):
     ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
     _raise(tw_ternarize_pack(_ptr(W), N, K, _ptr(packed), packed.numel(), _ptr(mean_abs),
                              _ptr(wscale), _ptr(ws), wsb, _stream(stream)))
+    return packed, mean_abs[:1], wscale[:1]
+
+
+def ternarize_pack_noalloc(W: torch.Tensor, packed=None, mean_abs=None, wscale=None,
+                           stream=None):
+    """Like ternarize_pack, through the entry point that takes no scratch
+    (for callers that cannot allocate device memory at the call site).
+    Outputs may be passed in pre-allocated; N <= NOALLOC_MAX_N."""
+    _need(W, torch.float32, "W")
+    N, K = W.shape
+    dev = W.device
+    if packed is None:
+        packed = torch.empty(max(packed_bytes(N, K), 16), dtype=torch.uint8, device=dev)
+    if mean_abs is None:
+        mean_abs = torch.empty(2, dtype=torch.float64, device=dev)
+    if wscale is None:
+        wscale = torch.empty(4, dtype=torch.float32, device=dev)
+    _raise(tw_ternarize_pack_noalloc(_ptr(W), N, K, _ptr(packed), packed.numel(),
+                                     _ptr(mean_abs), _ptr(wscale), _stream(stream)))
     return packed, mean_abs[:1], wscale[:1]
 
 
