@@ -261,14 +261,12 @@ def main():
 
     M = args.m
     shapes, descs, x_host, x_all, y_all = build_workload(api, torch, dev, M, args.layers, rank)
-    table = api.SweepTable(descs, M, device=dev)
-    algo_bytes, algo_codes, _ = sweep_bytes(shapes, M)
-    launches_per_step = table.launches
     if M > 32:   # prefill sweeps consume int8 activations quantised beforehand
         for d in descs:
             d["xq"], d["amax"], d["qsum"] = api.quantize_act(d["x"])
-        table = api.SweepTable(descs, M, device=dev)
-        launches_per_step = table.launches
+    table = api.SweepTable(descs, M, device=dev)
+    algo_bytes, algo_codes, _ = sweep_bytes(shapes, M)
+    launches_per_step = table.launches
 
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):

@@ -348,6 +348,8 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
         max_K = s.K > max_K ? s.K : max_K;
         sum_K += s.K;
     }
+    if (rb > INT32_MAX || tiles > ((int64_t)1 << 40))
+        return fail(TW_ERR_SHAPE, "sweep too large: %lld row blocks", (long long)rb);
     hdr->magic = tw::kTableMagic;
     hdr->count = count;
     hdr->M = M;

@@ -14,14 +14,15 @@
 // with amax/127 and sum(q).  It lets launch 2 start at once (programmatic
 // dependent launch), so the weight stream below overlaps it.
 //
-// Launch 2 (k_decode), one CTA per SM, 9 warps:
+// Launch 2 (k_decode), one CTA per SM:
 //   * The grid splits the concatenated 16-row blocks of all projections into
 //     equal shares of packed bytes; each CTA streams its share once.
-//   * Warps 0..7 (consumer warps) each own every 8th row block of the share
-//     and keep a private ring of 4 KB slots that they fill with 1-D bulk
-//     copies (the TMA engine) several chunks ahead, so the codes stream from
-//     HBM independently of the arithmetic.
-//   * Warp 8 (activation warp) waits for launch 1, then bulk-copies each
+//   * NC consumer warps (15 for up to 8 tokens, 11 or 7 for more) each own
+//     every NC-th row block of the share and keep a private ring of 4 KB
+//     slots that they fill with 1-D bulk copies (the TMA engine) ahead of
+//     the arithmetic; a slot is refilled as soon as its tiles are in
+//     registers, so the codes stream from HBM independently of the math.
+//   * The last warp (activation warp) waits for launch 1, then bulk-copies each
 //     projection's int8 rows, amax/127 and sum(q) into one of up to four
 //     shared-memory buffers ahead of the consumers.
 //   * Codes are decoded in registers with one AND per register:
@@ -40,8 +41,6 @@
 namespace tw {
 namespace {
 
-constexpr int kNC = 8;                      // consumer warps
-constexpr int kThreads = (kNC + 1) * 32;    // + activation warp
 constexpr int kCT = 8;                      // tiles per ring chunk
 constexpr int kChunk = kCT * kTileBytes;    // 4 KB
 constexpr int kMaxXB = 4;                   // activation buffers
@@ -222,17 +221,22 @@ __device__ int desc_of_rb(const DecodeParams &p, int64_t rb)
     return lo;
 }
 
-// Walks the chunks of one consumer warp: every kNC-th row block of the CTA
-// share, each cut into ceil(KT / kCT) chunks.
+// Walks the chunks of one consumer warp: every NC-th row block of the CTA
+// share, each cut into ceil(KT / kCT) chunks.  The fields of the current
+// projection are cached here so that issuing a chunk reads no global memory.
+template <int NC>
 struct ChunkIter {
-    int64_t rb, rb_end, rb_hi;
+    const uint8_t *packed;
+    int rb, rb_begin, rb_end, rb_hi;   // row-block indices (< 2^31)
     int d, kc, nch, KT;
     bool valid;
 
     __device__ void load_desc(const DecodeParams &p)
     {
         const DescRecord &r = rec(p, d);
-        rb_end = r.rb_begin + rb_count(r);
+        packed = r.packed;
+        rb_begin = (int)r.rb_begin;
+        rb_end = (int)(r.rb_begin + rb_count(r));
         KT = (int)(r.K / kTileK);
         nch = (KT + kCT - 1) / kCT;
     }
@@ -245,8 +249,8 @@ struct ChunkIter {
     }
     __device__ void init(const DecodeParams &p, const Plan &pl, int w)
     {
-        rb = pl.rb_lo + w;
-        rb_hi = pl.rb_hi;
+        rb = (int)pl.rb_lo + w;
+        rb_hi = (int)pl.rb_hi;
         kc = 0;
         valid = rb < rb_hi;
         if (valid) {
@@ -260,24 +264,22 @@ struct ChunkIter {
         if (++kc < nch)
             return;
         kc = 0;
-        rb += kNC;
+        rb += NC;
         valid = rb < rb_hi;
         if (valid)
             seek(p);
     }
+    // Bulk-copy this chunk's tiles into dst, completing on bar.
+    __device__ __forceinline__ void issue(uint32_t dst, uint32_t bar) const
+    {
+        const int kt0 = kc * kCT;
+        const int n = min(kCT, KT - kt0);
+        const uint8_t *src =
+            packed + ((int64_t)(rb - rb_begin) * KT + kt0) * (int64_t)kTileBytes;
+        mbar_arrive_expect_tx(bar, (uint32_t)(n * kTileBytes));
+        bulk_g2s(dst, src, (uint32_t)(n * kTileBytes), bar);
+    }
 };
-
-__device__ __forceinline__ void issue_chunk(const DecodeParams &p, const ChunkIter &it,
-                                            uint32_t dst, uint32_t bar)
-{
-    const DescRecord &r = rec(p, it.d);
-    const int kt0 = it.kc * kCT;
-    const int n = min(kCT, it.KT - kt0);
-    const uint8_t *src =
-        r.packed + ((it.rb - r.rb_begin) * (int64_t)it.KT + kt0) * (int64_t)kTileBytes;
-    mbar_arrive_expect_tx(bar, (uint32_t)(n * kTileBytes));
-    bulk_g2s(dst, src, (uint32_t)(n * kTileBytes), bar);
-}
 
 // D(16x8, s32) += A(16x32, u8, row) * B(32x8, s8, col).
 __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -319,15 +321,16 @@ __device__ __forceinline__ void tile_mma(int (&acc)[NT][4][4], const uint4 &a,
     }
 }
 
-template <int NT>
-__global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ DecodeParams p)
+template <int NT, int NC>
+__global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_constant__ DecodeParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
+    constexpr int kThr = (NC + 1) * 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // Layout: rings | zero row (at 64 mod 128) | activation buffers (rows at
     // 0 mod 128, stride xs = 64 mod 128) | token info | barriers | plan.
-    const int ring_bytes = kNC * p.slots * kChunk;
+    const int ring_bytes = NC * p.slots * kChunk;
     uint8_t *ring = smem;
     uint8_t *zero_row = smem + ring_bytes + 64;
     uint8_t *xbase = smem + ring_bytes + 64 + p.xs;  // = ring + K + 128: 0 mod 128
@@ -336,18 +339,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     misc += (128 - (smem_u32(misc) & 127)) & 127;
     uint8_t *info = misc;                                    // [xb][256]: sa[32], qs[32]
     uint64_t *bars = reinterpret_cast<uint64_t *>(misc + 256 * kMaxXB);
-    // bars: ring_full[kNC*slots], x_full[kMaxXB], x_empty[kMaxXB]
-    Plan *plan = reinterpret_cast<Plan *>(misc + 256 * kMaxXB + 8 * (kNC * p.slots + 2 * kMaxXB));
+    // bars: ring_full[NC*slots], x_full[kMaxXB], x_empty[kMaxXB]
+    Plan *plan = reinterpret_cast<Plan *>(misc + 256 * kMaxXB + 8 * (NC * p.slots + 2 * kMaxXB));
     const uint32_t bar_ring = smem_u32(bars);
-    const uint32_t bar_xfull = bar_ring + 8 * kNC * p.slots;
+    const uint32_t bar_xfull = bar_ring + 8 * NC * p.slots;
     const uint32_t bar_xempty = bar_xfull + 8 * kMaxXB;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNC * p.slots; ++i)
+        for (int i = 0; i < NC * p.slots; ++i)
             mbar_init(bar_ring + 8 * i, 1);
         for (int b = 0; b < kMaxXB; ++b) {
             mbar_init(bar_xfull + 8 * b, 1);
-            mbar_init(bar_xempty + 8 * b, kNC * 32);
+            mbar_init(bar_xempty + 8 * b, NC * 32);
         }
         fence_barrier_init();
         const int G = gridDim.x, c = blockIdx.x;
@@ -362,13 +365,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             plan->d_hi = -1;
         }
     }
-    for (int i = threadIdx.x; i < p.xs / 16; i += kThreads)
+    for (int i = threadIdx.x; i < p.xs / 16; i += kThr)
         reinterpret_cast<uint4 *>(zero_row)[i] = make_uint4(0, 0, 0, 0);
     __syncthreads();
     const Plan pl = *plan;
     volatile int *abort_flag = &plan->abort_flag;
 
-    if (warp == kNC) {
+    if (warp == NC) {
         // ------------------------------------------------ activation warp
         if (lane == 0) {
             pdl_wait();  // launch 1 has finished writing the int8 rows
@@ -400,20 +403,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
 
     // ---------------------------------------------------- consumer warps
     const int g = lane >> 2, t = lane & 3;
-    const uint32_t ring_w = smem_u32(ring) + warp * p.slots * kChunk;
-    const uint32_t bar_w = bar_ring + 8 * warp * p.slots;
+    const int S = p.slots;
+    const uint32_t ring_w = smem_u32(ring) + warp * S * kChunk + lane * 16;  // this lane's slot
+    const uint32_t ring_w0 = smem_u32(ring) + warp * S * kChunk;
+    const uint32_t bar_w = bar_ring + 8 * warp * S;
     const uint32_t zero_s = smem_u32(zero_row);
 
-    ChunkIter cons, prod;
+    ChunkIter<NC> cons, prod;
     cons.init(p, pl, warp);
     prod = cons;
     int issued = 0, consumed = 0;
-    for (int s = 0; s < p.slots && prod.valid; ++s) {
+    for (int s = 0; s < S && prod.valid; ++s) {
         if (lane == 0)
-            issue_chunk(p, prod, ring_w + s * kChunk, bar_w + 8 * s);
+            prod.issue(ring_w0 + s * kChunk, bar_w + 8 * s);
         prod.next(p);
         ++issued;
     }
+    int cslot = 0;
+    uint32_t cphase = 0;
 
     bool ok = true;
     for (int d = pl.d_lo; d <= pl.d_hi && ok; ++d) {
@@ -422,8 +429,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             ok = false;
             break;
         }
+        // this projection's fields, read once
         const DescRecord &r = rec(p, d);
         const float wscale = __ldg(r.wscale);
+        const int64_t N = r.N, rbeg = r.rb_begin;
+        float *const y = r.y;
+        int32_t *const acc_out = r.acc_out;
         const float *sa = reinterpret_cast<const float *>(info + 256 * b);
         const int *qs = reinterpret_cast<const int *>(info + 256 * b + 128);
         uint32_t xrow[NT];
@@ -446,57 +457,57 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
             const int64_t rb = cons.rb;
             const int nch = cons.nch, KT = cons.KT;  // cons moves on after the last chunk
             for (int kc = 0; kc < nch; ++kc) {
-                const int slot = consumed % p.slots;
-                if (!mbar_wait(bar_w + 8 * slot, (consumed / p.slots) & 1, p.ctl, abort_flag)) {
+                if (!mbar_wait(bar_w + 8 * cslot, cphase, p.ctl, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const int kt0 = kc * kCT;
-                const int n = min(kCT, KT - kt0);
-                const uint32_t src = ring_w + slot * kChunk + lane * 16;
-                const uint32_t kbase = (uint32_t)kt0 * kTileK;
-                if (n == kCT) {
-                    uint4 a[kCT];
+                const int n = min(kCT, KT - kc * kCT);
+                // All 8 lane slots of the chunk go to registers (slots past n
+                // hold stale bytes and are not used) ...
+                uint4 a[kCT];
 #pragma unroll
-                    for (int i = 0; i < kCT; ++i)
-                        a[i] = lds128(src + i * kTileBytes);
-#pragma unroll
-                    for (int i = 0; i < kCT; ++i)
-                        tile_mma<NT>(acc, a[i], xrow, kbase + i * kTileK);
-                } else {
-                    for (int i = 0; i < n; ++i)
-                        tile_mma<NT>(acc, lds128(src + i * kTileBytes), xrow, kbase + i * kTileK);
-                }
+                for (int i = 0; i < kCT; ++i)
+                    a[i] = lds128(ring_w + cslot * kChunk + i * kTileBytes);
+                // ... so the slot is refilled before the arithmetic starts.
                 __syncwarp();
-                ++consumed;
                 if (prod.valid) {
                     if (lane == 0) {
                         fence_proxy_async_smem();
-                        issue_chunk(p, prod, ring_w + slot * kChunk, bar_w + 8 * slot);
+                        prod.issue(ring_w0 + cslot * kChunk, bar_w + 8 * cslot);
                     }
                     prod.next(p);
                     ++issued;
                 }
+                ++consumed;
+                if (++cslot == S) {
+                    cslot = 0;
+                    cphase ^= 1u;
+                }
+                const uint32_t kbase = (uint32_t)(kc * kCT * kTileK);
+#pragma unroll
+                for (int i = 0; i < kCT; ++i)
+                    if (i < n)
+                        tile_mma<NT>(acc, a[i], xrow, kbase + i * kTileK);
                 cons.next(p);
             }
             if (!ok)
                 break;
             // epilogue of row block rb: rows 16*rl + g (+8), tokens 8nt + 2t (+1)
-            const int64_t rl = rb - r.rb_begin;
+            const int64_t rl = rb - rbeg;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int tok = 8 * nt + 2 * t + (i & 1);
                     const int64_t row = rl * kTileRows + g + 8 * (i >> 1);
-                    if (tok < p.mg && row < r.N) {
+                    if (tok < p.mg && row < N) {
                         const int m = p.m0 + tok;  // sa/qs hold all M tokens
                         const int v = acc[nt][0][i] + (acc[nt][1][i] >> 2) +
                                       (acc[nt][2][i] >> 4) + (acc[nt][3][i] >> 6) - qs[m];
-                        const int64_t o = (int64_t)m * r.N + row;
-                        r.y[o] = __fmul_rn(__fmul_rn((float)v, sa[m]), wscale);
-                        if (r.acc_out)
-                            r.acc_out[o] = v;
+                        const int64_t o = (int64_t)m * N + row;
+                        y[o] = __fmul_rn(__fmul_rn((float)v, sa[m]), wscale);
+                        if (acc_out)
+                            acc_out[o] = v;
                     }
                 }
             }
@@ -511,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         WaitCtl drain = p.ctl;
         drain.timeout_ns = kDrainNs;
         for (int i = consumed; i < issued; ++i)
-            mbar_wait(bar_w + 8 * (i % p.slots), (i / p.slots) & 1, drain, nullptr);
+            mbar_wait(bar_w + 8 * (i % S), (i / S) & 1, drain, nullptr);
     }
 }
 
@@ -527,17 +538,27 @@ __global__ void k_wait_probe(WaitCtl ctl)
     mbar_wait(b, 0, ctl, nullptr);  // nothing arrives: must time out
 }
 
+// Consumer warps per block: more warps hide more latency, fewer leave
+// registers for the wider accumulators of larger token groups.
+// The block is a multiple of 4 warps so that each SM sub-partition's
+// register file holds the same number of warps (16, 12 or 8 in total).
+template <int NT>
+constexpr int consumers() { return NT == 1 ? 15 : NT == 2 ? 11 : 7; }
+
+int consumers_for(int mg) { const int nt = (mg + 7) / 8; return nt == 1 ? 15 : nt == 2 ? 11 : 7; }
+
 template <int NT>
 cudaError_t launch_nt(const DecodeParams &p, int grid, int smem, cudaStream_t stream)
 {
-    cudaError_t e = cudaFuncSetAttribute(k_decode<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
+    constexpr int NC = consumers<NT>();
+    cudaError_t e = cudaFuncSetAttribute(k_decode<NT, NC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return e;
     // Programmatic dependent launch: may start while k_quant_rows runs.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3((NC + 1) * 32);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -545,28 +566,36 @@ cudaError_t launch_nt(const DecodeParams &p, int grid, int smem, cudaStream_t st
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_decode<NT>, p);
+    return cudaLaunchKernelEx(&cfg, k_decode<NT, NC>, p);
 }
 
 // Bytes of dynamic shared memory of k_decode for this plan.
-int64_t smem_bytes(int slots, int mg, int xb, int64_t max_K)
+int64_t smem_bytes(int nc, int slots, int mg, int xb, int64_t max_K)
 {
     const int64_t xs = max_K + 64;
-    return 1024 + (int64_t)kNC * slots * kChunk + xs + 128 + (int64_t)xb * mg * xs + 256 +
+    return 1024 + (int64_t)nc * slots * kChunk + xs + 128 + (int64_t)xb * mg * xs + 256 +
            kMiscBytes;
 }
 
-// Largest token group (and its ring depth) that fits shared memory.
-bool plan_groups(int M, int64_t max_K, int *mg_out, int *slots_out)
+// Largest token group, then deepest ring (4..2 slots, 3..2 with 15 warps),
+// then most activation buffers (at least 2 when that fits) for the budget.
+bool plan_decode(int M, int64_t max_K, int *mg_out, int *slots_out, int *xb_out)
 {
     int mg = M;
     while (true) {
-        for (int s = 4; s >= 2; --s)
-            if (smem_bytes(s, mg, 1, max_K) <= kSmemLimit) {
-                *mg_out = mg;
-                *slots_out = s;
-                return true;
-            }
+        const int nc = consumers_for(mg);
+        const int smax = nc >= 15 ? 3 : 4;
+        for (int need_xb = 2; need_xb >= 1; --need_xb)
+            for (int s = smax; s >= 2; --s)
+                if (smem_bytes(nc, s, mg, need_xb, max_K) <= kSmemLimit) {
+                    int xb = need_xb;
+                    while (xb < kMaxXB && smem_bytes(nc, s, mg, xb + 1, max_K) <= kSmemLimit)
+                        ++xb;
+                    *mg_out = mg;
+                    *slots_out = s;
+                    *xb_out = xb;
+                    return true;
+                }
         if (mg == 1)
             return false;
         mg = mg > 8 ? mg - 8 : mg - 1;
@@ -577,8 +606,8 @@ bool plan_groups(int M, int64_t max_K, int *mg_out, int *slots_out)
 
 int decode_launches(int64_t M, int64_t max_K)
 {
-    int mg = 1, slots = 2;
-    if (!plan_groups((int)M, max_K, &mg, &slots))
+    int mg = 1, slots = 2, xb = 1;
+    if (!plan_decode((int)M, max_K, &mg, &slots, &xb))
         return 0;
     return 1 + (int)((M + mg - 1) / mg);  // quantise + one decode launch per group
 }
@@ -593,12 +622,9 @@ cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout
     if (e != cudaSuccess)
         return e;
     const int M = (int)L.M;
-    int mg = 1, slots = 2;
-    if (!plan_groups(M, L.max_K, &mg, &slots))
+    int mg = 1, slots = 2, xb = 1;
+    if (!plan_decode(M, L.max_K, &mg, &slots, &xb))
         return cudaErrorInvalidValue;
-    int xb = 1;
-    while (xb < kMaxXB && smem_bytes(slots, mg, xb + 1, L.max_K) <= kSmemLimit)
-        ++xb;
 
     // Launch 1: quantise every (projection, token) row.
     QuantParams q;
@@ -631,7 +657,7 @@ cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout
     p.ctl.timeout_ns = timeout_ns;
     p.slots = slots;
     p.xb = xb;
-    const int smem = (int)smem_bytes(slots, mg, xb, L.max_K);
+    const int smem = (int)smem_bytes(consumers_for(mg), slots, mg, xb, L.max_K);
     const int64_t grid64 = L.total_rb < sms ? L.total_rb : sms;
     const int grid = (int)(grid64 < 1 ? 1 : grid64);
 
