@@ -119,6 +119,13 @@ __device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void *src, uin
         : "memory");
 }
 
+// Bulk prefetch of [src, src + bytes) from global memory into L2 (no
+// shared-memory destination, no completion tracking).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first()
 {
     uint64_t p;

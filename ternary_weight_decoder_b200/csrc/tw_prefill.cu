@@ -13,7 +13,8 @@
 // page, "Layout".)
 //
 // Tile: 128 tokens x 256 weight rows, K in stages of 128 (one swizzle atom),
-// four MMAs of K = 32 per stage.  Persistent: one CTA per SM walks the
+// four MMAs of K = 32 per stage; four stages of A + code tiles in flight,
+// three expanded B tiles.  Persistent: one CTA per SM walks the
 // output tiles of every projection (all token tiles of a weight tile run
 // back to back across the grid, so the weight codes stream from HBM once
 // and the activations stay in L2).  Two TMEM accumulators let the epilogue
@@ -35,14 +36,18 @@ namespace {
 constexpr int kBM = 128;                 // tokens per tile (MMA M)
 constexpr int kBN = 256;                 // weight rows per tile (MMA N)
 constexpr int kBK = 128;                 // k per stage
-constexpr int kStages = 4;
+constexpr int kLoadStages = 4;           // A + code tiles in flight
+constexpr int kBStages = 3;              // expanded B tiles
 constexpr int kABytes = kBM * kBK;       // 16 KB
 constexpr int kBBytes = kBN * kBK;       // 32 KB
 constexpr int kCodeBytes = kBN / kTileRows * kTileBytes;  // 16 tiles = 8 KB
-constexpr int kStageBytes = kABytes + kBBytes + kCodeBytes;
+constexpr int kLoadBytes = kABytes + kCodeBytes;
 constexpr int kNumExp = 8;               // expansion warps
 constexpr int kThreads = (6 + kNumExp) * 32;
 constexpr int kTmemCols = 512;           // two 256-column accumulators
+constexpr int kStageRowF = 36;           // epilogue staging row (floats), 32 + 4 pad
+constexpr int kStagingBytes = 4 * 32 * kStageRowF * 4;
+constexpr int kSmemBytes = 1024 + kLoadStages * kLoadBytes + kBStages * kBBytes + kStagingBytes + 1024;
 constexpr uint64_t kDrainNs = 1000000000ull;
 
 struct PrefillParams {
@@ -59,27 +64,50 @@ __device__ __forceinline__ const DescRecord &prec(const PrefillParams &p, int d)
     return p.table ? p.table[d] : p.single;
 }
 
-// Output tile t -> projection d, token tile mi, weight tile nj.  Inside a
-// projection the token tiles of one weight tile are consecutive.
-struct TileCoord {
+// Walks this CTA's output tiles t = blockIdx.x, +G, ... in order, keeping
+// the fields of the current projection in registers (no search per tile).
+// Inside a projection the token tiles of one weight tile are consecutive:
+// local tile = nj * tm + mi.
+struct TileIter {
+    int64_t t, ptile_end, tm;
     int d;
-    int64_t mi, nj;
-};
+    int64_t mi, nj, K, N;
+    const DescRecord *r;
 
-__device__ TileCoord tile_coord(const PrefillParams &p, int64_t t)
-{
-    int lo = 0, hi = p.count - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (prec(p, mid).ptile_begin <= t)
-            lo = mid;
-        else
-            hi = mid - 1;
+    __device__ void load(const PrefillParams &p)
+    {
+        r = &prec(p, d);
+        K = r->K;
+        N = r->N;
+        ptile_end = r->ptile_begin + tm * ((N + kBN - 1) / kBN);
     }
-    const int64_t tm = (p.M + kBM - 1) / kBM;
-    const int64_t local = t - prec(p, lo).ptile_begin;
-    return TileCoord{lo, local % tm, local / tm};
-}
+    __device__ void locate(const PrefillParams &p)
+    {
+        while (t >= ptile_end && d + 1 < p.count) {
+            ++d;
+            load(p);
+        }
+        const int64_t local = t - r->ptile_begin;
+        mi = local % tm;
+        nj = local / tm;
+    }
+    __device__ void init(const PrefillParams &p, int64_t t0)
+    {
+        t = t0;
+        tm = (p.M + kBM - 1) / kBM;
+        d = 0;
+        load(p);
+        if (t < p.total_ptiles)
+            locate(p);
+    }
+    __device__ bool valid(const PrefillParams &p) const { return t < p.total_ptiles; }
+    __device__ void next(const PrefillParams &p, int64_t G)
+    {
+        t += G;
+        if (t < p.total_ptiles)
+            locate(p);
+    }
+};
 
 // ------------------------------------------------------------- tcgen05 PTX
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
@@ -169,10 +197,14 @@ constexpr uint32_t kIdesc = (2u << 4)            // D format: s32
                             | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 
 struct SmemLayout {
-    uint32_t base;  // 1024-aligned shared address of stage 0
-    __device__ uint32_t a(int s) const { return base + s * kStageBytes; }
-    __device__ uint32_t b(int s) const { return base + s * kStageBytes + kABytes; }
-    __device__ uint32_t codes(int s) const { return base + s * kStageBytes + kABytes + kBBytes; }
+    uint32_t base;  // 1024-aligned shared address
+    __device__ uint32_t a(int s) const { return base + s * kLoadBytes; }
+    __device__ uint32_t codes(int s) const { return base + s * kLoadBytes + kABytes; }
+    __device__ uint32_t b(int s) const { return base + kLoadStages * kLoadBytes + s * kBBytes; }
+    __device__ uint32_t staging(int w) const
+    {
+        return base + kLoadStages * kLoadBytes + kBStages * kBBytes + w * (32 * kStageRowF * 4);
+    }
 };
 
 __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__ PrefillParams p)
@@ -182,12 +214,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gen_base = smem_raw + (base - raw);
     SmemLayout L{base};
-    uint8_t *misc = gen_base + kStages * kStageBytes;
+    uint8_t *misc = gen_base + kLoadStages * kLoadBytes + kBStages * kBBytes + kStagingBytes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(misc);
-    // barriers: load_full[S], exp_full[S], empty[S], tmem_full[2], tmem_empty[2], drain
+    // barriers: ld_full[4], ld_empty[4], b_full[3], b_empty[3], tmem_full[2],
+    // tmem_empty[2], drain
     const uint32_t bar0 = smem_u32(bars);
-    const uint32_t b_load = bar0, b_exp = bar0 + 8 * kStages, b_empty = bar0 + 16 * kStages;
-    const uint32_t b_tfull = bar0 + 24 * kStages, b_tempty = b_tfull + 16;
+    const uint32_t b_ldfull = bar0, b_ldempty = bar0 + 8 * kLoadStages;
+    const uint32_t b_bfull = bar0 + 16 * kLoadStages, b_bempty = b_bfull + 8 * kBStages;
+    const uint32_t b_tfull = b_bempty + 8 * kBStages, b_tempty = b_tfull + 16;
     const uint32_t b_drain = b_tempty + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 512);
     int *abort_flag_p = reinterpret_cast<int *>(misc + 520);
@@ -195,10 +229,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(b_load + 8 * s, 1);
-            mbar_init(b_exp + 8 * s, kNumExp * 32);
-            mbar_init(b_empty + 8 * s, 1);
+        for (int s = 0; s < kLoadStages; ++s) {
+            mbar_init(b_ldfull + 8 * s, 1);
+            mbar_init(b_ldempty + 8 * s, 1);
+        }
+        for (int s = 0; s < kBStages; ++s) {
+            mbar_init(b_bfull + 8 * s, kNumExp * 32);
+            mbar_init(b_bempty + 8 * s, 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(b_tfull + 8 * a, 1);
@@ -214,53 +251,56 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
     const int64_t G = gridDim.x;
-    const int64_t ntiles = p.total_ptiles;
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
             int64_t it = 0;
-            for (int64_t t = blockIdx.x; t < ntiles && !*abort_flag; t += G) {
-                const TileCoord c = tile_coord(p, t);
-                const DescRecord &r = prec(p, c.d);
-                const int64_t KT = r.K / kBK;
-                const int64_t nrb = (r.N + kTileRows - 1) / kTileRows;
-                const int64_t rb0 = c.nj * (kBN / kTileRows);
+            TileIter ti;
+            for (ti.init(p, blockIdx.x); ti.valid(p) && !*abort_flag; ti.next(p, G)) {
+                const int64_t KT = ti.K / kBK;
+                const int64_t nrb = (ti.N + kTileRows - 1) / kTileRows;
+                const int64_t rb0 = ti.nj * (kBN / kTileRows);
                 const int nct = (int)min((int64_t)(kBN / kTileRows), nrb - rb0);
                 const uint32_t bytes = kABytes + nct * kTileBytes;
+                const uint8_t *codes0 = ti.r->packed + rb0 * KT * kTileBytes;
+                const void *tmap = ti.r->tmap_xq;
+                const int32_t ycoord = (int32_t)(ti.mi * kBM);
+                bool ok = true;
                 for (int64_t kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = (int)(it % kStages);
-                    if (it >= kStages &&
-                        !mbar_wait(b_empty + 8 * s, (uint32_t)((it / kStages - 1) & 1), p.ctl,
-                                   abort_flag))
+                    const int s = (int)(it % kLoadStages);
+                    if (it >= kLoadStages &&
+                        !mbar_wait(b_ldempty + 8 * s, (uint32_t)((it / kLoadStages - 1) & 1), p.ctl,
+                                   abort_flag)) {
+                        ok = false;
                         break;
-                    mbar_arrive_expect_tx(b_load + 8 * s, bytes);
-                    tma_load_2d(L.a(s), r.tmap_xq, (int32_t)(kt * kBK), (int32_t)(c.mi * kBM),
-                                b_load + 8 * s);
+                    }
+                    mbar_arrive_expect_tx(b_ldfull + 8 * s, bytes);
+                    tma_load_2d(L.a(s), tmap, (int32_t)(kt * kBK), ycoord, b_ldfull + 8 * s);
                     for (int i = 0; i < nct; ++i)
-                        bulk_g2s(L.codes(s) + i * kTileBytes,
-                                 r.packed + ((rb0 + i) * KT + kt) * kTileBytes, kTileBytes,
-                                 b_load + 8 * s);
+                        bulk_g2s(L.codes(s) + i * kTileBytes, codes0 + (i * KT + kt) * kTileBytes,
+                                 kTileBytes, b_ldfull + 8 * s);
                 }
+                if (!ok)
+                    break;
             }
-            // Drain: the last (up to) kStages loads must land before exit.
+            // Drain: the last (up to) kLoadStages loads must land before exit.
             WaitCtl drain = p.ctl;
             drain.timeout_ns = kDrainNs;
-            for (int64_t j = it - kStages; j < it; ++j)
+            for (int64_t j = it - kLoadStages; j < it; ++j)
                 if (j >= 0)
-                    mbar_wait(b_load + 8 * (int)(j % kStages), (uint32_t)((j / kStages) & 1), drain,
-                              nullptr);
+                    mbar_wait(b_ldfull + 8 * (int)(j % kLoadStages),
+                              (uint32_t)((j / kLoadStages) & 1), drain, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
             int64_t it = 0, tt = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < ntiles && ok; t += G, ++tt) {
-                const TileCoord c = tile_coord(p, t);
-                const int64_t KT = prec(p, c.d).K / kBK;
+            TileIter ti;
+            for (ti.init(p, blockIdx.x); ti.valid(p) && ok; ti.next(p, G), ++tt) {
+                const int64_t KT = ti.K / kBK;
                 const int ab = (int)(tt & 1);
                 if (tt >= 2 && !mbar_wait(b_tempty + 8 * ab, (uint32_t)((tt / 2 - 1) & 1), p.ctl,
                                           abort_flag)) {
@@ -270,20 +310,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(ab * kBN);
                 for (int64_t kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = (int)(it % kStages);
-                    const uint32_t par = (uint32_t)((it / kStages) & 1);
-                    if (!mbar_wait(b_load + 8 * s, par, p.ctl, abort_flag) ||
-                        !mbar_wait(b_exp + 8 * s, par, p.ctl, abort_flag)) {
+                    const int ls = (int)(it % kLoadStages), bs = (int)(it % kBStages);
+                    if (!mbar_wait(b_ldfull + 8 * ls, (uint32_t)((it / kLoadStages) & 1), p.ctl,
+                                   abort_flag) ||
+                        !mbar_wait(b_bfull + 8 * bs, (uint32_t)((it / kBStages) & 1), p.ctl,
+                                   abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t ad = sdesc_k_sw128(L.a(s));
-                    const uint64_t bd = sdesc_k_sw128(L.b(s));
+                    const uint64_t ad = sdesc_k_sw128(L.a(ls));
+                    const uint64_t bd = sdesc_k_sw128(L.b(bs));
 #pragma unroll
                     for (int j = 0; j < kBK / 32; ++j)  // +32 bytes of K = +2 in the address field
                         mma_i8(d_tmem, ad + 2 * j, bd + 2 * j, kIdesc, (kt > 0 || j > 0) ? 1u : 0u);
-                    mma_commit(b_empty + 8 * s);
+                    mma_commit(b_ldempty + 8 * ls);
+                    mma_commit(b_bempty + 8 * bs);
                 }
                 if (!ok)
                     break;
@@ -298,52 +340,78 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
         __syncwarp();
     } else if (warp < 6) {
         // ------------------------------------------------------ epilogue
-        const int quarter = warp & 3;                 // TMEM lanes 32q..32q+31
+        // Each warp owns TMEM lanes 32q..32q+31 (q = warp % 4): 32 token rows
+        // of the tile.  Per 32-column chunk: TMEM -> registers (thread = row),
+        // rescale, registers -> staging (row-major), then staging -> global
+        // with 4 rows x 128 contiguous bytes per store instruction.
+        const int quarter = warp & 3;
+        const uint32_t stg = L.staging(warp - 2);
+        float *stg_f = reinterpret_cast<float *>(gen_base + (stg - base));
         int64_t tt = 0;
-        for (int64_t t = blockIdx.x; t < ntiles; t += G, ++tt) {
-            const TileCoord c = tile_coord(p, t);
-            const DescRecord &r = prec(p, c.d);
+        TileIter ti;
+        for (ti.init(p, blockIdx.x); ti.valid(p); ti.next(p, G), ++tt) {
+            const DescRecord &r = *ti.r;
             const int ab = (int)(tt & 1);
-            if (!mbar_wait(b_tfull + 8 * ab, (uint32_t)((tt / 2) & 1), p.ctl, abort_flag))
-                break;
-            tc_fence_after();
-            const int64_t m = c.mi * kBM + quarter * 32 + lane;
+            const int64_t m_base = ti.mi * kBM + quarter * 32;   // first row of this warp
+            const int64_t m = m_base + lane;
             const bool row_ok = m < p.M;
+            // per-row and per-tensor scales (loaded before the wait)
             const float sa = row_ok ? __fdiv_rn(__ldg(r.amax + m), 127.f) : 0.f;
             const int qs = row_ok ? __ldg(r.qsum + m) : 0;
             const float wscale = __ldg(r.wscale);
-            const int64_t n0 = c.nj * kBN;
+            float *const y = r.y;
+            int32_t *const acc_out = r.acc_out;
+            const int64_t N = ti.N;
+            const int64_t n0 = ti.nj * kBN;
+            if (!mbar_wait(b_tfull + 8 * ab, (uint32_t)((tt / 2) & 1), p.ctl, abort_flag))
+                break;
+            tc_fence_after();
+            const bool vec = (N & 3) == 0;
             for (int cc = 0; cc < kBN / 32; ++cc) {
                 uint32_t v[32];
                 tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * kBN + cc * 32), v);
-                if (!row_ok)
-                    continue;
                 const int64_t nb = n0 + cc * 32;
-                float *yrow = r.y + m * r.N;
-                int32_t *arow = r.acc_out ? r.acc_out + m * r.N : nullptr;
-                if (nb + 32 <= r.N && (r.N & 3) == 0) {
+                if (nb >= N)
+                    continue;  // (uniform across the warp)
+                // pass 0: y, pass 1: acc_out
+                for (int pass = 0; pass < (acc_out ? 2 : 1); ++pass) {
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        int a4[4];
-                        float f4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            a4[e] = (int)v[4 * q + e] - qs;
-                            f4[e] = __fmul_rn(__fmul_rn((float)a4[e], sa), wscale);
+                        float4 f;
+                        int a0 = (int)v[4 * q + 0] - qs, a1 = (int)v[4 * q + 1] - qs;
+                        int a2 = (int)v[4 * q + 2] - qs, a3 = (int)v[4 * q + 3] - qs;
+                        if (pass == 0) {
+                            f = make_float4(__fmul_rn(__fmul_rn((float)a0, sa), wscale),
+                                            __fmul_rn(__fmul_rn((float)a1, sa), wscale),
+                                            __fmul_rn(__fmul_rn((float)a2, sa), wscale),
+                                            __fmul_rn(__fmul_rn((float)a3, sa), wscale));
+                        } else {
+                            f = make_float4(__int_as_float(a0), __int_as_float(a1),
+                                            __int_as_float(a2), __int_as_float(a3));
                         }
-                        *reinterpret_cast<float4 *>(yrow + nb + 4 * q) =
-                            make_float4(f4[0], f4[1], f4[2], f4[3]);
-                        if (arow)
-                            *reinterpret_cast<int4 *>(arow + nb + 4 * q) =
-                                make_int4(a4[0], a4[1], a4[2], a4[3]);
+                        *reinterpret_cast<float4 *>(stg_f + lane * kStageRowF + 4 * q) = f;
                     }
-                } else {
-                    for (int e = 0; e < 32 && nb + e < r.N; ++e) {
-                        const int a = (int)v[e] - qs;
-                        yrow[nb + e] = __fmul_rn(__fmul_rn((float)a, sa), wscale);
-                        if (arow)
-                            arow[nb + e] = a;
+                    __syncwarp();
+                    float *dst = pass == 0 ? y : reinterpret_cast<float *>(acc_out);
+                    if (vec && nb + 32 <= N) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int rr = 4 * i + (lane >> 3), c4 = (lane & 7) * 4;
+                            const int64_t mm = m_base + rr;
+                            if (mm < p.M) {
+                                const float4 f =
+                                    *reinterpret_cast<const float4 *>(stg_f + rr * kStageRowF + c4);
+                                *reinterpret_cast<float4 *>(dst + mm * N + nb + c4) = f;
+                            }
+                        }
+                    } else {
+                        for (int rr = 0; rr < 32; ++rr) {
+                            const int64_t mm = m_base + rr;
+                            if (mm < p.M && nb + lane < N)
+                                dst[mm * N + nb + lane] = stg_f[rr * kStageRowF + lane];
+                        }
                     }
+                    __syncwarp();
                 }
             }
             tc_fence_before();
@@ -354,12 +422,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
         const int e = threadIdx.x - 6 * 32;           // 0..255
         int64_t it = 0;
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < ntiles && ok; t += G) {
-            const TileCoord c = tile_coord(p, t);
-            const int64_t KT = prec(p, c.d).K / kBK;
+        TileIter ti;
+        for (ti.init(p, blockIdx.x); ti.valid(p) && ok; ti.next(p, G)) {
+            const int64_t KT = ti.K / kBK;
             for (int64_t kt = 0; kt < KT; ++kt, ++it) {
-                const int s = (int)(it % kStages);
-                if (!mbar_wait(b_load + 8 * s, (uint32_t)((it / kStages) & 1), p.ctl, abort_flag)) {
+                const int ls = (int)(it % kLoadStages), bs = (int)(it % kBStages);
+                if (!mbar_wait(b_ldfull + 8 * ls, (uint32_t)((it / kLoadStages) & 1), p.ctl,
+                               abort_flag) ||
+                    (it >= kBStages &&
+                     !mbar_wait(b_bempty + 8 * bs, (uint32_t)((it / kBStages - 1) & 1), p.ctl,
+                                abort_flag))) {
                     ok = false;
                     break;
                 }
@@ -370,15 +442,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
                     const int q = e + 256 * h;
                     const int tile = q >> 5, l = q & 31;
                     const int g = l >> 2, tq = l & 3;
-                    const uint4 w = lds128(L.codes(s) + tile * kTileBytes + l * 16);
-                    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+                    const uint4 w = lds128(L.codes(ls) + tile * kTileBytes + l * 16);
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                         const int j = (jj + 2 * (g & 1)) & 3;   // staggered: no bank conflicts
-                        const uint32_t wd = words[j];
+                        const uint32_t wd = j == 0 ? w.x : j == 1 ? w.y : j == 2 ? w.z : w.w;
                         const int row = tile * kTileRows + g + 8 * (j & 1);
                         const int chunk = 4 * (j >> 1) + tq;      // 16-byte chunk of the 128 B row
-                        const uint32_t dst = L.b(s) + row * 128 + ((chunk ^ (row & 7)) << 4);
+                        const uint32_t dst = L.b(bs) + row * 128 + ((chunk ^ (row & 7)) << 4);
                         const uint32_t m3 = 0x03030303u;
                         asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst),
                                      "r"(wd & m3), "r"((wd >> 2) & m3), "r"((wd >> 4) & m3),
@@ -387,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
                     }
                 }
                 fence_proxy_async_smem();  // make the B tile visible to the tensor cores
-                mbar_arrive(b_exp + 8 * s);
+                mbar_arrive(b_bfull + 8 * bs);
             }
         }
     }
@@ -459,7 +530,7 @@ cudaError_t launch_prefill(const PrefillLaunch &L, uint32_t *err, uint64_t timeo
     p.total_ptiles = L.total_ptiles;
     p.ctl.err = err;
     p.ctl.timeout_ns = timeout_ns;
-    const int smem = kStages * kStageBytes + 1024 /*align*/ + 1024 /*misc*/;
+    const int smem = kSmemBytes;
     e = cudaFuncSetAttribute(k_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return e;
