@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "tw_device.cuh"
@@ -94,6 +95,8 @@ int run_prefill_single(const int8_t *xq, const float *amax, const int32_t *qsum,
     r.N = N;
     r.K = K;
     int rc = tw::encode_xq_tmap(xq, M, K, r.tmap_xq);
+    if (!rc)
+        rc = tw::encode_codes_tmap(r.packed, N, K, r.tmap_codes);
     if (rc)
         return fail(TW_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", rc);
     tw::PrefillLaunch L{};
@@ -300,7 +303,9 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
     auto *hdr = static_cast<tw::TableHeader *>(table);
     auto *recs = reinterpret_cast<tw::DescRecord *>(hdr + 1);
     memset(table, 0, tw_sweep_table_bytes(count));
-    int64_t rb = 0, tiles = 0, ptiles = 0, max_K = 0, sum_K = 0, ws_off = 0;
+    int64_t rb = 0, tiles = 0, ptiles = 0, max_K = 0, units = 0;
+    // decode scratch: counters | row flags | int8 rows | scales
+    int64_t ws_off = tw::kWsCtrBytes + tw::round128(4 * (int64_t)count * M);
     for (int d = 0; d < count; ++d) {
         const tw_proj_desc &s = descs[d];
         if (int rc = check_shape(M, s.N, s.K))
@@ -333,20 +338,24 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
         r.ptile_begin = ptiles;
         if (!decode) {
             int rc = tw::encode_xq_tmap(s.xq, M, s.K, r.tmap_xq);
+            if (!rc)
+                rc = tw::encode_codes_tmap(r.packed, s.N, s.K, r.tmap_codes);
             if (rc)
                 return fail(TW_ERR_CUDA, "descriptor %d: cuTensorMapEncodeTiled failed (%d)", d,
                             rc);
         }
         ptiles += tw::prefill_tiles(M, s.N);
+        const int64_t nrb = tw::ceil_div(s.N, tw::kTileRows);
         if (decode) {
             r.ws_xq_off = ws_off;
             ws_off += tw::round128(M * s.K);
+            r.urb = std::max<int64_t>(1, tw::kUnitBytes / (4 * s.K));
+            r.unit_begin = units;
+            units += tw::ceil_div(nrb, r.urb);
         }
-        const int64_t nrb = tw::ceil_div(s.N, tw::kTileRows);
         rb += nrb;
         tiles += nrb * (s.K / tw::kTileK);
         max_K = s.K > max_K ? s.K : max_K;
-        sum_K += s.K;
     }
     if (rb > INT32_MAX || tiles > ((int64_t)1 << 40))
         return fail(TW_ERR_SHAPE, "sweep too large: %lld row blocks", (long long)rb);
@@ -358,7 +367,7 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
     hdr->total_ptiles = ptiles;
     hdr->ws_bytes = decode ? ws_off + 256 * (int64_t)count : 0;
     hdr->max_K = max_K;
-    hdr->sum_K = sum_K;
+    hdr->total_units = units;
     return TW_OK;
 }
 
@@ -400,6 +409,20 @@ int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, v
                     (long long)hdr->ws_bytes);
     if (!aligned16(ws))
         return fail(TW_ERR_ALIGN, "sweep workspace must be 16-byte aligned");
+    if (tw::decode_dyn_supported(hdr->M, hdr->max_K)) {
+        tw::DecodeDynLaunch D{};
+        D.table = reinterpret_cast<const tw::DescRecord *>(
+            static_cast<const tw::TableHeader *>(table_dev) + 1);
+        D.count = hdr->count;
+        D.M = hdr->M;
+        D.max_K = hdr->max_K;
+        D.total_units = hdr->total_units;
+        D.ws = static_cast<uint8_t *>(ws);
+        D.flags_off = tw::kWsCtrBytes;
+        D.sa_off = hdr->ws_bytes - 256 * (int64_t)hdr->count;
+        cudaError_t e = tw::launch_decode_dyn(D, err, kWaitNs, stream);
+        return e == cudaSuccess ? TW_OK : cuda_fail(e, "sweep launch");
+    }
     tw::DecodeLaunch L{};
     L.table = reinterpret_cast<const tw::DescRecord *>(
         static_cast<const tw::TableHeader *>(table_dev) + 1);
@@ -421,6 +444,8 @@ int tw_sweep_launches(const void *table_host)
     if (!hdr || hdr->magic != tw::kTableMagic)
         return 0;
     if (hdr->M > tw::kDecodeMaxM)
+        return 1;
+    if (tw::decode_dyn_supported(hdr->M, hdr->max_K))
         return 1;
     return tw::decode_launches(hdr->M, hdr->max_K);
 }

@@ -33,10 +33,12 @@ struct alignas(64) DescRecord {
     int64_t tile_begin;  // first 16x128 code tile of this projection
     int64_t ptile_begin; // first prefill output tile of this projection
     int64_t ws_xq_off;   // decode: offset of this projection's int8 rows in ws
-    int64_t reserved[2];
-    alignas(64) uint8_t tmap_xq[128];  // CUtensorMap of xq (prefill only)
+    int64_t unit_begin;  // decode: first work unit of this projection
+    int64_t urb;         // decode: row blocks per work unit
+    alignas(64) uint8_t tmap_xq[128];     // CUtensorMap of xq (prefill only)
+    alignas(64) uint8_t tmap_codes[128];  // CUtensorMap of the packed codes (prefill only)
 };
-static_assert(sizeof(DescRecord) == 256, "record size");
+static_assert(sizeof(DescRecord) == 384, "record size");
 
 struct alignas(64) TableHeader {
     uint32_t magic;
@@ -46,8 +48,8 @@ struct alignas(64) TableHeader {
     int64_t total_tiles;
     int64_t total_ptiles;
     int64_t max_K;
-    int64_t sum_K;
-    int64_t ws_bytes;    // decode: scratch for the quantised activations
+    int64_t total_units; // decode: work units of the sweep
+    int64_t ws_bytes;    // decode: scratch (counters, row flags, int8 rows, scales)
 };
 static_assert(sizeof(TableHeader) == 64, "header size");
 
@@ -74,6 +76,22 @@ struct DecodeLaunch {
 };
 // Kernel launches one decode call makes for M tokens (quantise + groups).
 int decode_launches(int64_t M, int64_t max_K);
+
+// Single-launch, dynamically balanced decode sweep (M <= kDynMaxM).
+constexpr int kDynMaxM = 4;
+constexpr int64_t kUnitBytes = 65536;   // target packed bytes per work unit
+constexpr int64_t kWsCtrBytes = 256;    // claim / done counters at the start of ws
+struct DecodeDynLaunch {
+    const DescRecord *table;  // device records
+    int count;
+    int64_t M, max_K, total_units;
+    uint8_t *ws;              // zero-filled before the first call; left so
+    int64_t flags_off;        // per-row ready flags (u32)
+    int64_t sa_off;           // per-projection amax/127, sum(q)
+};
+bool decode_dyn_supported(int64_t M, int64_t max_K);
+cudaError_t launch_decode_dyn(const DecodeDynLaunch &L, uint32_t *err, uint64_t timeout_ns,
+                              cudaStream_t stream);
 // Decode scratch: per projection its M int8 rows (128-byte aligned), then
 // per projection 256 bytes: 32 floats amax/127 and 32 ints sum(q).
 inline int64_t round128(int64_t b) { return (b + 127) / 128 * 128; }
@@ -94,6 +112,10 @@ int64_t prefill_tiles(int64_t M, int64_t N);
 // Encode the TMA descriptor of xq [M x K] int8 into out128 (128 bytes).
 // Returns 0, -1 when the driver entry point is unavailable, or a CUresult.
 int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, void *out128);
+// Encode the TMA descriptor of the packed codes of an [N x K] matrix, seen as
+// [ceil(N/16)] x [K/128] tiles of 128 32-bit words (one box = 16 row blocks
+// of one k tile).
+int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, void *out128);
 
 cudaError_t launch_wait_probe(uint32_t *err, uint64_t timeout_ns, cudaStream_t stream);
 

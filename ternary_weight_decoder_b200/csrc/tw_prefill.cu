@@ -167,6 +167,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 3-D TMA load of one box into shared memory (no multicast).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int32_t x, int32_t y,
+                                            int32_t z, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
 // 2-D TMA load of one box into shared memory (no multicast).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int32_t x, int32_t y,
                                             uint32_t bar)
@@ -260,12 +271,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
             TileIter ti;
             for (ti.init(p, blockIdx.x); ti.valid(p) && !*abort_flag; ti.next(p, G)) {
                 const int64_t KT = ti.K / kBK;
-                const int64_t nrb = (ti.N + kTileRows - 1) / kTileRows;
-                const int64_t rb0 = ti.nj * (kBN / kTileRows);
-                const int nct = (int)min((int64_t)(kBN / kTileRows), nrb - rb0);
-                const uint32_t bytes = kABytes + nct * kTileBytes;
-                const uint8_t *codes0 = ti.r->packed + rb0 * KT * kTileBytes;
+                const int32_t rb0 = (int32_t)(ti.nj * (kBN / kTileRows));
+                // the code box is always 16 row blocks (rows past N read as
+                // zero and only feed output columns that are not stored)
+                const uint32_t bytes = kABytes + kCodeBytes;
                 const void *tmap = ti.r->tmap_xq;
+                const void *tmap_c = ti.r->tmap_codes;
                 const int32_t ycoord = (int32_t)(ti.mi * kBM);
                 bool ok = true;
                 for (int64_t kt = 0; kt < KT; ++kt, ++it) {
@@ -278,9 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
                     }
                     mbar_arrive_expect_tx(b_ldfull + 8 * s, bytes);
                     tma_load_2d(L.a(s), tmap, (int32_t)(kt * kBK), ycoord, b_ldfull + 8 * s);
-                    for (int i = 0; i < nct; ++i)
-                        bulk_g2s(L.codes(s) + i * kTileBytes, codes0 + (i * KT + kt) * kTileBytes,
-                                 kTileBytes, b_ldfull + 8 * s);
+                    tma_load_3d(L.codes(s), tmap_c, 0, (int32_t)kt, rb0, b_ldfull + 8 * s);
                 }
                 if (!ok)
                     break;
@@ -502,6 +511,34 @@ int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, void *out128)
     if (r != CUDA_SUCCESS)
         return (int)r;
     static_assert(sizeof(CUtensorMap) == 128, "tensor map size");
+    memcpy(out128, &m, sizeof(m));
+    return 0;
+}
+
+int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, void *out128)
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !f)
+            return -1;
+        fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    CUtensorMap m;
+    memset(&m, 0, sizeof(m));
+    const int64_t KT = K / kTileK, nrb = (N + kTileRows - 1) / kTileRows;
+    const cuuint64_t dims[3] = {(cuuint64_t)(kTileBytes / 4), (cuuint64_t)KT, (cuuint64_t)nrb};
+    const cuuint64_t strides[2] = {(cuuint64_t)kTileBytes, (cuuint64_t)(KT * kTileBytes)};
+    const cuuint32_t box[3] = {kTileBytes / 4, 1, kBN / kTileRows};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t *>(packed), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return (int)r;
     memcpy(out128, &m, sizeof(m));
     return 0;
 }

@@ -65,11 +65,12 @@ def _descs(shapes, base=0x10000):
 REC = np.dtype([("x", "<u8"), ("xq", "<u8"), ("amax", "<u8"), ("qsum", "<u8"),
                 ("packed", "<u8"), ("wscale", "<u8"), ("y", "<u8"), ("acc_out", "<u8"),
                 ("N", "<i8"), ("K", "<i8"), ("rb_begin", "<i8"), ("tile_begin", "<i8"),
-                ("ptile_begin", "<i8"), ("ws_xq_off", "<i8"), ("res", "<i8", 2),
-                ("tmap", "u1", 128)])
+                ("ptile_begin", "<i8"), ("ws_xq_off", "<i8"), ("unit_begin", "<i8"),
+                ("urb", "<i8"),
+                ("tmap", "u1", 128), ("tmap_codes", "u1", 128)])
 HDR = np.dtype([("magic", "<u4"), ("count", "<i4"), ("M", "<i8"), ("total_rb", "<i8"),
                 ("total_tiles", "<i8"), ("total_ptiles", "<i8"), ("max_K", "<i8"),
-                ("sum_K", "<i8"), ("ws_bytes", "<i8")])
+                ("total_units", "<i8"), ("ws_bytes", "<i8")])
 
 
 def test_table_encode_prefix_sums(lib):
@@ -77,7 +78,7 @@ def test_table_encode_prefix_sums(lib):
     shapes = [(1536, 1536), (256, 1536), (17, 256), (1536, 8960)]
     arr = _descs(shapes)
     n = api.tw_sweep_table_bytes(len(shapes))
-    assert n == 64 + 256 * len(shapes)
+    assert n == 64 + 384 * len(shapes)
     buf = np.zeros(n, np.uint8)
     rc = api.tw_sweep_table_encode(arr, len(shapes), 1, buf.ctypes.data, n)
     assert rc == 0, api.tw_last_error()
@@ -89,13 +90,20 @@ def test_table_encode_prefix_sums(lib):
     assert recs["rb_begin"].tolist() == np.concatenate([[0], np.cumsum(nrb)[:-1]]).tolist()
     assert recs["tile_begin"].tolist() == np.concatenate([[0], np.cumsum(ntiles)[:-1]]).tolist()
     assert hdr["total_rb"] == sum(nrb) and hdr["total_tiles"] == sum(ntiles)
-    assert hdr["max_K"] == 8960 and hdr["sum_K"] == 1536 * 2 + 256 + 8960
+    assert hdr["max_K"] == 8960
+    urb = [max(1, 65536 // (4 * K)) for N, K in shapes]
+    assert recs["urb"].tolist() == urb
+    units = [-(-r // u) for r, u in zip(nrb, urb)]
+    assert recs["unit_begin"].tolist() == np.concatenate([[0], np.cumsum(units)[:-1]]).tolist()
+    assert hdr["total_units"] == sum(units)
     assert recs["N"].tolist() == [s[0] for s in shapes]
+    # scratch: 256 B of counters, one flag per (projection, token), int8 rows, scales
     xq = [-(-K // 128) * 128 for N, K in shapes]   # M = 1 rows, 128-byte aligned
-    assert recs["ws_xq_off"].tolist() == np.concatenate([[0], np.cumsum(xq)[:-1]]).tolist()
-    assert hdr["ws_bytes"] == sum(xq) + 256 * len(shapes)
+    head = 256 + 128
+    assert recs["ws_xq_off"].tolist() == (head + np.concatenate([[0], np.cumsum(xq)[:-1]])).tolist()
+    assert hdr["ws_bytes"] == head + sum(xq) + 256 * len(shapes)
     assert api.tw_sweep_workspace_bytes(buf.ctypes.data) == hdr["ws_bytes"]
-    assert api.tw_sweep_launches(buf.ctypes.data) == 2   # quantise + one decode launch
+    assert api.tw_sweep_launches(buf.ctypes.data) in (1, 2)   # dynamic path or quantise + decode
 
 
 @pytest.mark.parametrize("bad,status", [
