@@ -5,8 +5,11 @@ ternary matrices of a Qwen2.5-1.5B-shaped decoder (q/o 1536x1536, k/v
 256x1536, gate/up 8960x1536, down 1536x8960; 1,310,195,712 weights,
 327,548,928 bytes of 2-bit codes), one token (M = 1), seeded synthetic
 weights N(0, 0.02^2) and activations N(0, 1) with 1% outlier channels x20.
-A step is one pass of the whole hot path over every projection: fused
-activation quantisation, ternary product, rescale (one persistent launch).
+A step is one pass of the whole hot path over every projection: activation
+quantisation (one launch), then ternary product and rescale (one persistent
+launch per token group, started early by programmatic dependent launch).
+Prefill sizes (--m > 32) take int8 activations quantised beforehand and run
+the tensor-core kernel (one persistent launch).
 
 Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own
 replica of the sweep on its own token (data-parallel decode; no collective
@@ -52,6 +55,29 @@ def peaks():
         d = json.load(open(p))
         return d.get("hbm_gbs", FALLBACK_HBM_GBS), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def _sha256(path):
+    import hashlib
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def profiled_traffic(kernel_src, M, layers):
+    """DRAM bytes (read + write) per launch of the dominant kernel, from the
+    ncu capture recorded in profiles/traffic.json, or None when there is no
+    capture for this M or the kernel's source has changed since it was taken.
+    A capture of fewer layers is scaled by the layer count (the traffic of a
+    sweep grows in proportion to its projections at fixed M)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    src = os.path.join(ROOT, "ternary_weight_decoder_b200", "csrc", kernel_src)
+    digest = _sha256(src)
+    for e in json.load(open(p)).get("captures", []):
+        if e["kernel_src"] == kernel_src and e["M"] == M and e["source_sha256"] == digest:
+            return e["dram_bytes_per_launch"] * layers / e["layers"]
+    return None
 
 
 def sweep_bytes(shapes, M):
@@ -301,7 +327,8 @@ def main():
         # decode: HBM-bound; algorithmic bytes = 2-bit codes + fp32 x + fp32 y
         achieved = algo_bytes / (ms_per_step / 1e3) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                    "frac": achieved / hbm, "traffic": None,
+                    "frac": achieved / hbm,
+                    "traffic": profiled_traffic("tw_decode.cu", M, args.layers),
                     "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured"
                     else "fallback 6650 GB/s",
                     "algorithmic_bytes_per_step": algo_bytes,
@@ -315,7 +342,8 @@ def main():
         pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))).get("bf16_tflops") \
             if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else FALLBACK_BF16_TFLOPS
         roofline = {"bound": "tensor", "achieved": tops, "peak": 2 * pk, "unit": "TOP/s",
-                    "frac": tops / (2 * pk), "traffic": None,
+                    "frac": tops / (2 * pk),
+                    "traffic": profiled_traffic("tw_prefill.cu", M, args.layers),
                     "peak_source": "2 x measured bf16 burst (int8 dense = 2 x bf16 nominal)",
                     "ops_per_step": ops}
 
