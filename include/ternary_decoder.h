@@ -209,10 +209,10 @@ TW_API size_t tw_sweep_table_bytes(int count);
 TW_API int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M,
                           void *table, size_t table_bytes);
 
-/* Scratch needed by tw_decoder_projection_sweep for an encoded HOST table.
- * For decode (M <= 32) it holds work counters and per-row ready flags: it
- * must be zero-filled before its first use with a table, and every call
- * leaves it that way (after TW_ERR_TIMEOUT, zero it again). */
+/* Scratch needed by tw_decoder_projection_sweep for an encoded HOST table:
+ * for decode (M <= 32) the quantised rows of every projection and their
+ * scales, rewritten by every call (no initial contents needed); 0 for
+ * prefill, whose callers pass the quantised rows in the descriptors. */
 TW_API size_t tw_sweep_workspace_bytes(const void *table_host);
 
 /*

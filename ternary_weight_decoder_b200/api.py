@@ -230,8 +230,8 @@ class SweepTable:
             self.device = self.host.to(device, non_blocking=False)
         wsb = int(tw_sweep_workspace_bytes(_ptr(self.host)))
         self.launches = int(tw_sweep_launches(_ptr(self.host)))
-        # zero-filled once: the decode kernels keep their counters and flags
-        # here and leave them cleared after every call
+        # decode scratch: the quantised rows and their scales (rewritten by
+        # every call)
         self.ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=device) \
             if device is not None else None
         self.ws_bytes = wsb

@@ -96,7 +96,7 @@ int run_prefill_single(const int8_t *xq, const float *amax, const int32_t *qsum,
     r.K = K;
     int rc = tw::encode_xq_tmap(xq, M, K, r.tmap_xq);
     if (!rc)
-        rc = tw::encode_codes_tmap(r.packed, N, K, r.tmap_codes);
+        rc = tw::encode_codes_tmap(r.packed, N, K, 16, r.tmap_codes);
     if (rc)
         return fail(TW_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", rc);
     tw::PrefillLaunch L{};
@@ -241,7 +241,7 @@ int tw_ternary_linear(const float *x, int64_t M, int64_t N, int64_t K, const voi
         L.count = 1;
         L.M = M;
         L.total_rb = tw::ceil_div(N, tw::kTileRows);
-        L.total_tiles = L.total_rb * (K / tw::kTileK);
+        L.total_cost = L.total_rb * tw::rb_cost(K);
         L.max_K = K;
         L.ws = static_cast<uint8_t *>(ws);
         L.ws_sa_off = tw::round128(M * K);
@@ -283,7 +283,7 @@ size_t tw_sweep_table_bytes(int count)
 {
     if (count < 1)
         return 0;
-    return sizeof(tw::TableHeader) + (size_t)count * sizeof(tw::DescRecord);
+    return sizeof(tw::TableHeader) + (size_t)count * (sizeof(tw::DescRecord) + sizeof(tw::UnitOrder));
 }
 
 int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void *table,
@@ -303,9 +303,11 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
     auto *hdr = static_cast<tw::TableHeader *>(table);
     auto *recs = reinterpret_cast<tw::DescRecord *>(hdr + 1);
     memset(table, 0, tw_sweep_table_bytes(count));
-    int64_t rb = 0, tiles = 0, ptiles = 0, max_K = 0, units = 0;
-    // decode scratch: counters | row flags | int8 rows | scales
-    int64_t ws_off = tw::kWsCtrBytes + tw::round128(4 * (int64_t)count * M);
+    int64_t rb = 0, tiles = 0, ptiles = 0, max_K = 0, cost = 0;
+    // decode scratch: counters | per projection its token rows or blocks
+    // (room for tc_tokens(M) >= M rows of K bytes) | scales
+    int64_t ws_off = tw::kWsCtrBytes;
+    const int64_t rows = decode ? tw::tc_tokens(M) : 0;
     for (int d = 0; d < count; ++d) {
         const tw_proj_desc &s = descs[d];
         if (int rc = check_shape(M, s.N, s.K))
@@ -336,22 +338,26 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
         r.rb_begin = rb;
         r.tile_begin = tiles;
         r.ptile_begin = ptiles;
-        if (!decode) {
-            int rc = tw::encode_xq_tmap(s.xq, M, s.K, r.tmap_xq);
+        {
+            // prefill: xq tiles of 128 tokens and 256-row code boxes; decode:
+            // 128-row code boxes of the tensor-core sweep.  Without a CUDA
+            // driver (-1) a decode table is still encoded for its sizes; the
+            // sweep refuses it.
+            int rc = decode ? 0 : tw::encode_xq_tmap(s.xq, M, s.K, r.tmap_xq);
             if (!rc)
-                rc = tw::encode_codes_tmap(r.packed, s.N, s.K, r.tmap_codes);
-            if (rc)
+                rc = tw::encode_codes_tmap(r.packed, s.N, s.K, decode ? 8 : 16, r.tmap_codes);
+            if (rc && !(decode && rc == -1))
                 return fail(TW_ERR_CUDA, "descriptor %d: cuTensorMapEncodeTiled failed (%d)", d,
                             rc);
+            r.tmap_ok = rc == 0;
         }
         ptiles += tw::prefill_tiles(M, s.N);
         const int64_t nrb = tw::ceil_div(s.N, tw::kTileRows);
         if (decode) {
             r.ws_xq_off = ws_off;
-            ws_off += tw::round128(M * s.K);
-            r.urb = std::max<int64_t>(1, tw::kUnitBytes / (4 * s.K));
-            r.unit_begin = units;
-            units += tw::ceil_div(nrb, r.urb);
+            ws_off += tw::round128(rows * s.K);
+            r.cost_begin = cost;
+            cost += nrb * tw::rb_cost(s.K);
         }
         rb += nrb;
         tiles += nrb * (s.K / tw::kTileK);
@@ -359,15 +365,31 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
     }
     if (rb > INT32_MAX || tiles > ((int64_t)1 << 40))
         return fail(TW_ERR_SHAPE, "sweep too large: %lld row blocks", (long long)rb);
+    // Order of the tensor-core sweep's units: projections of larger K first
+    // (stable), 128 rows per unit.
+    auto *order = reinterpret_cast<tw::UnitOrder *>(recs + count);
+    for (int d = 0; d < count; ++d)
+        order[d].d = d;
+    std::stable_sort(order, order + count, [&](const tw::UnitOrder &a, const tw::UnitOrder &b) {
+        return recs[a.d].K > recs[b.d].K;
+    });
+    int64_t units = 0;
+    for (int i = 0; i < count; ++i) {
+        order[i].units = (int32_t)tw::ceil_div(recs[order[i].d].N, 128);
+        order[i].unit_begin = units;
+        units += order[i].units;
+    }
+    if (units > INT32_MAX)
+        return fail(TW_ERR_SHAPE, "sweep too large: %lld units", (long long)units);
     hdr->magic = tw::kTableMagic;
     hdr->count = count;
     hdr->M = M;
     hdr->total_rb = rb;
-    hdr->total_tiles = tiles;
+    hdr->total_units = units;
     hdr->total_ptiles = ptiles;
     hdr->ws_bytes = decode ? ws_off + 256 * (int64_t)count : 0;
     hdr->max_K = max_K;
-    hdr->total_units = units;
+    hdr->total_cost = cost;
     return TW_OK;
 }
 
@@ -409,32 +431,34 @@ int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, v
                     (long long)hdr->ws_bytes);
     if (!aligned16(ws))
         return fail(TW_ERR_ALIGN, "sweep workspace must be 16-byte aligned");
-    if (tw::decode_dyn_supported(hdr->M, hdr->max_K)) {
-        tw::DecodeDynLaunch D{};
-        D.table = reinterpret_cast<const tw::DescRecord *>(
-            static_cast<const tw::TableHeader *>(table_dev) + 1);
-        D.count = hdr->count;
-        D.M = hdr->M;
-        D.max_K = hdr->max_K;
-        D.total_units = hdr->total_units;
-        D.ws = static_cast<uint8_t *>(ws);
-        D.flags_off = tw::kWsCtrBytes;
-        D.sa_off = hdr->ws_bytes - 256 * (int64_t)hdr->count;
-        cudaError_t e = tw::launch_decode_dyn(D, err, kWaitNs, stream);
+    const auto *recs_dev = reinterpret_cast<const tw::DescRecord *>(
+        static_cast<const tw::TableHeader *>(table_dev) + 1);
+    if (!tw::decode_sweep_on_tensor_cores(hdr->M)) {
+        tw::DecodeLaunch L{};
+        L.table = recs_dev;
+        L.single = nullptr;
+        L.count = hdr->count;
+        L.M = hdr->M;
+        L.total_rb = hdr->total_rb;
+        L.total_cost = hdr->total_cost;
+        L.max_K = hdr->max_K;
+        L.ws = static_cast<uint8_t *>(ws);
+        L.ws_sa_off = hdr->ws_bytes - 256 * (int64_t)hdr->count;
+        cudaError_t e = tw::launch_decode(L, err, kWaitNs, stream);
         return e == cudaSuccess ? TW_OK : cuda_fail(e, "sweep launch");
     }
-    tw::DecodeLaunch L{};
-    L.table = reinterpret_cast<const tw::DescRecord *>(
-        static_cast<const tw::TableHeader *>(table_dev) + 1);
-    L.single = nullptr;
-    L.count = hdr->count;
-    L.M = hdr->M;
-    L.total_rb = hdr->total_rb;
-    L.total_tiles = hdr->total_tiles;
-    L.max_K = hdr->max_K;
-    L.ws = static_cast<uint8_t *>(ws);
-    L.ws_sa_off = hdr->ws_bytes - 256 * (int64_t)hdr->count;
-    cudaError_t e = tw::launch_decode(L, err, kWaitNs, stream);
+    if (!reinterpret_cast<const tw::DescRecord *>(hdr + 1)->tmap_ok)
+        return fail(TW_ERR_CUDA, "table was encoded without the CUDA driver's TMA encoder");
+    tw::DecodeTcLaunch T{};
+    T.table = recs_dev;
+    T.order = reinterpret_cast<const tw::UnitOrder *>(recs_dev + hdr->count);
+    T.count = hdr->count;
+    T.M = hdr->M;
+    T.total_units = hdr->total_units;
+    T.ws = static_cast<uint8_t *>(ws);
+    T.ws_sa_off = hdr->ws_bytes - 256 * (int64_t)hdr->count;
+    T.ctr = reinterpret_cast<uint32_t *>(ws);
+    cudaError_t e = tw::launch_decode_tc(T, err, kWaitNs, stream);
     return e == cudaSuccess ? TW_OK : cuda_fail(e, "sweep launch");
 }
 
@@ -445,9 +469,9 @@ int tw_sweep_launches(const void *table_host)
         return 0;
     if (hdr->M > tw::kDecodeMaxM)
         return 1;
-    if (tw::decode_dyn_supported(hdr->M, hdr->max_K))
-        return 1;
-    return tw::decode_launches(hdr->M, hdr->max_K);
+    if (!tw::decode_sweep_on_tensor_cores(hdr->M))
+        return tw::decode_launches(hdr->M, hdr->max_K);
+    return 2;  // quantise + the tensor-core sweep
 }
 
 int tw_check(tw_stream_t stream)

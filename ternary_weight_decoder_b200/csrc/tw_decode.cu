@@ -59,7 +59,7 @@ struct DecodeParams {
     int xb;                   // activation buffers (1..4)
     int xs;                   // activation row stride in shared memory
     int slots;                // ring slots per consumer warp
-    int64_t total_rb, total_tiles;
+    int64_t total_rb, total_cost;
     const uint8_t *ws;        // quantised activations (launch 1 output)
     int64_t ws_sa_off;        // offset of the per-projection amax/127, sum(q)
     WaitCtl ctl;
@@ -69,6 +69,7 @@ struct QuantParams {
     const DescRecord *table;
     DescRecord single;
     int count, M;
+    int ntok;                 // 0: plain int8 rows; 8/16/32: tensor-core token blocks
     uint8_t *ws;
     int64_t ws_sa_off;
 };
@@ -111,6 +112,19 @@ __device__ __forceinline__ uint32_t quant4(float4 v, float scale, bool zero, int
 __device__ __forceinline__ float amax4(float4 v)
 {
     return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+}
+
+// Offset, in the tensor-core token blocks of one projection, of the four
+// bytes q[4 idx .. 4 idx + 3] of token m: k tile kt = idx / 32 is a block of
+// ntok rows x 128 bytes; logical k group G = idx mod 32 = 16h + 4t + s goes
+// to column c = 8s + 2t + h (4 bytes each) of row m, whose 16-byte chunks
+// are swizzled by m mod 8.
+__device__ __forceinline__ int64_t tc_block_offset(int64_t idx, int m, int ntok)
+{
+    const int G = (int)(idx & 31);
+    const int h = G >> 4, t = (G >> 2) & 3, s = G & 3;
+    const int c = 8 * s + 2 * t + h;
+    return (idx >> 5) * (int64_t)ntok * 128 + m * 128 + ((((c >> 2) ^ (m & 7)) << 4) | ((c & 3) << 2));
 }
 
 // Block (d, m): quantise token row m of projection d.  amax = max|x|,
@@ -157,16 +171,27 @@ __global__ void __launch_bounds__(kQThreads) k_quant_rows(const __grid_constant_
     const bool zero = (a == 0.f);
     const float scale = zero ? 0.f : __fdiv_rn(127.f, a);
     int sum = 0;
+    uint8_t *blocks = p.ws + r.ws_xq_off;
     if (in_regs) {
 #pragma unroll
         for (int i = 0; i < kQRegs; ++i) {
             const int64_t idx = tid + (int64_t)i * kQThreads;
-            if (idx < K4)
-                qrow[idx] = quant4(v[i], scale, zero, sum);
+            if (idx < K4) {
+                const uint32_t u = quant4(v[i], scale, zero, sum);
+                if (p.ntok)
+                    *reinterpret_cast<uint32_t *>(blocks + tc_block_offset(idx, m, p.ntok)) = u;
+                else
+                    qrow[idx] = u;
+            }
         }
     } else {
-        for (int64_t i = tid; i < K4; i += kQThreads)
-            qrow[i] = quant4(__ldg(row + i), scale, zero, sum);
+        for (int64_t i = tid; i < K4; i += kQThreads) {
+            const uint32_t u = quant4(__ldg(row + i), scale, zero, sum);
+            if (p.ntok)
+                *reinterpret_cast<uint32_t *>(blocks + tc_block_offset(i, m, p.ntok)) = u;
+            else
+                qrow[i] = u;
+        }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1)
@@ -185,27 +210,31 @@ __global__ void __launch_bounds__(kQThreads) k_quant_rows(const __grid_constant_
 }
 
 // ----------------------------------------------------------------- launch 2
-// First row block owned by CTA i of G: the first block whose first tile is
-// at or after tile floor(total_tiles * i / G).
+// Cost of one 16-row block (the host's rb_cost): 16 units per 128-column
+// tile plus a fixed part for its epilogue and loop set-up.
+__device__ __forceinline__ int64_t rb_cost_dev(int64_t K) { return rb_cost(K); }
+
+// First row block owned by CTA i of G: the first block whose cost range
+// starts at or after floor(total_cost * i / G).
 __device__ int64_t share_boundary(const DecodeParams &p, int i, int G)
 {
     if (i <= 0)
         return 0;
     if (i >= G)
         return p.total_rb;
-    const int64_t t = p.total_tiles * i / G;  // total_tiles < 2^40, i < 2^16
-    int lo = 0, hi = p.count - 1;  // largest d with tile_begin <= t
+    const int64_t t = p.total_cost * i / G;  // total_cost < 2^44, i < 2^16
+    int lo = 0, hi = p.count - 1;  // largest d with cost_begin <= t
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (rec(p, mid).tile_begin <= t)
+        if (rec(p, mid).cost_begin <= t)
             lo = mid;
         else
             hi = mid - 1;
     }
     const DescRecord &r = rec(p, lo);
-    const int64_t KT = r.K / kTileK;
-    const int64_t rl = (t - r.tile_begin + KT - 1) / KT;
-    return r.rb_begin + rl;
+    const int64_t c = rb_cost_dev(r.K);
+    const int64_t rl = (t - r.cost_begin + c - 1) / c;
+    return min(r.rb_begin + rl, r.rb_begin + rb_count(r));
 }
 
 __device__ int desc_of_rb(const DecodeParams &p, int64_t rb)
@@ -604,6 +633,21 @@ bool plan_decode(int M, int64_t max_K, int *mg_out, int *slots_out, int *xb_out)
 
 }  // namespace
 
+cudaError_t launch_quant_tc(const DescRecord *table, int count, int64_t M, int ntok, uint8_t *ws,
+                            int64_t ws_sa_off, cudaStream_t stream)
+{
+    QuantParams q;
+    memset(&q, 0, sizeof(q));
+    q.table = table;
+    q.count = count;
+    q.M = (int)M;
+    q.ntok = ntok;
+    q.ws = ws;
+    q.ws_sa_off = ws_sa_off;
+    k_quant_rows<<<(unsigned)(count * M), kQThreads, 0, stream>>>(q);
+    return cudaGetLastError();
+}
+
 int decode_launches(int64_t M, int64_t max_K)
 {
     int mg = 1, slots = 2, xb = 1;
@@ -649,7 +693,7 @@ cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout
     p.count = L.count;
     p.M = M;
     p.total_rb = L.total_rb;
-    p.total_tiles = L.total_tiles;
+    p.total_cost = L.total_cost;
     p.xs = (int)(L.max_K + 64);
     p.ws = L.ws;
     p.ws_sa_off = L.ws_sa_off;

@@ -33,8 +33,8 @@ struct alignas(64) DescRecord {
     int64_t tile_begin;  // first 16x128 code tile of this projection
     int64_t ptile_begin; // first prefill output tile of this projection
     int64_t ws_xq_off;   // decode: offset of this projection's int8 rows in ws
-    int64_t unit_begin;  // decode: first work unit of this projection
-    int64_t urb;         // decode: row blocks per work unit
+    int64_t cost_begin;  // decode: first cost unit of this projection (static split)
+    int64_t tmap_ok;     // 1: tmap_codes holds an encoded descriptor
     alignas(64) uint8_t tmap_xq[128];     // CUtensorMap of xq (prefill only)
     alignas(64) uint8_t tmap_codes[128];  // CUtensorMap of the packed codes (prefill only)
 };
@@ -45,11 +45,11 @@ struct alignas(64) TableHeader {
     int32_t count;
     int64_t M;
     int64_t total_rb;
-    int64_t total_tiles;
+    int64_t total_units; // decode: 128-row units of the tensor-core sweep
     int64_t total_ptiles;
     int64_t max_K;
-    int64_t total_units; // decode: work units of the sweep
-    int64_t ws_bytes;    // decode: scratch (counters, row flags, int8 rows, scales)
+    int64_t total_cost;  // decode: cost units of the sweep
+    int64_t ws_bytes;    // decode: scratch (counter, ready flags, int8 rows, scales)
 };
 static_assert(sizeof(TableHeader) == 64, "header size");
 
@@ -65,11 +65,17 @@ cudaError_t launch_unpack(const uint8_t *packed, int64_t N, int64_t K, int8_t *c
 cudaError_t launch_quantize(const float *x, int64_t M, int64_t K, int8_t *xq, float *amax,
                             int32_t *qsum, cudaStream_t stream);
 
+// Static split of a decode sweep: a 16-row block of a projection with K
+// columns costs 16 units per 128-column tile plus a fixed part for its
+// epilogue and loop set-up.
+constexpr int64_t kRbFixedCost = 45;
+__host__ __device__ inline int64_t rb_cost(int64_t K) { return 16 * (K / kTileK) + kRbFixedCost; }
+
 struct DecodeLaunch {
     const DescRecord *table;  // device records (or null: use `single`)
     int count;
     int64_t M;
-    int64_t total_rb, total_tiles, max_K;
+    int64_t total_rb, total_cost, max_K;
     const DescRecord *single; // host copy of a one-record sweep (table == null)
     uint8_t *ws;              // scratch: int8 rows at each record's ws_xq_off,
     int64_t ws_sa_off;        // then 256 bytes of amax/127, sum(q) per record
@@ -77,23 +83,41 @@ struct DecodeLaunch {
 // Kernel launches one decode call makes for M tokens (quantise + groups).
 int decode_launches(int64_t M, int64_t max_K);
 
-// Single-launch, dynamically balanced decode sweep (M <= kDynMaxM).
-constexpr int kDynMaxM = 4;
-constexpr int64_t kUnitBytes = 65536;   // target packed bytes per work unit
-constexpr int64_t kWsCtrBytes = 256;    // claim / done counters at the start of ws
-struct DecodeDynLaunch {
-    const DescRecord *table;  // device records
-    int count;
-    int64_t M, max_K, total_units;
-    uint8_t *ws;              // zero-filled before the first call; left so
-    int64_t flags_off;        // per-row ready flags (u32)
-    int64_t sa_off;           // per-projection amax/127, sum(q)
+// Decode scratch of the single-matrix path: the M int8 rows (128-byte
+// aligned), then 256 bytes: 32 floats amax/127 and 32 ints sum(q).
+
+// Tensor-core decode sweep (tw_decode_tc.cu).  Its scratch: 256 bytes of
+// counters (claim, finished blocks; zero between calls), then per projection
+// its token blocks -- K/128 blocks of tc_tokens(M) rows x 128 bytes, 128-byte
+// swizzled -- then per projection 256 bytes of amax/127 and sum(q).
+constexpr int64_t kWsCtrBytes = 256;
+inline int tc_tokens(int64_t M) { return M <= 8 ? 8 : M <= 16 ? 16 : 32; }
+// Which decode kernel runs a sweep of M tokens (measured on B200: the
+// tensor-core sweep wins once the int8 MMAs of the register path, 4 per
+// 8 tokens per tile, and their operand loads no longer keep up with HBM).
+inline bool decode_sweep_on_tensor_cores(int64_t M) { return M > 16; }
+// Projections in the order their units are handed out (K descending); the
+// units of entry i are [unit_begin, unit_begin + units), one per 128 rows.
+struct UnitOrder {
+    int32_t d;
+    int32_t units;
+    int64_t unit_begin;
 };
-bool decode_dyn_supported(int64_t M, int64_t max_K);
-cudaError_t launch_decode_dyn(const DecodeDynLaunch &L, uint32_t *err, uint64_t timeout_ns,
-                              cudaStream_t stream);
-// Decode scratch: per projection its M int8 rows (128-byte aligned), then
-// per projection 256 bytes: 32 floats amax/127 and 32 ints sum(q).
+static_assert(sizeof(UnitOrder) == 16, "unit order entry");
+struct DecodeTcLaunch {
+    const DescRecord *table;  // device records
+    const UnitOrder *order;   // device copy of the order (follows the records)
+    int count;
+    int64_t M, total_units;
+    uint8_t *ws;
+    int64_t ws_sa_off;
+    uint32_t *ctr;
+};
+cudaError_t launch_decode_tc(const DecodeTcLaunch &L, uint32_t *err, uint64_t timeout_ns,
+                             cudaStream_t stream);
+// Quantise every (projection, token) row into the token blocks above.
+cudaError_t launch_quant_tc(const DescRecord *table, int count, int64_t M, int ntok, uint8_t *ws,
+                            int64_t ws_sa_off, cudaStream_t stream);
 inline int64_t round128(int64_t b) { return (b + 127) / 128 * 128; }
 cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout_ns,
                           cudaStream_t stream);
@@ -113,9 +137,9 @@ int64_t prefill_tiles(int64_t M, int64_t N);
 // Returns 0, -1 when the driver entry point is unavailable, or a CUresult.
 int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, void *out128);
 // Encode the TMA descriptor of the packed codes of an [N x K] matrix, seen as
-// [ceil(N/16)] x [K/128] tiles of 128 32-bit words (one box = 16 row blocks
-// of one k tile).
-int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, void *out128);
+// [ceil(N/16)] x [K/128] tiles of 128 32-bit words (one box = box_rb row
+// blocks of one k tile; row blocks past the matrix read as zero).
+int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, int box_rb, void *out128);
 
 cudaError_t launch_wait_probe(uint32_t *err, uint64_t timeout_ns, cudaStream_t stream);
 

@@ -29,6 +29,7 @@
 
 #include "tw_device.cuh"
 #include "tw_internal.h"
+#include "tw_tc.cuh"
 
 namespace tw {
 namespace {
@@ -108,98 +109,6 @@ struct TileIter {
             locate(p);
     }
 };
-
-// ------------------------------------------------------------- tcgen05 PTX
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
-{
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 ::"r"(dst_smem), "r"(ncols) : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
-{
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::i8, int32 accumulate.
-__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrive on `bar` when every MMA issued so far by this thread has completed.
-__device__ __forceinline__ void mma_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 ::"r"(bar) : "memory");
-}
-
-// 32 lanes x 32 consecutive 32-bit columns: thread i gets row (lane base + i).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
-          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
-          "=r"(v[31])
-        : "r"(taddr)
-        : "memory");
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// 3-D TMA load of one box into shared memory (no multicast).
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int32_t x, int32_t y,
-                                            int32_t z, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];"
-        ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar)
-        : "memory");
-}
-
-// 2-D TMA load of one box into shared memory (no multicast).
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int32_t x, int32_t y,
-                                            uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle,
-// 8-row groups 1024 bytes apart (SBO), leading offset unused (1).
-__device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr)
-{
-    uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
-    d |= (uint64_t)1 << 16;
-    d |= (uint64_t)(1024 >> 4) << 32;
-    d |= (uint64_t)1 << 46;   // descriptor version for sm_100
-    d |= (uint64_t)2 << 61;   // 128-byte swizzle
-    return d;
-}
 
 // Instruction descriptor: int8 x int8 -> int32, both K-major, M = 128, N = 256.
 constexpr uint32_t kIdesc = (2u << 4)            // D format: s32
@@ -515,7 +424,7 @@ int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, void *out128)
     return 0;
 }
 
-int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, void *out128)
+int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, int box_rb, void *out128)
 {
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
@@ -532,7 +441,7 @@ int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, void *out128)
     const int64_t KT = K / kTileK, nrb = (N + kTileRows - 1) / kTileRows;
     const cuuint64_t dims[3] = {(cuuint64_t)(kTileBytes / 4), (cuuint64_t)KT, (cuuint64_t)nrb};
     const cuuint64_t strides[2] = {(cuuint64_t)kTileBytes, (cuuint64_t)(KT * kTileBytes)};
-    const cuuint32_t box[3] = {kTileBytes / 4, 1, kBN / kTileRows};
+    const cuuint32_t box[3] = {kTileBytes / 4, 1, (cuuint32_t)box_rb};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t *>(packed), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,

@@ -65,12 +65,12 @@ def _descs(shapes, base=0x10000):
 REC = np.dtype([("x", "<u8"), ("xq", "<u8"), ("amax", "<u8"), ("qsum", "<u8"),
                 ("packed", "<u8"), ("wscale", "<u8"), ("y", "<u8"), ("acc_out", "<u8"),
                 ("N", "<i8"), ("K", "<i8"), ("rb_begin", "<i8"), ("tile_begin", "<i8"),
-                ("ptile_begin", "<i8"), ("ws_xq_off", "<i8"), ("unit_begin", "<i8"),
-                ("urb", "<i8"),
+                ("ptile_begin", "<i8"), ("ws_xq_off", "<i8"), ("cost_begin", "<i8"),
+                ("tmap_ok", "<i8"),
                 ("tmap", "u1", 128), ("tmap_codes", "u1", 128)])
 HDR = np.dtype([("magic", "<u4"), ("count", "<i4"), ("M", "<i8"), ("total_rb", "<i8"),
-                ("total_tiles", "<i8"), ("total_ptiles", "<i8"), ("max_K", "<i8"),
-                ("total_units", "<i8"), ("ws_bytes", "<i8")])
+                ("total_units", "<i8"), ("total_ptiles", "<i8"), ("max_K", "<i8"),
+                ("total_cost", "<i8"), ("ws_bytes", "<i8")])
 
 
 def test_table_encode_prefix_sums(lib):
@@ -78,32 +78,40 @@ def test_table_encode_prefix_sums(lib):
     shapes = [(1536, 1536), (256, 1536), (17, 256), (1536, 8960)]
     arr = _descs(shapes)
     n = api.tw_sweep_table_bytes(len(shapes))
-    assert n == 64 + 384 * len(shapes)
+    assert n == 64 + (384 + 16) * len(shapes)   # header, records, unit order
     buf = np.zeros(n, np.uint8)
     rc = api.tw_sweep_table_encode(arr, len(shapes), 1, buf.ctypes.data, n)
     assert rc == 0, api.tw_last_error()
     hdr = buf[:64].view(HDR)[0]
-    recs = buf[64:].view(REC)
+    recs = buf[64:64 + 384 * len(shapes)].view(REC)
+    order = buf[64 + 384 * len(shapes):].view(np.dtype([("d", "<i4"), ("units", "<i4"),
+                                                          ("unit_begin", "<i8")]))
     assert hdr["magic"] == 0x54574431 and hdr["count"] == 4 and hdr["M"] == 1
     nrb = [-(-N // 16) for N, K in shapes]
     ntiles = [r * (K // 128) for r, (N, K) in zip(nrb, shapes)]
     assert recs["rb_begin"].tolist() == np.concatenate([[0], np.cumsum(nrb)[:-1]]).tolist()
     assert recs["tile_begin"].tolist() == np.concatenate([[0], np.cumsum(ntiles)[:-1]]).tolist()
-    assert hdr["total_rb"] == sum(nrb) and hdr["total_tiles"] == sum(ntiles)
-    assert hdr["max_K"] == 8960
-    urb = [max(1, 65536 // (4 * K)) for N, K in shapes]
-    assert recs["urb"].tolist() == urb
-    units = [-(-r // u) for r, u in zip(nrb, urb)]
-    assert recs["unit_begin"].tolist() == np.concatenate([[0], np.cumsum(units)[:-1]]).tolist()
+    assert hdr["total_rb"] == sum(nrb)
+    # tensor-core units: 128 rows each, projections of larger K first (stable)
+    assert order["d"].tolist() == [3, 0, 1, 2]
+    units = [-(-shapes[d][0] // 128) for d in order["d"]]
+    assert order["units"].tolist() == units
+    assert order["unit_begin"].tolist() == np.concatenate([[0], np.cumsum(units)[:-1]]).tolist()
     assert hdr["total_units"] == sum(units)
+    assert hdr["max_K"] == 8960
+    # static split by cost: 16 units per 128-column tile + 45 per row block
+    cost = [r * (16 * (K // 128) + 45) for r, (N, K) in zip(nrb, shapes)]
+    assert recs["cost_begin"].tolist() == np.concatenate([[0], np.cumsum(cost)[:-1]]).tolist()
+    assert hdr["total_cost"] == sum(cost)
     assert recs["N"].tolist() == [s[0] for s in shapes]
-    # scratch: 256 B of counters, one flag per (projection, token), int8 rows, scales
-    xq = [-(-K // 128) * 128 for N, K in shapes]   # M = 1 rows, 128-byte aligned
-    head = 256 + 128
+    # scratch: 256 bytes of counters, then per projection room for 8 token
+    # rows (the tensor-core blocks of M <= 8), then the scales
+    xq = [8 * K for N, K in shapes]
+    head = 256
     assert recs["ws_xq_off"].tolist() == (head + np.concatenate([[0], np.cumsum(xq)[:-1]])).tolist()
     assert hdr["ws_bytes"] == head + sum(xq) + 256 * len(shapes)
     assert api.tw_sweep_workspace_bytes(buf.ctypes.data) == hdr["ws_bytes"]
-    assert api.tw_sweep_launches(buf.ctypes.data) in (1, 2)   # dynamic path or quantise + decode
+    assert api.tw_sweep_launches(buf.ctypes.data) == 2   # quantise + decode
 
 
 @pytest.mark.parametrize("bad,status", [
