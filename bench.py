@@ -328,7 +328,9 @@ def main():
         achieved = algo_bytes / (ms_per_step / 1e3) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                     "frac": achieved / hbm,
-                    "traffic": profiled_traffic("tw_decode.cu", M, args.layers),
+                    # sweeps of more than 16 tokens run the tensor-core decode kernel
+                    "traffic": profiled_traffic("tw_decode_tc.cu" if M > 16 else "tw_decode.cu",
+                                                M, args.layers),
                     "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured"
                     else "fallback 6650 GB/s",
                     "algorithmic_bytes_per_step": algo_bytes,

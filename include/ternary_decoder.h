@@ -203,23 +203,33 @@ TW_API size_t tw_sweep_table_bytes(int count);
  * tw_sweep_table_bytes(count)).  The caller copies the table to device
  * memory (64-byte aligned) and passes that copy to
  * tw_decoder_projection_sweep; the table stays valid for as long as the
- * buffers it names do.  For M > 32 it embeds TMA descriptors of each xq and
- * therefore needs the CUDA driver.
+ * buffers it names do.  Layout: a 64-byte header, one 384-byte record per
+ * projection, then one 16-byte entry per projection giving the order in
+ * which the tensor-core decode sweep hands out its 128-row units
+ * (projections of larger K first).  The records embed TMA descriptors --
+ * of each xq (M > 32) and of the packed codes (every M) -- and therefore
+ * need the CUDA driver: a decode table encoded where the driver is missing
+ * still answers the size queries, but the sweep refuses it (TW_ERR_CUDA).
  */
 TW_API int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M,
                           void *table, size_t table_bytes);
 
-/* Scratch needed by tw_decoder_projection_sweep for an encoded HOST table:
- * for decode (M <= 32) the quantised rows of every projection and their
- * scales, rewritten by every call (no initial contents needed); 0 for
- * prefill, whose callers pass the quantised rows in the descriptors. */
+/* Scratch needed by tw_decoder_projection_sweep for an encoded HOST table;
+ * 0 for prefill, whose callers pass the quantised rows in the descriptors.
+ * For decode (M <= 32) it holds 256 bytes of work counters, then the
+ * quantised rows of every projection (room for 8, 16 or 32 token rows of K
+ * bytes) and their scales.  It must be zero-filled before its first use
+ * with a table; every call leaves the counters zero again (after
+ * TW_ERR_TIMEOUT, zero it again). */
 TW_API size_t tw_sweep_workspace_bytes(const void *table_host);
 
 /*
- * Run the layer over every projection of an encoded table: one persistent
- * launch for decode (M <= 32; two or more only when M*K of the widest
- * projection does not fit shared memory and the tokens are split into
- * groups), one grouped tensor-core launch for prefill.
+ * Run the layer over every projection of an encoded table.  Decode
+ * (M <= 32): one quantisation launch, then for M <= 16 one persistent
+ * launch of the register (mma.sync) kernel -- more only when M*K of the
+ * widest projection does not fit shared memory and the tokens are split
+ * into groups -- and for 16 < M <= 32 one launch of the tensor-core decode
+ * kernel.  Prefill (M > 32): one grouped tensor-core launch.
  *   table_host  the host table written by tw_sweep_table_encode (read for the
  *               launch configuration: count, M, sizes);
  *   table_dev   the caller's device copy of the same bytes (64-byte aligned),
