@@ -43,9 +43,9 @@ namespace {
 
 constexpr int kCT = 8;                      // tiles per ring chunk
 constexpr int kChunk = kCT * kTileBytes;    // 4 KB
-constexpr int kMaxXB = 4;                   // activation buffers
+constexpr int kXE = 8;                      // activation ring entries
 constexpr int kSmemLimit = 227 * 1024;
-constexpr int kMiscBytes = 2048 + 256 * kMaxXB;  // barriers, token info, plan
+constexpr int kMiscBytes = 2048 + 256 * kXE;  // token info, barriers, plan, entry offsets
 constexpr uint64_t kDrainNs = 1000000000ull;
 constexpr int kQThreads = 256;
 constexpr int kQRegs = 12;                  // float4 per thread kept in registers
@@ -56,8 +56,8 @@ struct DecodeParams {
     int count;
     int M;
     int m0, mg;               // token group [m0, m0 + mg)
-    int xb;                   // activation buffers (1..4)
-    int xs;                   // activation row stride in shared memory
+    int xcap;                 // bytes of the activation ring (multiple of 128)
+    int xs;                   // max_K + 64: bytes of the zero row
     int slots;                // ring slots per consumer warp
     int64_t total_rb, total_cost;
     const uint8_t *ws;        // quantised activations (launch 1 output)
@@ -70,6 +70,7 @@ struct QuantParams {
     DescRecord single;
     int count, M;
     int ntok;                 // 0: plain int8 rows; 8/16/32: tensor-core token blocks
+    int wpr;                  // warps per row (set by launch_quant_rows)
     uint8_t *ws;
     int64_t ws_sa_off;
 };
@@ -127,46 +128,63 @@ __device__ __forceinline__ int64_t tc_block_offset(int64_t idx, int m, int ntok)
     return (idx >> 5) * (int64_t)ntok * 128 + m * 128 + ((((c >> 2) ^ (m & 7)) << 4) | ((c & 3) << 2));
 }
 
-// Block (d, m): quantise token row m of projection d.  amax = max|x|,
-// scale = 127/amax (IEEE fp32), q = clamp(rint(x*scale), -128, 127).
+// Quantise token row m of projection d.  amax = max|x|, scale = 127/amax
+// (IEEE fp32), q = clamp(rint(x*scale), -128, 127).  A row is handled by
+// p.wpr warps (1, 2, 4 or 8; more when there are few rows, so that the
+// launch fills the GPU in one wave of short rows); a block of 8 warps holds
+// 8 / wpr rows.  Each row is held in registers when it fits, else read twice.
 __global__ void __launch_bounds__(kQThreads) k_quant_rows(const __grid_constant__ QuantParams p)
 {
     pdl_launch_dependents();
     __shared__ float red_f[kQThreads / 32];
     __shared__ int red_i[kQThreads / 32];
-    const int d = blockIdx.x / p.M, m = blockIdx.x % p.M;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int wpr = p.wpr, rloc = warp / wpr, wr = warp % wpr;
+    const int64_t row_id = (int64_t)blockIdx.x * (kQThreads / 32 / wpr) + rloc;
+    const bool live = row_id < (int64_t)p.count * p.M;
+    const int d = live ? (int)(row_id / p.M) : 0, m = live ? (int)(row_id % p.M) : 0;
     const DescRecord &r = rec(p, d);
-    const int64_t K4 = r.K / 4;
+    const int64_t K4 = live ? r.K / 4 : 0;
     const float4 *row = reinterpret_cast<const float4 *>(r.x + (int64_t)m * r.K);
     uint32_t *qrow = reinterpret_cast<uint32_t *>(p.ws + r.ws_xq_off + (int64_t)m * r.K);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bool in_regs = K4 <= (int64_t)kQRegs * kQThreads;
+    const int T = 32 * wpr, ti = 32 * wr + lane;   // threads of the row, index within it
+    const bool in_regs = K4 <= (int64_t)kQRegs * T;
 
     float4 v[kQRegs];
     float a = 0.f;
     if (in_regs) {
 #pragma unroll
         for (int i = 0; i < kQRegs; ++i) {
-            const int64_t idx = tid + (int64_t)i * kQThreads;
+            const int64_t idx = ti + (int64_t)i * T;
             v[i] = idx < K4 ? __ldg(row + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int i = 0; i < kQRegs; ++i)
             a = fmaxf(a, amax4(v[i]));
     } else {
-        for (int64_t i = tid; i < K4; i += kQThreads)
-            a = fmaxf(a, amax4(__ldg(row + i)));
+        // batches of kQRegs independent loads per thread
+        for (int64_t b0 = ti; b0 < K4; b0 += (int64_t)kQRegs * T) {
+#pragma unroll
+            for (int i = 0; i < kQRegs; ++i) {
+                const int64_t idx = b0 + (int64_t)i * T;
+                v[i] = idx < K4 ? __ldg(row + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int i = 0; i < kQRegs; ++i)
+                a = fmaxf(a, amax4(v[i]));
+        }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1)
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if (lane == 0)
-        red_f[warp] = a;
-    __syncthreads();
-    a = red_f[0];
-#pragma unroll
-    for (int w = 1; w < kQThreads / 32; ++w)
-        a = fmaxf(a, red_f[w]);
+    if (wpr > 1) {  // (uniform over the block)
+        if (lane == 0)
+            red_f[warp] = a;
+        __syncthreads();
+        a = red_f[rloc * wpr];
+        for (int w = 1; w < wpr; ++w)
+            a = fmaxf(a, red_f[rloc * wpr + w]);
+    }
 
     const bool zero = (a == 0.f);
     const float scale = zero ? 0.f : __fdiv_rn(127.f, a);
@@ -175,7 +193,7 @@ __global__ void __launch_bounds__(kQThreads) k_quant_rows(const __grid_constant_
     if (in_regs) {
 #pragma unroll
         for (int i = 0; i < kQRegs; ++i) {
-            const int64_t idx = tid + (int64_t)i * kQThreads;
+            const int64_t idx = ti + (int64_t)i * T;
             if (idx < K4) {
                 const uint32_t u = quant4(v[i], scale, zero, sum);
                 if (p.ntok)
@@ -185,28 +203,64 @@ __global__ void __launch_bounds__(kQThreads) k_quant_rows(const __grid_constant_
             }
         }
     } else {
-        for (int64_t i = tid; i < K4; i += kQThreads) {
-            const uint32_t u = quant4(__ldg(row + i), scale, zero, sum);
-            if (p.ntok)
-                *reinterpret_cast<uint32_t *>(blocks + tc_block_offset(i, m, p.ntok)) = u;
-            else
-                qrow[i] = u;
+        for (int64_t b0 = ti; b0 < K4; b0 += (int64_t)kQRegs * T) {
+#pragma unroll
+            for (int i = 0; i < kQRegs; ++i) {
+                const int64_t idx = b0 + (int64_t)i * T;
+                v[i] = idx < K4 ? __ldg(row + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int i = 0; i < kQRegs; ++i) {
+                const int64_t idx = b0 + (int64_t)i * T;
+                if (idx < K4) {
+                    const uint32_t u = quant4(v[i], scale, zero, sum);
+                    if (p.ntok)
+                        *reinterpret_cast<uint32_t *>(blocks + tc_block_offset(idx, m, p.ntok)) = u;
+                    else
+                        qrow[idx] = u;
+                }
+            }
         }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1)
         sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0)
-        red_i[warp] = sum;
-    __syncthreads();
-    if (tid == 0) {
-        int s = 0;
-        for (int w = 0; w < kQThreads / 32; ++w)
-            s += red_i[w];
+    if (wpr > 1) {
+        if (lane == 0)
+            red_i[warp] = sum;
+        __syncthreads();
+        sum = 0;
+        for (int w = 0; w < wpr; ++w)
+            sum += red_i[rloc * wpr + w];
+    }
+    if (live && ti == 0) {
         uint8_t *info = p.ws + p.ws_sa_off + 256 * (int64_t)d;
         reinterpret_cast<float *>(info)[m] = __fdiv_rn(a, 127.f);
-        reinterpret_cast<int *>(info + 128)[m] = s;
+        reinterpret_cast<int *>(info + 128)[m] = sum;
     }
+}
+
+// Warps per row for `rows` rows: enough warps in flight to fill the GPU
+// (about 24 resident per SM at this kernel's register use) in one wave.
+int quant_warps_per_row(int64_t rows, int sms)
+{
+    const int64_t target = (int64_t)sms * 24;
+    int w = 8;
+    while (w > 1 && rows * w > target)
+        w >>= 1;
+    return w;
+}
+
+cudaError_t launch_quant_rows(QuantParams &q, cudaStream_t stream)
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t rows = (int64_t)q.count * q.M;
+    q.wpr = quant_warps_per_row(rows, sms);
+    const int64_t per_block = kQThreads / 32 / q.wpr;
+    k_quant_rows<<<(unsigned)((rows + per_block - 1) / per_block), kQThreads, 0, stream>>>(q);
+    return cudaGetLastError();
 }
 
 // ----------------------------------------------------------------- launch 2
@@ -357,27 +411,31 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
     constexpr int kThr = (NC + 1) * 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // Layout: rings | zero row (at 64 mod 128) | activation buffers (rows at
-    // 0 mod 128, stride xs = 64 mod 128) | token info | barriers | plan.
+    // Layout: rings | zero row (at 64 mod 128) | activation ring (xcap bytes,
+    // 0 mod 128) | token info | barriers | plan | entry offsets.
+    // The activation ring holds one entry per projection in flight: its mg
+    // int8 rows at stride K + 64 (rows 64 bytes apart mod 128, so the
+    // 16-byte token loads of a warp hit distinct banks), starting at 0 mod
+    // 128; entries are allocated in order and freed in order.
     const int ring_bytes = NC * p.slots * kChunk;
     uint8_t *ring = smem;
     uint8_t *zero_row = smem + ring_bytes + 64;
     uint8_t *xbase = smem + ring_bytes + 64 + p.xs;  // = ring + K + 128: 0 mod 128
-    const int xbuf_bytes = p.mg * p.xs;
-    uint8_t *misc = xbase + p.xb * xbuf_bytes + 128;
+    uint8_t *misc = xbase + p.xcap + 128;
     misc += (128 - (smem_u32(misc) & 127)) & 127;
-    uint8_t *info = misc;                                    // [xb][256]: sa[32], qs[32]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(misc + 256 * kMaxXB);
-    // bars: ring_full[NC*slots], x_full[kMaxXB], x_empty[kMaxXB]
-    Plan *plan = reinterpret_cast<Plan *>(misc + 256 * kMaxXB + 8 * (NC * p.slots + 2 * kMaxXB));
+    uint8_t *info = misc;                                    // [kXE][256]: sa[32], qs[32]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(misc + 256 * kXE);
+    // bars: ring_full[NC*slots], x_full[kXE], x_empty[kXE]
+    Plan *plan = reinterpret_cast<Plan *>(misc + 256 * kXE + 8 * (NC * p.slots + 2 * kXE));
+    volatile int *xoff = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(plan) + 64);
     const uint32_t bar_ring = smem_u32(bars);
     const uint32_t bar_xfull = bar_ring + 8 * NC * p.slots;
-    const uint32_t bar_xempty = bar_xfull + 8 * kMaxXB;
+    const uint32_t bar_xempty = bar_xfull + 8 * kXE;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NC * p.slots; ++i)
             mbar_init(bar_ring + 8 * i, 1);
-        for (int b = 0; b < kMaxXB; ++b) {
+        for (int b = 0; b < kXE; ++b) {
             mbar_init(bar_xfull + 8 * b, 1);
             mbar_init(bar_xempty + 8 * b, NC * 32);
         }
@@ -404,27 +462,49 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
         // ------------------------------------------------ activation warp
         if (lane == 0) {
             pdl_wait();  // launch 1 has finished writing the int8 rows
-            for (int d = pl.d_lo; d <= pl.d_hi; ++d) {
-                const int seg = d - pl.d_lo, b = seg % p.xb;
-                if (seg >= p.xb &&
-                    !mbar_wait(bar_xempty + 8 * b, ((seg / p.xb) - 1) & 1, p.ctl, abort_flag))
-                    break;
+            // Positions are counted monotonically; entry seg lives at
+            // start[seg % kXE] mod xcap.  `tail` is the oldest entry not yet
+            // known to be free.
+            int64_t head = 0, start[kXE];
+            int tail = 0;
+            bool ok = true;
+            for (int d = pl.d_lo; d <= pl.d_hi && ok; ++d) {
+                const int seg = d - pl.d_lo, e = seg % kXE;
                 const DescRecord &r = rec(p, d);
-                const uint32_t bx = bar_xfull + 8 * b;
-                const uint32_t dst = smem_u32(xbase + b * xbuf_bytes);
+                const int64_t rs = r.K + 64;
+                const int64_t size = (p.mg * rs + 127) / 128 * 128;
+                int64_t pos = head;
+                if (pos % p.xcap + size > p.xcap)  // an entry never wraps
+                    pos = (pos / p.xcap + 1) * p.xcap;
+                // free entries (in order) until the slot and the bytes are available
+                while (tail < seg && (seg - tail >= kXE || pos + size - start[tail % kXE] > p.xcap)) {
+                    if (!mbar_wait(bar_xempty + 8 * (tail % kXE), (tail / kXE) & 1, p.ctl, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    ++tail;
+                }
+                if (!ok)
+                    break;
+                start[e] = pos;
+                head = pos + size;
+                const int off = (int)(pos % p.xcap);
+                xoff[e] = off;
+                const uint32_t bx = bar_xfull + 8 * e;
+                const uint32_t dst = smem_u32(xbase + off);
                 mbar_arrive_expect_tx(bx, (uint32_t)(p.mg * r.K + 256));
                 for (int tok = 0; tok < p.mg; ++tok)
-                    bulk_g2s(dst + tok * p.xs, p.ws + r.ws_xq_off + (int64_t)(p.m0 + tok) * r.K,
+                    bulk_g2s(dst + tok * (uint32_t)rs, p.ws + r.ws_xq_off + (int64_t)(p.m0 + tok) * r.K,
                              (uint32_t)r.K, bx);
-                bulk_g2s(smem_u32(info + 256 * b), p.ws + p.ws_sa_off + 256 * (int64_t)d, 256, bx);
+                bulk_g2s(smem_u32(info + 256 * e), p.ws + p.ws_sa_off + 256 * (int64_t)d, 256, bx);
             }
-            // Drain: the activation copies of the last buffers land before exit.
+            // Drain: the activation copies of the last entries land before exit.
             WaitCtl drain = p.ctl;
             drain.timeout_ns = kDrainNs;
             const int nseg = pl.d_hi - pl.d_lo + 1;
-            for (int seg = nseg - p.xb; seg < nseg; ++seg)
+            for (int seg = nseg - kXE; seg < nseg; ++seg)
                 if (seg >= 0)
-                    mbar_wait(bar_xfull + 8 * (seg % p.xb), (seg / p.xb) & 1, drain, nullptr);
+                    mbar_wait(bar_xfull + 8 * (seg % kXE), (seg / kXE) & 1, drain, nullptr);
         }
         __syncwarp();
         return;
@@ -453,8 +533,8 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
 
     bool ok = true;
     for (int d = pl.d_lo; d <= pl.d_hi && ok; ++d) {
-        const int seg = d - pl.d_lo, b = seg % p.xb;
-        if (!mbar_wait(bar_xfull + 8 * b, (seg / p.xb) & 1, p.ctl, abort_flag)) {
+        const int seg = d - pl.d_lo, b = seg % kXE;
+        if (!mbar_wait(bar_xfull + 8 * b, (seg / kXE) & 1, p.ctl, abort_flag)) {
             ok = false;
             break;
         }
@@ -470,7 +550,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int tok = 8 * nt + g;
-            xrow[nt] = (tok < p.mg ? smem_u32(xbase + b * xbuf_bytes + tok * p.xs) : zero_s) +
+            xrow[nt] = (tok < p.mg ? smem_u32(xbase + xoff[b]) + tok * (uint32_t)(r.K + 64) : zero_s) +
                        16 * t;
         }
 
@@ -571,15 +651,15 @@ __global__ void k_wait_probe(WaitCtl ctl)
 // registers for the wider accumulators of larger token groups.
 // The block is a multiple of 4 warps so that each SM sub-partition's
 // register file holds the same number of warps (16, 12 or 8 in total).
-template <int NT>
-constexpr int consumers() { return NT == 1 ? 15 : NT == 2 ? 11 : 7; }
+// Consumer warps per block: more warps hide more latency, fewer leave
+// registers for the wider accumulators of larger token groups and shared
+// memory for their activation rows.  The block is a multiple of 4 warps so
+// that each SM sub-partition's register file holds the same number of warps.
+int max_consumers(int nt) { return nt == 1 ? 15 : nt == 2 ? 11 : 7; }
 
-int consumers_for(int mg) { const int nt = (mg + 7) / 8; return nt == 1 ? 15 : nt == 2 ? 11 : 7; }
-
-template <int NT>
+template <int NT, int NC>
 cudaError_t launch_nt(const DecodeParams &p, int grid, int smem, cudaStream_t stream)
 {
-    constexpr int NC = consumers<NT>();
     cudaError_t e = cudaFuncSetAttribute(k_decode<NT, NC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
@@ -599,36 +679,54 @@ cudaError_t launch_nt(const DecodeParams &p, int grid, int smem, cudaStream_t st
 }
 
 // Bytes of dynamic shared memory of k_decode for this plan.
-int64_t smem_bytes(int nc, int slots, int mg, int xb, int64_t max_K)
+int64_t smem_bytes(int nc, int slots, int xcap, int64_t max_K)
 {
     const int64_t xs = max_K + 64;
-    return 1024 + (int64_t)nc * slots * kChunk + xs + 128 + (int64_t)xb * mg * xs + 256 +
-           kMiscBytes;
+    return 1024 + (int64_t)nc * slots * kChunk + xs + 128 + xcap + 256 + kMiscBytes;
 }
 
-// Largest token group, then deepest ring (4..2 slots, 3..2 with 15 warps),
-// then most activation buffers (at least 2 when that fits) for the budget.
-bool plan_decode(int M, int64_t max_K, int *mg_out, int *slots_out, int *xb_out)
+struct DecodePlan {
+    int mg, nc, slots, xcap;
+};
+
+// Largest token group; for it the most consumer warps (max_consumers, then
+// 4 fewer at a time down to 7); for those the deepest ring of code slots
+// (4..2, 3..2 with 15 warps) that leaves the activation ring room for two
+// entries of the widest projection, else for one; the ring takes the rest
+// of the budget.
+bool plan_decode(int M, int64_t max_K, DecodePlan *out)
 {
     int mg = M;
     while (true) {
-        const int nc = consumers_for(mg);
-        const int smax = nc >= 15 ? 3 : 4;
-        for (int need_xb = 2; need_xb >= 1; --need_xb)
-            for (int s = smax; s >= 2; --s)
-                if (smem_bytes(nc, s, mg, need_xb, max_K) <= kSmemLimit) {
-                    int xb = need_xb;
-                    while (xb < kMaxXB && smem_bytes(nc, s, mg, xb + 1, max_K) <= kSmemLimit)
-                        ++xb;
-                    *mg_out = mg;
-                    *slots_out = s;
-                    *xb_out = xb;
-                    return true;
+        const int nt = (mg + 7) / 8;
+        const int64_t entry = (mg * (max_K + 64) + 127) / 128 * 128;
+        for (int nc = max_consumers(nt); nc >= 7; nc -= 4)
+            for (int need = 2; need >= 1; --need)
+                for (int s = nc >= 15 ? 3 : 4; s >= 2; --s) {
+                    const int64_t rest = kSmemLimit - smem_bytes(nc, s, 0, max_K);
+                    const int64_t xcap = rest / 128 * 128;
+                    if (xcap >= need * entry) {
+                        *out = DecodePlan{mg, nc, s, (int)xcap};
+                        return true;
+                    }
                 }
         if (mg == 1)
             return false;
         mg = mg > 8 ? mg - 8 : mg - 1;
     }
+}
+
+cudaError_t launch_plan(const DecodeParams &p, const DecodePlan &g, int grid, int smem,
+                        cudaStream_t stream)
+{
+    const int nt = (p.mg + 7) / 8;
+    if (nt == 1 && g.nc == 15) return launch_nt<1, 15>(p, grid, smem, stream);
+    if (nt == 1 && g.nc == 11) return launch_nt<1, 11>(p, grid, smem, stream);
+    if (nt == 1) return launch_nt<1, 7>(p, grid, smem, stream);
+    if (nt == 2 && g.nc == 11) return launch_nt<2, 11>(p, grid, smem, stream);
+    if (nt == 2) return launch_nt<2, 7>(p, grid, smem, stream);
+    if (nt == 3) return launch_nt<3, 7>(p, grid, smem, stream);
+    return launch_nt<4, 7>(p, grid, smem, stream);
 }
 
 }  // namespace
@@ -644,16 +742,15 @@ cudaError_t launch_quant_tc(const DescRecord *table, int count, int64_t M, int n
     q.ntok = ntok;
     q.ws = ws;
     q.ws_sa_off = ws_sa_off;
-    k_quant_rows<<<(unsigned)(count * M), kQThreads, 0, stream>>>(q);
-    return cudaGetLastError();
+    return launch_quant_rows(q, stream);
 }
 
 int decode_launches(int64_t M, int64_t max_K)
 {
-    int mg = 1, slots = 2, xb = 1;
-    if (!plan_decode((int)M, max_K, &mg, &slots, &xb))
+    DecodePlan g{};
+    if (!plan_decode((int)M, max_K, &g))
         return 0;
-    return 1 + (int)((M + mg - 1) / mg);  // quantise + one decode launch per group
+    return 1 + (int)((M + g.mg - 1) / g.mg);  // quantise + one decode launch per group
 }
 
 cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout_ns,
@@ -666,8 +763,8 @@ cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout
     if (e != cudaSuccess)
         return e;
     const int M = (int)L.M;
-    int mg = 1, slots = 2, xb = 1;
-    if (!plan_decode(M, L.max_K, &mg, &slots, &xb))
+    DecodePlan g{};
+    if (!plan_decode(M, L.max_K, &g))
         return cudaErrorInvalidValue;
 
     // Launch 1: quantise every (projection, token) row.
@@ -680,8 +777,7 @@ cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout
     q.M = M;
     q.ws = L.ws;
     q.ws_sa_off = L.ws_sa_off;
-    k_quant_rows<<<(unsigned)(L.count * (int64_t)M), kQThreads, 0, stream>>>(q);
-    e = cudaGetLastError();
+    e = launch_quant_rows(q, stream);
     if (e != cudaSuccess)
         return e;
 
@@ -699,22 +795,16 @@ cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout
     p.ws_sa_off = L.ws_sa_off;
     p.ctl.err = err;
     p.ctl.timeout_ns = timeout_ns;
-    p.slots = slots;
-    p.xb = xb;
-    const int smem = (int)smem_bytes(consumers_for(mg), slots, mg, xb, L.max_K);
+    p.slots = g.slots;
+    p.xcap = g.xcap;
+    const int smem = (int)smem_bytes(g.nc, g.slots, g.xcap, L.max_K);
     const int64_t grid64 = L.total_rb < sms ? L.total_rb : sms;
     const int grid = (int)(grid64 < 1 ? 1 : grid64);
 
-    for (int m0 = 0; m0 < M; m0 += mg) {
+    for (int m0 = 0; m0 < M; m0 += g.mg) {
         p.m0 = m0;
-        p.mg = (M - m0) < mg ? (M - m0) : mg;
-        const int nt = (p.mg + 7) / 8;
-        switch (nt) {
-        case 1: e = launch_nt<1>(p, grid, smem, stream); break;
-        case 2: e = launch_nt<2>(p, grid, smem, stream); break;
-        case 3: e = launch_nt<3>(p, grid, smem, stream); break;
-        default: e = launch_nt<4>(p, grid, smem, stream); break;
-        }
+        p.mg = (M - m0) < g.mg ? (M - m0) : g.mg;
+        e = launch_plan(p, g, grid, smem, stream);
         if (e != cudaSuccess)
             return e;
     }
