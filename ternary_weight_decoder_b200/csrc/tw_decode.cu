@@ -45,7 +45,9 @@ constexpr int kCT = 8;                      // tiles per ring chunk
 constexpr int kChunk = kCT * kTileBytes;    // 4 KB
 constexpr int kXE = 8;                      // activation ring entries
 constexpr int kSmemLimit = 227 * 1024;
-constexpr int kMiscBytes = 2048 + 256 * kXE;  // token info, barriers, plan, entry offsets
+constexpr int kPC = 32;                     // projections cached in shared memory per block
+constexpr int kMiscBytes = 2048 + 256 * kXE + 64 * kPC;  // token info, barriers, plan,
+                                                          // entry offsets, projection cache
 constexpr uint64_t kDrainNs = 1000000000ull;
 constexpr int kQThreads = 256;
 constexpr int kQRegs = 12;                  // float4 per thread kept in registers
@@ -304,6 +306,36 @@ __device__ int desc_of_rb(const DecodeParams &p, int64_t rb)
     return lo;
 }
 
+// The fields of one projection that the decode block needs, copied once
+// into shared memory (the first kPC projections of the block's share), so
+// that moving to the next projection reads no global memory.
+struct ProjC {
+    const uint8_t *packed;
+    float *y;
+    int32_t *acc_out;
+    int64_t N;
+    int64_t ws_xq_off;
+    int rb_begin, rb_end, KT, K;
+    float wscale;
+    int pad;
+};
+static_assert(sizeof(ProjC) == 64, "projection cache entry");
+
+__device__ __forceinline__ ProjC load_proj(const DecodeParams &p, int d)
+{
+    const DescRecord &r = rec(p, d);
+    return ProjC{r.packed, r.y, r.acc_out, r.N, r.ws_xq_off, (int)r.rb_begin,
+                 (int)(r.rb_begin + rb_count(r)), (int)(r.K / kTileK), (int)r.K, __ldg(r.wscale), 0};
+}
+
+// Projection d of a block whose share starts at projection d0: from the
+// cache when it is there.
+__device__ __forceinline__ ProjC get_proj(const DecodeParams &p, const ProjC *pc, int d0, int npc,
+                                          int d)
+{
+    return d - d0 < npc ? pc[d - d0] : load_proj(p, d);
+}
+
 // Walks the chunks of one consumer warp: every NC-th row block of the CTA
 // share, each cut into ceil(KT / kCT) chunks.  The fields of the current
 // projection are cached here so that issuing a chunk reads no global memory.
@@ -313,14 +345,16 @@ struct ChunkIter {
     int rb, rb_begin, rb_end, rb_hi;   // row-block indices (< 2^31)
     int d, kc, nch, KT;
     bool valid;
+    const ProjC *pc;                   // projection cache of the block
+    int d0, npc;
 
     __device__ void load_desc(const DecodeParams &p)
     {
-        const DescRecord &r = rec(p, d);
-        packed = r.packed;
-        rb_begin = (int)r.rb_begin;
-        rb_end = (int)(r.rb_begin + rb_count(r));
-        KT = (int)(r.K / kTileK);
+        const ProjC c = get_proj(p, pc, d0, npc, d);
+        packed = c.packed;
+        rb_begin = c.rb_begin;
+        rb_end = c.rb_end;
+        KT = c.KT;
         nch = (KT + kCT - 1) / kCT;
     }
     __device__ void seek(const DecodeParams &p)
@@ -330,8 +364,12 @@ struct ChunkIter {
             load_desc(p);
         }
     }
-    __device__ void init(const DecodeParams &p, const Plan &pl, int w)
+    __device__ void init(const DecodeParams &p, const Plan &pl, int w, const ProjC *cache,
+                         int ncache)
     {
+        pc = cache;
+        d0 = pl.d_lo;
+        npc = ncache;
         rb = (int)pl.rb_lo + w;
         rb_hi = (int)pl.rb_hi;
         kc = 0;
@@ -428,6 +466,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
     // bars: ring_full[NC*slots], x_full[kXE], x_empty[kXE]
     Plan *plan = reinterpret_cast<Plan *>(misc + 256 * kXE + 8 * (NC * p.slots + 2 * kXE));
     volatile int *xoff = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(plan) + 64);
+    ProjC *pcache = reinterpret_cast<ProjC *>(reinterpret_cast<uint8_t *>(plan) + 128);
     const uint32_t bar_ring = smem_u32(bars);
     const uint32_t bar_xfull = bar_ring + 8 * NC * p.slots;
     const uint32_t bar_xempty = bar_xfull + 8 * kXE;
@@ -457,6 +496,10 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
     __syncthreads();
     const Plan pl = *plan;
     volatile int *abort_flag = &plan->abort_flag;
+    const int npc = pl.d_hi - pl.d_lo + 1 < kPC ? pl.d_hi - pl.d_lo + 1 : kPC;
+    for (int i = threadIdx.x; i < npc; i += kThr)
+        pcache[i] = load_proj(p, pl.d_lo + i);
+    __syncthreads();
 
     if (warp == NC) {
         // ------------------------------------------------ activation warp
@@ -470,7 +513,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
             bool ok = true;
             for (int d = pl.d_lo; d <= pl.d_hi && ok; ++d) {
                 const int seg = d - pl.d_lo, e = seg % kXE;
-                const DescRecord &r = rec(p, d);
+                const ProjC r = get_proj(p, pcache, pl.d_lo, npc, d);
                 const int64_t rs = r.K + 64;
                 const int64_t size = (p.mg * rs + 127) / 128 * 128;
                 int64_t pos = head;
@@ -519,7 +562,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
     const uint32_t zero_s = smem_u32(zero_row);
 
     ChunkIter<NC> cons, prod;
-    cons.init(p, pl, warp);
+    cons.init(p, pl, warp, pcache, npc);
     prod = cons;
     int issued = 0, consumed = 0;
     for (int s = 0; s < S && prod.valid; ++s) {
@@ -539,8 +582,8 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
             break;
         }
         // this projection's fields, read once
-        const DescRecord &r = rec(p, d);
-        const float wscale = __ldg(r.wscale);
+        const ProjC r = get_proj(p, pcache, pl.d_lo, npc, d);
+        const float wscale = r.wscale;
         const int64_t N = r.N, rbeg = r.rb_begin;
         float *const y = r.y;
         int32_t *const acc_out = r.acc_out;
