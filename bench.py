@@ -142,6 +142,27 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def rank_layer_seed(layer, rank):
+    """Layer index the activations of `rank` are seeded with: every rank of a
+    data-parallel run decodes its own token stream over the same weights."""
+    return layer + 1000 * rank
+
+
+def max_over_ranks(ms, dist, device):
+    """The slowest rank's time (all ranks take the same collective step)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(M, world, steps, max_ms):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return M * world * steps / (max_ms / 1e3)
+
+
 def build_workload(api, torch, dev, M, layers, rank):
     """Generate, upload and ternarise the sweep; return descriptors and buffers."""
     from ternary_weight_decoder_b200 import synth
@@ -171,7 +192,7 @@ def build_workload(api, torch, dev, M, layers, rank):
         packed, mean_abs, wscale = api.ternarize_pack(Wd)
         del Wd, W
         # each rank decodes its own token stream
-        xn[x_off[i]:x_off[i] + M * K] = synth.activations(l + 1000 * rank, p, M, K).ravel()
+        xn[x_off[i]:x_off[i] + M * K] = synth.activations(rank_layer_seed(l, rank), p, M, K).ravel()
         descs.append(dict(x=x_all[x_off[i]:x_off[i] + M * K].view(M, K), packed=packed,
                           wscale=wscale, y=y_all[y_off[i]:y_off[i] + M * N].view(M, N),
                           N=N, K=K))
@@ -313,14 +334,9 @@ def main():
         e1.record(stream)
         barrier()
     api.check()
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     ms_per_step = ms / args.steps
-    tokens = M * world * args.steps
-    value = tokens / (ms / 1e3)
+    value = job_value(M, world, args.steps, ms)
 
     hbm, src = peaks()
     if M <= 32:
@@ -370,12 +386,8 @@ def main():
         f1.record(stream)
         barrier()
         wall = time.perf_counter() - t0
-        ems = f0.elapsed_time(f1)
-        if dist is not None:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": M * world * k2 / (ems / 1e3), "unit": UNIT,
+        ems = max_over_ranks(f0.elapsed_time(f1), dist, dev)
+        e2e = {"value": job_value(M, world, k2, ems), "unit": UNIT,
                "h2d_bytes_per_step": x_all.numel() * 4, "d2h_bytes_per_step": y_all.numel() * 4,
                "steps": k2, "ms_per_step": ems / k2, "host_wall_ms_per_step": wall * 1e3 / k2}
 
