@@ -401,6 +401,16 @@ size_t tw_sweep_workspace_bytes(const void *table_host)
     return (size_t)hdr->ws_bytes;
 }
 
+// Projections of a host table with K > kQuantSmallK (they lead the unit order).
+static int big_k_projections(const tw::TableHeader *hdr)
+{
+    const auto *recs = reinterpret_cast<const tw::DescRecord *>(hdr + 1);
+    int n = 0;
+    for (int d = 0; d < hdr->count; ++d)
+        n += recs[d].K > tw::kQuantSmallK;
+    return n;
+}
+
 int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, void *ws,
                                 size_t ws_bytes, tw_stream_t stream)
 {
@@ -433,9 +443,13 @@ int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, v
         return fail(TW_ERR_ALIGN, "sweep workspace must be 16-byte aligned");
     const auto *recs_dev = reinterpret_cast<const tw::DescRecord *>(
         static_cast<const tw::TableHeader *>(table_dev) + 1);
+    const auto *order_dev = reinterpret_cast<const tw::UnitOrder *>(recs_dev + hdr->count);
+    const int n_big = big_k_projections(hdr);
     if (!tw::decode_sweep_on_tensor_cores(hdr->M)) {
         tw::DecodeLaunch L{};
         L.table = recs_dev;
+        L.order = order_dev;
+        L.n_big = n_big;
         L.single = nullptr;
         L.count = hdr->count;
         L.M = hdr->M;
@@ -451,7 +465,8 @@ int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, v
         return fail(TW_ERR_CUDA, "table was encoded without the CUDA driver's TMA encoder");
     tw::DecodeTcLaunch T{};
     T.table = recs_dev;
-    T.order = reinterpret_cast<const tw::UnitOrder *>(recs_dev + hdr->count);
+    T.order = order_dev;
+    T.n_big = n_big;
     T.count = hdr->count;
     T.M = hdr->M;
     T.total_units = hdr->total_units;
@@ -469,9 +484,10 @@ int tw_sweep_launches(const void *table_host)
         return 0;
     if (hdr->M > tw::kDecodeMaxM)
         return 1;
+    const int n_big = big_k_projections(hdr);
     if (!tw::decode_sweep_on_tensor_cores(hdr->M))
-        return tw::decode_launches(hdr->M, hdr->max_K);
-    return 2;  // quantise + the tensor-core sweep
+        return tw::decode_launches(hdr->count, hdr->M, hdr->max_K, n_big);
+    return tw::quant_launches(hdr->count, hdr->M, n_big) + 1;  // quantise + the tensor-core sweep
 }
 
 int tw_check(tw_stream_t stream)

@@ -16,15 +16,18 @@
 //
 // Launch 2 (k_decode), one CTA per SM:
 //   * The grid splits the concatenated 16-row blocks of all projections into
-//     equal shares of packed bytes; each CTA streams its share once.
-//   * NC consumer warps (15 for up to 8 tokens, 11 or 7 for more) each own
-//     every NC-th row block of the share and keep a private ring of 4 KB
-//     slots that they fill with 1-D bulk copies (the TMA engine) ahead of
-//     the arithmetic; a slot is refilled as soon as its tiles are in
-//     registers, so the codes stream from HBM independently of the math.
+//     shares of equal estimated cost (16 per 128-column tile + a fixed part
+//     per row block); each CTA streams its share once.
+//   * NC consumer warps (19 for up to 8 tokens, fewer for more, as shared
+//     memory allows) each own every NC-th row block of the share and keep a
+//     private ring of 4 KB slots that they fill with 1-D bulk copies (the TMA
+//     engine) ahead of the arithmetic; each tile's lane slot is read from
+//     shared memory just before its MMAs (few registers, so more warps fit)
+//     and the slot is refilled once the chunk is done.
 //   * The last warp (activation warp) waits for launch 1, then bulk-copies each
-//     projection's int8 rows, amax/127 and sum(q) into one of up to four
-//     shared-memory buffers ahead of the consumers.
+//     projection's int8 rows, amax/127 and sum(q) into a byte ring in shared
+//     memory (entries sized per projection, up to 8 in flight) ahead of the
+//     consumers.
 //   * Codes are decoded in registers with one AND per register:
 //     word & (0x03030303 << 2s) holds four codes + 1 of consecutive k,
 //     scaled by 4^s, as unsigned bytes; they feed m16n8k32 u8 x s8 MMAs
@@ -70,9 +73,12 @@ struct DecodeParams {
 struct QuantParams {
     const DescRecord *table;
     DescRecord single;
-    int count, M;
+    int count, M;             // projections of this launch, tokens
     int ntok;                 // 0: plain int8 rows; 8/16/32: tensor-core token blocks
     int wpr;                  // warps per row (set by launch_quant_rows)
+    const UnitOrder *order;   // null: projection i is record i; else order[i0 + i].d
+    int i0;
+    int wait_prev;            // wait for the preceding launch before finishing
     uint8_t *ws;
     int64_t ws_sa_off;
 };
@@ -144,7 +150,8 @@ __global__ void __launch_bounds__(kQThreads) k_quant_rows(const __grid_constant_
     const int wpr = p.wpr, rloc = warp / wpr, wr = warp % wpr;
     const int64_t row_id = (int64_t)blockIdx.x * (kQThreads / 32 / wpr) + rloc;
     const bool live = row_id < (int64_t)p.count * p.M;
-    const int d = live ? (int)(row_id / p.M) : 0, m = live ? (int)(row_id % p.M) : 0;
+    const int pi = live ? (int)(row_id / p.M) : 0, m = live ? (int)(row_id % p.M) : 0;
+    const int d = p.order ? p.order[p.i0 + pi].d : pi;
     const DescRecord &r = rec(p, d);
     const int64_t K4 = live ? r.K / 4 : 0;
     const float4 *row = reinterpret_cast<const float4 *>(r.x + (int64_t)m * r.K);
@@ -240,6 +247,11 @@ __global__ void __launch_bounds__(kQThreads) k_quant_rows(const __grid_constant_
         reinterpret_cast<float *>(info)[m] = __fdiv_rn(a, 127.f);
         reinterpret_cast<int *>(info + 128)[m] = sum;
     }
+    // This launch overlaps the preceding one (programmatic dependent launch);
+    // it completes only after that one has, so that waiting for this launch
+    // covers both.
+    if (p.wait_prev)
+        pdl_wait();
 }
 
 // Warps per row for `rows` rows: enough warps in flight to fill the GPU
@@ -253,16 +265,66 @@ int quant_warps_per_row(int64_t rows, int sms)
     return w;
 }
 
-cudaError_t launch_quant_rows(QuantParams &q, cudaStream_t stream)
+int sm_count()
 {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+cudaError_t launch_quant_once(const QuantParams &q, bool pdl, cudaStream_t stream)
+{
     const int64_t rows = (int64_t)q.count * q.M;
-    q.wpr = quant_warps_per_row(rows, sms);
     const int64_t per_block = kQThreads / 32 / q.wpr;
-    k_quant_rows<<<(unsigned)((rows + per_block - 1) / per_block), kQThreads, 0, stream>>>(q);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((rows + per_block - 1) / per_block));
+    cfg.blockDim = dim3(kQThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_quant_rows, q);
+}
+
+// Launches of the quantisation pass: one, or -- when there are so many rows
+// that a row would get at most 2 warps, and the large-K rows then need two
+// passes over x -- two: the projections of the order with K > kQuantSmallK
+// (entries [0, n_big)) at 8 warps per row, so that each row is read once
+// into registers, and the rest with as many warps per row as fill the GPU.
+// (Measured on B200: the second launch pays off from 8 tokens of the
+// 196-projection sweep on, not at 4.)
+int quant_launches_impl(int64_t count, int64_t M, int n_big)
+{
+    const int w = quant_warps_per_row(count * M, sm_count());
+    return (w <= 2 && n_big > 0 && n_big < count) ? 2 : 1;
+}
+
+cudaError_t launch_quant_rows(QuantParams &q, int n_big, cudaStream_t stream)
+{
+    const int sms = sm_count();
+    if (!q.order || quant_launches_impl(q.count, q.M, n_big) == 1) {
+        q.wpr = quant_warps_per_row((int64_t)q.count * q.M, sms);
+        q.order = nullptr;   // one launch: the projections in record order
+        q.i0 = 0;
+        q.wait_prev = 0;
+        return launch_quant_once(q, false, stream);
+    }
+    QuantParams a = q, b = q;
+    a.i0 = 0;
+    a.count = n_big;
+    a.wpr = 8;
+    a.wait_prev = 0;
+    b.i0 = n_big;
+    b.count = q.count - n_big;
+    b.wpr = quant_warps_per_row((int64_t)b.count * q.M, sms);
+    b.wait_prev = 1;
+    cudaError_t e = launch_quant_once(a, false, stream);
+    if (e == cudaSuccess)
+        e = launch_quant_once(b, true, stream);
+    return e;
 }
 
 // ----------------------------------------------------------------- launch 2
@@ -614,13 +676,12 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
                     break;
                 }
                 const int n = min(kCT, KT - kc * kCT);
-                // All 8 lane slots of the chunk go to registers (slots past n
-                // hold stale bytes and are not used) ...
-                uint4 a[kCT];
+                const uint32_t kbase = (uint32_t)(kc * kCT * kTileK);
 #pragma unroll
                 for (int i = 0; i < kCT; ++i)
-                    a[i] = lds128(ring_w + cslot * kChunk + i * kTileBytes);
-                // ... so the slot is refilled before the arithmetic starts.
+                    if (i < n)
+                        tile_mma<NT>(acc, lds128(ring_w + cslot * kChunk + i * kTileBytes), xrow,
+                                     kbase + i * kTileK);
                 __syncwarp();
                 if (prod.valid) {
                     if (lane == 0) {
@@ -635,11 +696,6 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
                     cslot = 0;
                     cphase ^= 1u;
                 }
-                const uint32_t kbase = (uint32_t)(kc * kCT * kTileK);
-#pragma unroll
-                for (int i = 0; i < kCT; ++i)
-                    if (i < n)
-                        tile_mma<NT>(acc, a[i], xrow, kbase + i * kTileK);
                 cons.next(p);
             }
             if (!ok)
@@ -694,11 +750,13 @@ __global__ void k_wait_probe(WaitCtl ctl)
 // registers for the wider accumulators of larger token groups.
 // The block is a multiple of 4 warps so that each SM sub-partition's
 // register file holds the same number of warps (16, 12 or 8 in total).
-// Consumer warps per block: more warps hide more latency, fewer leave
-// registers for the wider accumulators of larger token groups and shared
-// memory for their activation rows.  The block is a multiple of 4 warps so
-// that each SM sub-partition's register file holds the same number of warps.
-int max_consumers(int nt) { return nt == 1 ? 15 : nt == 2 ? 11 : 7; }
+// Consumer warps per block: more warps hide more latency (measured on B200:
+// 19 beat 15 by 6 % at one token; 23 spill at the 80 registers they leave),
+// fewer leave registers for the wider accumulators of larger token groups
+// and shared memory for their activation rows.  The block is a multiple of 4
+// warps so that each SM sub-partition's register file holds the same number
+// of warps.
+int max_consumers(int nt) { return nt == 1 ? 19 : nt == 2 ? 11 : 7; }
 
 template <int NT, int NC>
 cudaError_t launch_nt(const DecodeParams &p, int grid, int smem, cudaStream_t stream)
@@ -763,6 +821,7 @@ cudaError_t launch_plan(const DecodeParams &p, const DecodePlan &g, int grid, in
                         cudaStream_t stream)
 {
     const int nt = (p.mg + 7) / 8;
+    if (nt == 1 && g.nc == 19) return launch_nt<1, 19>(p, grid, smem, stream);
     if (nt == 1 && g.nc == 15) return launch_nt<1, 15>(p, grid, smem, stream);
     if (nt == 1 && g.nc == 11) return launch_nt<1, 11>(p, grid, smem, stream);
     if (nt == 1) return launch_nt<1, 7>(p, grid, smem, stream);
@@ -774,8 +833,13 @@ cudaError_t launch_plan(const DecodeParams &p, const DecodePlan &g, int grid, in
 
 }  // namespace
 
-cudaError_t launch_quant_tc(const DescRecord *table, int count, int64_t M, int ntok, uint8_t *ws,
-                            int64_t ws_sa_off, cudaStream_t stream)
+int quant_launches(int64_t count, int64_t M, int n_big)
+{
+    return quant_launches_impl(count, M, n_big);
+}
+
+cudaError_t launch_quant_tc(const DescRecord *table, const UnitOrder *order, int n_big, int count,
+                            int64_t M, int ntok, uint8_t *ws, int64_t ws_sa_off, cudaStream_t stream)
 {
     QuantParams q;
     memset(&q, 0, sizeof(q));
@@ -783,17 +847,19 @@ cudaError_t launch_quant_tc(const DescRecord *table, int count, int64_t M, int n
     q.count = count;
     q.M = (int)M;
     q.ntok = ntok;
+    q.order = order;
     q.ws = ws;
     q.ws_sa_off = ws_sa_off;
-    return launch_quant_rows(q, stream);
+    return launch_quant_rows(q, n_big, stream);
 }
 
-int decode_launches(int64_t M, int64_t max_K)
+int decode_launches(int64_t count, int64_t M, int64_t max_K, int n_big)
 {
     DecodePlan g{};
     if (!plan_decode((int)M, max_K, &g))
         return 0;
-    return 1 + (int)((M + g.mg - 1) / g.mg);  // quantise + one decode launch per group
+    // quantise (one or two launches) + one decode launch per token group
+    return quant_launches(count, M, n_big) + (int)((M + g.mg - 1) / g.mg);
 }
 
 cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout_ns,
@@ -820,7 +886,8 @@ cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout
     q.M = M;
     q.ws = L.ws;
     q.ws_sa_off = L.ws_sa_off;
-    e = launch_quant_rows(q, stream);
+    q.order = L.order;
+    e = launch_quant_rows(q, L.n_big, stream);
     if (e != cudaSuccess)
         return e;
 

@@ -475,7 +475,8 @@ cudaError_t launch_decode_tc(const DecodeTcLaunch &L, uint32_t *err, uint64_t ti
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess)
         return e;
-    e = launch_quant_tc(L.table, L.count, L.M, tc_tokens(L.M), L.ws, L.ws_sa_off, stream);
+    e = launch_quant_tc(L.table, L.order, L.n_big, L.count, L.M, tc_tokens(L.M), L.ws, L.ws_sa_off,
+                        stream);
     if (e != cudaSuccess)
         return e;
     TcParams p;

@@ -71,6 +71,8 @@ cudaError_t launch_quantize(const float *x, int64_t M, int64_t K, int8_t *xq, fl
 constexpr int64_t kRbFixedCost = 45;
 __host__ __device__ inline int64_t rb_cost(int64_t K) { return 16 * (K / kTileK) + kRbFixedCost; }
 
+struct UnitOrder;
+
 struct DecodeLaunch {
     const DescRecord *table;  // device records (or null: use `single`)
     int count;
@@ -79,9 +81,13 @@ struct DecodeLaunch {
     const DescRecord *single; // host copy of a one-record sweep (table == null)
     uint8_t *ws;              // scratch: int8 rows at each record's ws_xq_off,
     int64_t ws_sa_off;        // then 256 bytes of amax/127, sum(q) per record
+    const UnitOrder *order;   // projections by K descending (sweeps; null: single)
+    int n_big;                // leading entries of `order` with K > kQuantSmallK
 };
 // Kernel launches one decode call makes for M tokens (quantise + groups).
-int decode_launches(int64_t M, int64_t max_K);
+int decode_launches(int64_t count, int64_t M, int64_t max_K, int n_big);
+// Launches of the quantisation pass for `count` projections of M tokens.
+int quant_launches(int64_t count, int64_t M, int n_big);
 
 // Decode scratch of the single-matrix path: the M int8 rows (128-byte
 // aligned), then 256 bytes: 32 floats amax/127 and 32 ints sum(q).
@@ -91,6 +97,9 @@ int decode_launches(int64_t M, int64_t max_K);
 // its token blocks -- K/128 blocks of tc_tokens(M) rows x 128 bytes, 128-byte
 // swizzled -- then per projection 256 bytes of amax/127 and sum(q).
 constexpr int64_t kWsCtrBytes = 256;
+// Rows of projections with K above this are quantised by 8 warps each (they
+// do not fit one warp's registers); the others by as few as fill the GPU.
+constexpr int64_t kQuantSmallK = 1536;
 inline int tc_tokens(int64_t M) { return M <= 8 ? 8 : M <= 16 ? 16 : 32; }
 // Which decode kernel runs a sweep of M tokens (measured on B200: the
 // tensor-core sweep wins once the int8 MMAs of the register path, 4 per
@@ -107,6 +116,7 @@ static_assert(sizeof(UnitOrder) == 16, "unit order entry");
 struct DecodeTcLaunch {
     const DescRecord *table;  // device records
     const UnitOrder *order;   // device copy of the order (follows the records)
+    int n_big;                // leading entries of `order` with K > kQuantSmallK
     int count;
     int64_t M, total_units;
     uint8_t *ws;
@@ -116,8 +126,8 @@ struct DecodeTcLaunch {
 cudaError_t launch_decode_tc(const DecodeTcLaunch &L, uint32_t *err, uint64_t timeout_ns,
                              cudaStream_t stream);
 // Quantise every (projection, token) row into the token blocks above.
-cudaError_t launch_quant_tc(const DescRecord *table, int count, int64_t M, int ntok, uint8_t *ws,
-                            int64_t ws_sa_off, cudaStream_t stream);
+cudaError_t launch_quant_tc(const DescRecord *table, const UnitOrder *order, int n_big, int count,
+                            int64_t M, int ntok, uint8_t *ws, int64_t ws_sa_off, cudaStream_t stream);
 inline int64_t round128(int64_t b) { return (b + 127) / 128 * 128; }
 cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout_ns,
                           cudaStream_t stream);

@@ -268,6 +268,38 @@ def test_sweep_ragged_small_projections(dev, api):
         G.assert_y_close(d["y"].cpu().numpy(), ref["y"])
 
 
+@pytest.mark.parametrize("M", [17, 20, 24, 31])
+def test_sweep_tensor_core_decode_ragged(dev, api, M):
+    """The tensor-core decode kernel (17..32 tokens): every token-block width,
+    projections whose N is not a multiple of 128 (the last 128-row unit
+    partial, row blocks past N read as zero), several K, and the unit order
+    (larger K first) different from the record order."""
+    import torch
+    shapes = [(200, 256), (128, 1536), (17, 384), (385, 640), (256, 2048), (1, 128)]
+    descs, keep = [], []
+    for i, (N, K) in enumerate(shapes):
+        W = _weights(N, K, 3000 + 10 * M + i)
+        x = _acts(M, K, 4000 + 10 * M + i)
+        packed, _, wscale = G.ternarize_gpu(W, dev)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+        acc = torch.full((M, N), int(POISON_I32), dtype=torch.int32, device=dev)
+        descs.append(dict(x=G.to_dev(x, dev), packed=packed, wscale=wscale, y=y, acc_out=acc,
+                          N=N, K=K))
+        keep.append((W, x))
+    table = api.SweepTable(descs, M, device=dev)
+    for _ in range(2):   # twice: the work counters are left zero for the next call
+        api.decoder_projection_sweep(table)
+        api.check()
+        for d, (W, x) in zip(descs, keep):
+            codes, mean = orc.ternarize(W)
+            ref = orc.ternary_linear(x, codes, mean)
+            assert (d["acc_out"].cpu().numpy() == ref["acc"]).all(), (M, d["N"], d["K"])
+            G.assert_y_close(d["y"].cpu().numpy(), ref["y"])
+        for d in descs:
+            d["y"].fill_(float("nan"))
+            d["acc_out"].fill_(int(POISON_I32))
+
+
 # ------------------------------------------------------------ errors
 def test_wait_timeout_is_reported(dev, api):
     api.debug_wait_timeout(2_000_000)   # 2 ms; nothing ever arrives
