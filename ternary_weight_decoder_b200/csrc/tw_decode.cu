@@ -20,7 +20,7 @@
 //     per row block); each CTA streams its share once.
 //   * NC consumer warps (19 for up to 8 tokens, fewer for more, as shared
 //     memory allows) each own every NC-th row block of the share and keep a
-//     private ring of 4 KB slots that they fill with 1-D bulk copies (the TMA
+//     private ring of 3.5 KB slots that they fill with 1-D bulk copies (the TMA
 //     engine) ahead of the arithmetic; each tile's lane slot is read from
 //     shared memory just before its MMAs (few registers, so more warps fit)
 //     and the slot is refilled once the chunk is done.
@@ -44,8 +44,10 @@
 namespace tw {
 namespace {
 
-constexpr int kCT = 8;                      // tiles per ring chunk
-constexpr int kChunk = kCT * kTileBytes;    // 4 KB
+constexpr int kCT = 7;                      // tiles per ring chunk (3.5 KB; measured on
+                                            // B200 against 5..10: a K = 8960 row block
+                                            // is exactly 10 chunks)
+constexpr int kChunk = kCT * kTileBytes;    // 3.5 KB, a multiple of 128
 constexpr int kXE = 8;                      // activation ring entries
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kPC = 32;                     // projections cached in shared memory per block
