@@ -117,7 +117,7 @@ def _run_linear(api, dev, W, x, N):
 @pytest.mark.parametrize("M", list(range(1, 34)))
 def test_linear_m_tails(dev, api, M):
     """M = 1..32 run the decode kernel, M = 33 the tensor-core prefill."""
-    N, K = 80, 640   # 5 row blocks, 5 k tiles (a partial 8-tile chunk)
+    N, K = 80, 640   # 5 row blocks, 5 k tiles (one partial ring chunk)
     W = _weights(N, K, 100 + M)
     x = _acts(M, K, 200 + M)
     y, acc = _run_linear(api, dev, W, x, N)
@@ -266,6 +266,33 @@ def test_sweep_ragged_small_projections(dev, api):
         ref = orc.ternary_linear(x, codes, mean)
         assert (d["acc_out"].cpu().numpy() == ref["acc"]).all()
         G.assert_y_close(d["y"].cpu().numpy(), ref["y"])
+
+
+@pytest.mark.parametrize("M", [1, 3, 5, 8, 13, 16])
+def test_sweep_chunk_tails(dev, api, M):
+    """K = 128 .. 1792 (1 to 14 k tiles) in one sweep: every length of the
+    last ring chunk of a row block (1..6 tiles for 7-tile chunks up to 4
+    tokens, 1..5 for 6-tile chunks above) and whole chunks, with ragged N."""
+    import torch
+    shapes = [(16 * kt + 8 * (kt % 3) + kt % 5, 128 * kt) for kt in range(1, 15)]
+    descs, keep = [], []
+    for i, (N, K) in enumerate(shapes):
+        W = _weights(N, K, 3000 + 50 * M + i)
+        x = _acts(M, K, 4000 + 50 * M + i)
+        packed, _, wscale = G.ternarize_gpu(W, dev)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+        acc = torch.full((M, N), int(POISON_I32), dtype=torch.int32, device=dev)
+        descs.append(dict(x=G.to_dev(x, dev), packed=packed, wscale=wscale, y=y, acc_out=acc,
+                          N=N, K=K))
+        keep.append((W, x))
+    table = api.SweepTable(descs, M, device=dev)
+    api.decoder_projection_sweep(table)
+    api.check()
+    for (N, K), d, (W, x) in zip(shapes, descs, keep):
+        codes, mean = orc.ternarize(W)
+        ref = orc.ternary_linear(x, codes, mean)
+        assert (d["acc_out"].cpu().numpy() == ref["acc"]).all(), f"M={M} N={N} K={K}"
+        G.assert_y_close(d["y"].cpu().numpy(), ref["y"], f"M={M} N={N} K={K}")
 
 
 @pytest.mark.parametrize("M", [17, 20, 24, 31])
