@@ -47,11 +47,12 @@ namespace {
 
 // Tiles per ring chunk of the register kernel.  Measured on B200 with the
 // full-chunk fast path: 7 tiles (3.5 KB; a K = 8960 row block is exactly 10
-// chunks) for groups of up to 4 tokens; 6 tiles (3 KB) for larger groups,
-// whose activation rows need the shared memory (at 16 tokens 11 consumer
-// warps fit instead of 7).  A partial chunk runs as 4 + 2 + 1 tiles, so a
-// chunk holds at most 8.
-constexpr int chunk_tiles(int mg) { return mg <= 4 ? 7 : 6; }
+// chunks) for groups of up to 4 tokens; 6 tiles (3 KB) for 5 to 8 and 17 to
+// 32 tokens, whose activation rows need the shared memory; 4 tiles (2 KB)
+// for 9 to 16, so that 15 consumer warps fit beside 16 rows of K = 8960 (11
+// with 3 KB chunks, 7 with 3.5 KB).  A partial chunk runs as 4 + 2 + 1
+// tiles, so a chunk holds at most 8.
+constexpr int chunk_tiles(int mg) { return mg <= 4 ? 7 : mg > 8 && mg <= 16 ? 4 : 6; }
 constexpr int kXE = 8;                      // activation ring entries
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kPC = 32;                     // projections cached in shared memory per block
@@ -784,12 +785,13 @@ __global__ void k_wait_probe(WaitCtl ctl)
 }
 
 // Consumer warps per block: more warps hide more latency (measured on B200:
-// 19 beat 15 by 6 % at one token; 23 spill at the 80 registers they leave),
-// fewer leave registers for the wider accumulators of larger token groups
-// and shared memory for their activation rows.  The block is a multiple of 4
+// 19 beat 15 by 6 % at one token; 23 spill at the 80 registers they leave;
+// for two token tiles 15 beat 11 by 2-5 % at 9 to 16 tokens, in 128
+// registers), fewer leave registers for the wider accumulators of larger
+// token groups and shared memory for their activation rows.  The block is a multiple of 4
 // warps so that each SM sub-partition's register file holds the same number
 // of warps.
-int max_consumers(int nt) { return nt == 1 ? 19 : nt == 2 ? 11 : 7; }
+int max_consumers(int nt) { return nt == 1 ? 19 : nt == 2 ? 15 : 7; }
 
 template <int NT, int NC, int CT>
 cudaError_t launch_nt(const DecodeParams &p, int grid, int smem, cudaStream_t stream)
@@ -853,6 +855,7 @@ bool plan_decode(int M, int64_t max_K, DecodePlan *out)
 cudaError_t launch_plan(const DecodeParams &p, const DecodePlan &g, int grid, int smem,
                         cudaStream_t stream)
 {
+    // (token tiles, chunk tiles) as chunk_tiles() and max_consumers() give them
     const int nt = (p.mg + 7) / 8;
     if (nt == 1 && g.ct == 7) {
         if (g.nc == 19) return launch_nt<1, 19, 7>(p, grid, smem, stream);
@@ -860,16 +863,20 @@ cudaError_t launch_plan(const DecodeParams &p, const DecodePlan &g, int grid, in
         if (g.nc == 11) return launch_nt<1, 11, 7>(p, grid, smem, stream);
         return launch_nt<1, 7, 7>(p, grid, smem, stream);
     }
-    if (g.ct != 6)
-        return cudaErrorInvalidValue;
-    if (nt == 1 && g.nc == 19) return launch_nt<1, 19, 6>(p, grid, smem, stream);
-    if (nt == 1 && g.nc == 15) return launch_nt<1, 15, 6>(p, grid, smem, stream);
-    if (nt == 1 && g.nc == 11) return launch_nt<1, 11, 6>(p, grid, smem, stream);
-    if (nt == 1) return launch_nt<1, 7, 6>(p, grid, smem, stream);
-    if (nt == 2 && g.nc == 11) return launch_nt<2, 11, 6>(p, grid, smem, stream);
-    if (nt == 2) return launch_nt<2, 7, 6>(p, grid, smem, stream);
-    if (nt == 3) return launch_nt<3, 7, 6>(p, grid, smem, stream);
-    return launch_nt<4, 7, 6>(p, grid, smem, stream);
+    if (nt == 1 && g.ct == 6) {
+        if (g.nc == 19) return launch_nt<1, 19, 6>(p, grid, smem, stream);
+        if (g.nc == 15) return launch_nt<1, 15, 6>(p, grid, smem, stream);
+        if (g.nc == 11) return launch_nt<1, 11, 6>(p, grid, smem, stream);
+        return launch_nt<1, 7, 6>(p, grid, smem, stream);
+    }
+    if (nt == 2 && g.ct == 4) {
+        if (g.nc == 15) return launch_nt<2, 15, 4>(p, grid, smem, stream);
+        if (g.nc == 11) return launch_nt<2, 11, 4>(p, grid, smem, stream);
+        return launch_nt<2, 7, 4>(p, grid, smem, stream);
+    }
+    if (nt == 3 && g.ct == 6) return launch_nt<3, 7, 6>(p, grid, smem, stream);
+    if (nt == 4 && g.ct == 6) return launch_nt<4, 7, 6>(p, grid, smem, stream);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
