@@ -57,25 +57,47 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def _sha256(path):
+def _strip_comments(text):
+    """C/C++/CUDA source without comments, trailing blanks or empty lines."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(l.rstrip() for l in text.splitlines() if l.strip())
+
+
+def code_digest(kernel_src, read=None):
+    """sha256 over the code of one kernel source file and of the library's
+    headers (comments and blank lines removed): an ncu capture stays valid
+    across comment edits and stops applying on any change of code.
+    `read(relpath)` returns a file's text (default: the working tree)."""
+    import glob
     import hashlib
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+    if read is None:
+        def read(rel):
+            with open(os.path.join(ROOT, rel)) as f:
+                return f.read()
+    csrc = os.path.join("ternary_weight_decoder_b200", "csrc")
+    rels = [os.path.join(csrc, kernel_src)]
+    for pat in (os.path.join(csrc, "*.cuh"), os.path.join(csrc, "*.h"), os.path.join("include", "*.h")):
+        rels += sorted(os.path.relpath(q, ROOT) for q in glob.glob(os.path.join(ROOT, pat)))
+    h = hashlib.sha256()
+    for rel in rels:
+        h.update(rel.encode() + b"\0" + _strip_comments(read(rel)).encode() + b"\0")
+    return h.hexdigest()
 
 
 def profiled_traffic(kernel_src, M, layers):
     """DRAM bytes (read + write) per launch of the dominant kernel, from the
     ncu capture recorded in profiles/traffic.json, or None when there is no
-    capture for this M or the kernel's source has changed since it was taken.
+    capture for this M or the kernel's code has changed since it was taken.
     A capture of fewer layers is scaled by the layer count (the traffic of a
     sweep grows in proportion to its projections at fixed M)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    src = os.path.join(ROOT, "ternary_weight_decoder_b200", "csrc", kernel_src)
-    digest = _sha256(src)
+    digest = code_digest(kernel_src)
     for e in json.load(open(p)).get("captures", []):
-        if e["kernel_src"] == kernel_src and e["M"] == M and e["source_sha256"] == digest:
+        if e["kernel_src"] == kernel_src and e["M"] == M and e["code_sha256"] == digest:
             return e["dram_bytes_per_launch"] * layers / e["layers"]
     return None
 

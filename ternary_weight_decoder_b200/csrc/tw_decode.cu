@@ -9,22 +9,24 @@
 // bounds decode: "The Paper Says ARM Support" post, "What the model is
 // trying to do".)
 //
-// Launch 1 (k_quant_rows): one block per (projection, token) quantises the
-// row, held in registers (one HBM round trip), into int8 scratch together
-// with amax/127 and sum(q).  It lets launch 2 start at once (programmatic
-// dependent launch), so the weight stream below overlaps it.
+// Launch 1 (k_quant_rows): 8, 4, 2 or 1 warps per (projection, token) row,
+// by the number of rows, quantise the row, held in registers (one HBM round
+// trip), into int8 scratch together with amax/127 and sum(q); with many rows
+// the large-K rows get a launch of their own at 8 warps per row.  It lets
+// launch 2 start at once (programmatic dependent launch), so the weight
+// stream below overlaps it.
 //
 // Launch 2 (k_decode), one CTA per SM:
 //   * The grid splits the concatenated 16-row blocks of all projections into
 //     shares of equal estimated cost (16 per 128-column tile + a fixed part
 //     per row block); each CTA streams its share once.
-//   * NC consumer warps (19 for up to 8 tokens, fewer for more, as shared
-//     memory allows) each own every NC-th row block of the share and keep a
-//     private ring of 3.5 KB slots (3 KB above 4 tokens) that they fill with
-//     1-D bulk copies (the TMA engine) ahead of the arithmetic; each tile's
-//     lane slot is read from shared memory just before its MMAs (few
-//     registers, so more warps fit) and the slot is refilled once the chunk
-//     is done.
+//   * NC consumer warps (19 for up to 8 tokens, 15 for 9 to 16, 7 above, or
+//     fewer as shared memory allows) each own every NC-th row block of the
+//     share and keep a private ring of 2 to 3.5 KB slots (by the token
+//     count) that they fill with 1-D bulk copies (the TMA engine) ahead of
+//     the arithmetic; each tile's lane slot is read from shared memory just
+//     before its MMAs (few registers, so more warps fit) and the slot is
+//     refilled once the chunk is done.
 //   * The last warp (activation warp) waits for launch 1, then bulk-copies each
 //     projection's int8 rows, amax/127 and sum(q) into a byte ring in shared
 //     memory (entries sized per projection, up to 8 in flight) ahead of the
