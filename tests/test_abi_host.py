@@ -148,3 +148,28 @@ def test_layout_spec_round_trip():
         w = p.view(np.uint32).astype(np.int64)
         dec = [int((w[0] >> (8 * b + 2 * s)) & 3) - 1 for s in range(4) for b in range(4)]
         assert dec == c[0, :16].tolist()
+
+
+QWEN_LAYER = [(1536, 1536), (256, 1536), (256, 1536), (1536, 1536),
+              (8960, 1536), (8960, 1536), (1536, 8960)]
+
+
+@pytest.mark.parametrize("M", list(range(1, 33)))
+def test_sweep_launch_count_196(lib, M):
+    """Launches per step of the 196-projection sweep, as the host plans them
+    for 148 SMs: one or two quantisation launches (two once a row gets at
+    most 2 warps: the 28 K = 8960 rows split off), then one decode launch.
+    Up to 16 tokens that is one register-kernel launch (every token group
+    fits: 15 consumer warps with 2 KB chunks beside 16 rows of K = 8960),
+    above that the tensor-core kernel."""
+    from ternary_weight_decoder_b200 import api
+    shapes = QWEN_LAYER * 28
+    arr = _descs(shapes)
+    n = api.tw_sweep_table_bytes(len(shapes))
+    buf = np.zeros(n, np.uint8)
+    assert api.tw_sweep_table_encode(arr, len(shapes), M, buf.ctypes.data, n) == 0, \
+        api.tw_last_error()
+    # warps per row: the largest of 8, 4, 2, 1 with 196*M*w <= 148*24, i.e.
+    # 8 for M <= 2, 4 for M = 3..4, 2 or 1 from M = 5 on
+    quant = 1 if M <= 4 else 2
+    assert api.tw_sweep_launches(buf.ctypes.data) == quant + 1
