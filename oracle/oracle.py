@@ -3,7 +3,9 @@
 TEST INFRASTRUCTURE ONLY.  Imported by ``tests/``, by ``__graft_entry__.smoke``
 and by the CPU-baseline leg of ``bench.py``; never by the product package.
 This module only marshals numpy arrays into the C functions; every step of
-the arithmetic lives in ``ternary_oracle.c``.
+the arithmetic lives in ``ternary_oracle.c``.  ``decoder_layer`` composes
+them in the order of a decoder layer, rounding each projection output to
+float32 as the chain passes it on.
 """
 from __future__ import annotations
 
@@ -44,6 +46,12 @@ def _bind(lib):
     lib.orc_ternary_acc.argtypes = [p, i64, i64, p, i64, p]
     lib.orc_rescale.restype = None
     lib.orc_rescale.argtypes = [p, i64, i64, p, ctypes.c_double, p]
+    lib.orc_gqa_expand.restype = None
+    lib.orc_gqa_expand.argtypes = [p, i64, i64, i64, i64, p]
+    lib.orc_add_f32.restype = None
+    lib.orc_add_f32.argtypes = [p, p, i64, p]
+    lib.orc_silu_mul.restype = None
+    lib.orc_silu_mul.argtypes = [p, p, i64, p]
     return lib
 
 
@@ -141,3 +149,56 @@ def ternary_linear(x, codes, mean: float):
     acc = ternary_acc(codes, q)
     y = rescale(acc, amax, mean)
     return {"q": q, "amax": amax, "acc": acc, "y": y}
+
+
+# ------------------------------------------------ decoder-layer chain (R13-R16)
+def gqa_expand(v, hidden: int, head_dim: int):
+    """Identity attention (R13): a [M, hidden] float32 from v [M, kv_dim]."""
+    v, pv = _c(v, np.float32)
+    M, kv_dim = v.shape
+    assert hidden % head_dim == 0 and kv_dim % head_dim == 0
+    assert (hidden // head_dim) % (kv_dim // head_dim) == 0
+    a = np.empty((M, hidden), np.float32)
+    _load().orc_gqa_expand(pv, M, kv_dim, hidden, head_dim, a.ctypes.data)
+    return a
+
+
+def add_f32(x, y):
+    """Residual add (R15): float32 x + y, elementwise."""
+    x, px = _c(x, np.float32)
+    y, py = _c(y, np.float32)
+    assert x.shape == y.shape
+    out = np.empty(x.shape, np.float32)
+    _load().orc_add_f32(px, py, x.size, out.ctypes.data)
+    return out
+
+
+def silu_mul(g, u):
+    """SiLU(g) * u in float64 (R16)."""
+    g, pg = _c(g, np.float32)
+    u, pu = _c(u, np.float32)
+    assert g.shape == u.shape
+    out = np.empty(g.shape, np.float64)
+    _load().orc_silu_mul(pg, pu, g.size, out.ctypes.data)
+    return out
+
+
+def decoder_layer(h, layer, head_dim: int = 128):
+    """One layer of the chain in the oracle's own precision, from float32 h
+    [M, hidden] and ``layer`` = dict(q, k, v, o, gate, up, down), each a
+    (codes, mean) pair.  Every projection output is rounded to float32
+    before it is used (the chain passes float32 activations).  Returns a
+    dict of every intermediate; ``h_next`` is the layer's output."""
+    def proj(x, name):
+        codes, mean = layer[name]
+        return ternary_linear(x, codes, mean)["y"].astype(np.float32)
+    hidden = h.shape[1]
+    q, k, v = proj(h, "q"), proj(h, "k"), proj(h, "v")
+    a = gqa_expand(v, hidden, head_dim)
+    o = proj(a, "o")
+    h1 = add_f32(h, o)
+    g, u = proj(h1, "gate"), proj(h1, "up")
+    act = silu_mul(g, u).astype(np.float32)
+    d = proj(act, "down")
+    return {"q": q, "k": k, "v": v, "a": a, "o": o, "h1": h1, "g": g, "u": u,
+            "act": act, "d": d, "h_next": add_f32(h1, d)}

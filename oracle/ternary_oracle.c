@@ -157,3 +157,53 @@ int orc_ternary_linear(const float *x, int64_t M, const int8_t *codes,
     orc_rescale(acc_out, M, N, amax_out, mean, y_out);
     return ovf;
 }
+
+/* ------------------------------------------------------------------------
+ * Decoder-layer chain: the steps on either side of the projections.
+ *
+ * A layer of the LM decoder (a Qwen2.5-1.5B decoder: "VibeVoice-ASR-BitNet-
+ * ONNX" model page, "Layout", where decoder_model_merged maps inputs_embeds
+ * and the KV cache to logits) runs q, k and v on one input, attention, o,
+ * then gate and up on a second input, SiLU(gate) * up, and down.  The chain
+ * keeps those data dependencies and replaces what would need trained weights
+ * or a KV cache by weight-free stand-ins (readings taken here, listed with
+ * the others in the design notes):
+ *   R13 attention is the identity over positions: every token attends only
+ *       to itself, so its output is its own v, each KV head repeated for the
+ *       query heads of its group (hidden/head_dim query heads, kv/head_dim KV
+ *       heads in equal groups).
+ *   R14 no normalisation layers (their gains are weights).
+ *   R15 a residual connection around each block, added in fp32:
+ *       h1 = h + o, then h' = h1 + d.
+ *   R16 SiLU(g) * u with SiLU(z) = z / (1 + e^-z), evaluated here in fp64
+ *       from the fp32 inputs.
+ * ---------------------------------------------------------------------- */
+
+/* R13: a [M x hidden] from v [M x kv_dim]. */
+void orc_gqa_expand(const float *v, int64_t M, int64_t kv_dim, int64_t hidden,
+                    int64_t head_dim, float *a)
+{
+    const int64_t n_heads = hidden / head_dim;
+    const int64_t n_kv = kv_dim / head_dim;
+    const int64_t group = n_heads / n_kv;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t h = 0; h < n_heads; ++h)
+            for (int64_t c = 0; c < head_dim; ++c)
+                a[m * hidden + h * head_dim + c] = v[m * kv_dim + (h / group) * head_dim + c];
+}
+
+/* R15: out = x + y, one IEEE single-precision addition per element. */
+void orc_add_f32(const float *x, const float *y, int64_t n, float *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = x[i] + y[i];
+}
+
+/* R16: out = SiLU(g) * u in fp64. */
+void orc_silu_mul(const float *g, const float *u, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        const double z = (double)g[i];
+        out[i] = z / (1.0 + exp(-z)) * (double)u[i];
+    }
+}

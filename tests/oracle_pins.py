@@ -304,5 +304,92 @@ def pin_nonfinite_weight_rejected():
     raise AssertionError("non-finite W accepted")
 
 
+# ---------------------------------------------- decoder-layer chain stand-ins
+def pin_gqa_expand_hand():
+    """Hand-worked identity attention: 4 query heads of 2 channels over 2 KV
+    heads (groups of 2), then one KV head shared by all, then groups of 1."""
+    v = np.array([[10, 11, 20, 21], [30, 31, 40, 41]], np.float32)
+    assert orc.gqa_expand(v, 8, 2).tolist() == [
+        [10, 11, 10, 11, 20, 21, 20, 21],
+        [30, 31, 30, 31, 40, 41, 40, 41]]
+    assert orc.gqa_expand(v[:, :2], 8, 2).tolist() == [
+        [10, 11] * 4, [30, 31] * 4]
+    assert orc.gqa_expand(v, 4, 2).tolist() == v.tolist()
+
+
+def pin_add_f32_ieee():
+    """Single-precision addition: numpy's float32 add, and the half-even
+    ties 1 + 2^-24 = 1 and 1 + 3*2^-24 = 1 + 2^-22."""
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal(1000).astype(np.float32)
+    y = (rng.standard_normal(1000) * 1e-3).astype(np.float32)
+    assert np.array_equal(orc.add_f32(x, y), x + y)
+    one = np.ones(2, np.float32)
+    t = np.array([2.0 ** -24, 3 * 2.0 ** -24], np.float32)
+    assert orc.add_f32(one, t).tolist() == [1.0, 1.0 + 2.0 ** -22]
+
+
+def pin_silu_closed_forms():
+    """SiLU(0) = 0; SiLU(z) - SiLU(-z) = z; the logistic form z * expit(z)
+    (scipy); large |z| gives z and -0."""
+    from scipy.special import expit
+    one = np.ones(1, np.float32)
+    assert orc.silu_mul(np.zeros(1, np.float32), one)[0] == 0.0
+    z = np.random.default_rng(12).uniform(-20, 20, 500).astype(np.float32)
+    ones = np.ones_like(z)
+    sp, sm = orc.silu_mul(z, ones), orc.silu_mul(-z, ones)
+    assert np.allclose(sp - sm, z.astype(np.float64), rtol=1e-14, atol=1e-14)
+    ref = z.astype(np.float64) * expit(z.astype(np.float64))
+    assert np.allclose(sp, ref, rtol=1e-14, atol=1e-300)
+    big = np.array([1000.0, -1000.0], np.float32)
+    assert orc.silu_mul(big, np.ones(2, np.float32)).tolist() == [1000.0, 0.0]
+
+
+def pin_silu_mul_linear_in_u():
+    """SiLU(g) * u scales with u: u = 0 gives 0, u = c gives c * SiLU(g)."""
+    rng = np.random.default_rng(13)
+    g = rng.standard_normal(200).astype(np.float32)
+    u = rng.standard_normal(200).astype(np.float32)
+    base = orc.silu_mul(g, np.ones_like(g))
+    assert np.array_equal(orc.silu_mul(g, u), base * u.astype(np.float64))
+    assert not orc.silu_mul(g, np.zeros_like(u)).any()
+
+
+def _chain_layer(rng, hidden, kv, inter, zero=()):
+    shapes = {"q": (hidden, hidden), "k": (kv, hidden), "v": (kv, hidden),
+              "o": (hidden, hidden), "gate": (inter, hidden), "up": (inter, hidden),
+              "down": (hidden, inter)}
+    layer = {}
+    for name, (N, K) in shapes.items():
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+        if name in zero:
+            W[:] = 0
+        layer[name] = orc.ternarize(W)
+    return layer
+
+
+def pin_decoder_layer_zero_weights():
+    """All seven projections zero: every intermediate is zero and the layer
+    returns its input exactly (the residuals add +0)."""
+    rng = np.random.default_rng(14)
+    layer = _chain_layer(rng, 256, 128, 512, zero=("q", "k", "v", "o", "gate", "up", "down"))
+    h = rng.standard_normal((3, 256)).astype(np.float32)
+    out = orc.decoder_layer(h, layer)
+    for name in ("q", "k", "v", "a", "o", "g", "u", "act", "d"):
+        assert not out[name].any(), name
+    assert np.array_equal(out["h1"], h) and np.array_equal(out["h_next"], h)
+
+
+def pin_decoder_layer_attention_reads_v():
+    """Identity attention passes v only: with v zero (q, k random) the
+    attention block adds nothing, h1 == h; with v random it does."""
+    rng = np.random.default_rng(15)
+    h = rng.standard_normal((2, 256)).astype(np.float32)
+    zero_v = orc.decoder_layer(h, _chain_layer(rng, 256, 128, 512, zero=("v",)))
+    assert np.array_equal(zero_v["h1"], h)
+    with_v = orc.decoder_layer(h, _chain_layer(rng, 256, 128, 512))
+    assert not np.array_equal(with_v["h1"], h)
+
+
 ALL_PINS = {name: fn for name, fn in sorted(globals().items())
             if name.startswith("pin_") and callable(fn)}

@@ -38,6 +38,10 @@ MUTANTS = {
     "no_floor": ("if (mean < ORC_MEAN_FLOOR)\n        mean = ORC_MEAN_FLOOR;", ""),
     "amax_signed": ("float v = fabsf(row[k]);", "float v = row[k];"),
     "fp32_row_sum": ("double row = 0.0;", "float row = 0.0f;"),
+    "gqa_head_mod": ("(h / group) * head_dim + c]", "(h % n_kv) * head_dim + c]"),
+    "add_subtracts": ("out[i] = x[i] + y[i];", "out[i] = x[i] - y[i];"),
+    "silu_sign": ("z / (1.0 + exp(-z))", "z / (1.0 + exp(z))"),
+    "silu_drops_u": ("exp(-z)) * (double)u[i];", "exp(-z));"),
 }
 # Not listed: removing the amax == 0 special case.  On x86-64 the resulting
 # NaN converts to 0 anyway, so that mutant is equivalent and uncatchable; the
