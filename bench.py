@@ -11,6 +11,11 @@ launch per token group, started early by programmatic dependent launch).
 Prefill sizes (--m > 32) take int8 activations quantised beforehand and run
 the tensor-core kernel (one persistent launch).
 
+--chain times the decoder-layer chain instead: the layers' projections in
+dependency order (q/k/v on one input, identity attention, o and a residual,
+gate/up, SiLU * up, down and a residual), each step all layers from one
+token state, under its own metric name.
+
 Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own
 replica of the sweep on its own token (data-parallel decode; no collective
 on the data path), value = all ranks' tokens / max-over-ranks time.
@@ -46,6 +51,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=28)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--chain", action="store_true",
+                    help="time the dependent decoder-layer chain instead of the sweep")
     return ap.parse_args()
 
 
@@ -225,6 +232,108 @@ def build_workload(api, torch, dev, M, layers, rank):
     return shapes, descs, x_host, x_all, y_all
 
 
+CHAIN_METRIC = "decoder-layer chain tokens/s (28 dependent layers; % of HBM roofline)"
+CHAIN_DIMS = (1536, 256, 128, 8960)   # hidden, kv_dim, head_dim, inter (Qwen2.5-1.5B)
+
+
+def chain_bytes(shapes, M, dims=CHAIN_DIMS):
+    """Algorithmic bytes of one chain step: the sweep's (codes, fp32 x read
+    and y written per projection) plus the element-wise steps per layer
+    (attention stand-in: v read, a written; two residual adds: two reads and
+    a write each; SiLU * up: two reads and a write)."""
+    hidden, kv, hd, inter = dims
+    algo, codes, _ = sweep_bytes(shapes, M)
+    layers = len(shapes) // 7
+    ew = M * 4 * ((kv + hidden) + 2 * 3 * hidden + 3 * inter)
+    return algo + layers * ew, codes
+
+
+def run_chain(args, api, torch, dev, rank, world, dist, local):
+    from ternary_weight_decoder_b200 import synth
+    M = args.m
+    if not 1 <= M <= 32:
+        raise SystemExit("--chain runs decode token counts only (1..32)")
+    shapes, descs, _, x_all, y_all = build_workload(api, torch, dev, M, args.layers, rank)
+    layers = [dict() for _ in range(args.layers)]
+    for (l, _, name, _, _), d in zip(shapes, descs):
+        layers[l][name] = (d["packed"], d["wscale"])
+    del descs, x_all, y_all
+    hidden, kv, hd, inter = CHAIN_DIMS
+    chain = api.DecoderChain(layers, M, hidden, kv, hd, inter, dev)
+    h0_host = torch.from_numpy(synth.activations(rank_layer_seed(0, rank), 0, M, hidden)).pin_memory()
+    h0 = h0_host.to(dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        chain.h.copy_(h0, non_blocking=True)   # every step starts from the same token state
+        api.decoder_chain(chain)
+
+    for _ in range(args.warmup):
+        step()
+    api.check()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        barrier()
+    api.check()
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    ms_per_step = ms / args.steps
+    algo, codes = chain_bytes(shapes, M)
+    hbm, src = peaks()
+    achieved = algo / (ms_per_step / 1e3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        out = torch.empty(M * hidden, dtype=torch.float32).pin_memory()
+        k2 = max(3, min(args.steps, 500))
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(k2):
+            chain.h.copy_(h0_host, non_blocking=True)
+            api.decoder_chain(chain)
+            out.copy_(chain.h.view(-1), non_blocking=True)
+            stream.synchronize()
+        f1.record(stream)
+        barrier()
+        ems = max_over_ranks(f0.elapsed_time(f1), dist, dev)
+        e2e = {"value": job_value(M, world, k2, ems), "unit": UNIT,
+               "h2d_bytes_per_step": M * hidden * 4, "d2h_bytes_per_step": M * hidden * 4,
+               "steps": k2, "ms_per_step": ems / k2}
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": CHAIN_METRIC, "value": job_value(M, world, args.steps, ms), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8xternary->int32, f32 in/out", "data": "synthetic",
+        "config": {"workload": f"decoder_chain_{args.layers}L_M{M}", "M": M,
+                   "layers": args.layers, "hidden": hidden, "kv_dim": kv, "head_dim": hd,
+                   "inter": inter, "parallelism": f"dp{world} (independent replicas)",
+                   "l2": f"codes {codes / 1e6:.0f} MB > 126 MB L2; no flush"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured"
+                     else "fallback 6650 GB/s",
+                     "algorithmic_bytes_per_step": algo, "weight_bytes_per_step": codes,
+                     "note": "step = all layers: per layer 4 sweeps + 4 element-wise launches"},
+        "cpu_baseline": None, "e2e": e2e,
+        "gpu_launches": chain.launches * args.steps, "clocks": clk.summary(),
+    }))
+
+
 def cpu_oracle_sample(M, budget_s=10.0, sample_layers=4, layers=28):
     """Time the reference oracle, as it stands, on one host core: repeated
     passes over the projections of the first `sample_layers` layers until
@@ -328,6 +437,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
+    if args.chain:
+        return run_chain(args, api, torch, dev, rank, world, dist, local)
     M = args.m
     shapes, descs, x_host, x_all, y_all = build_workload(api, torch, dev, M, args.layers, rank)
     if M > 32:   # prefill sweeps consume int8 activations quantised beforehand

@@ -244,6 +244,75 @@ TW_API int tw_decoder_projection_sweep(const void *table_host, const void *table
  * on this encoded table makes (0 for a malformed table). */
 TW_API int tw_sweep_launches(const void *table_host);
 
+/*
+ * Decoder-layer chain
+ * -------------------
+ * The projections of consecutive decoder layers with their data
+ * dependencies.  Per layer: q, k and v read one input h; attention is the
+ * identity over positions (every token attends only to itself, so its
+ * output is its own v, each KV head repeated for the query heads of its
+ * group); o reads that; h1 = h + o; gate and up read h1; act = SiLU(gate) *
+ * up with SiLU(z) = z / (1 + e^-z); down reads act; the layer's output
+ * h1 + down replaces h.  This is the decoder layer of the Qwen2.5-1.5B LM
+ * ("VibeVoice-ASR-BitNet-ONNX" model page, "Layout": decoder_model_merged
+ * maps inputs_embeds and the KV cache to logits) without the parts that need
+ * trained weights or a cache: attention scores, the KV cache and the
+ * normalisation gains.  Residual adds are single-precision; SiLU uses expf.
+ * Decode only: 1 <= M <= 32.
+ */
+typedef struct tw_chain_buffers {
+    float *h;     /* [M x hidden] input of the first layer; output of the last   */
+    float *v;     /* [M x kv_dim] output of v                                     */
+    float *a;     /* [M x hidden] attention output, the input of o                */
+    float *o;     /* [M x hidden] output of o                                     */
+    float *h1;    /* [M x hidden] h + o, the input of gate and up                 */
+    float *g;     /* [M x inter]  output of gate                                  */
+    float *u;     /* [M x inter]  output of up                                    */
+    float *act;   /* [M x inter]  SiLU(g) * u, the input of down                  */
+    float *d;     /* [M x hidden] output of down                                  */
+    int64_t M, hidden, kv_dim, head_dim, inter;
+} tw_chain_buffers;
+
+/*
+ * One layer as four encoded sweep tables (host bytes and device copies, as
+ * for tw_decoder_projection_sweep), encoded for M tokens and the buffers:
+ *   qkv   q [hidden x hidden], k and v [kv_dim x hidden]; every x = h;
+ *         v's y = v (q's and k's outputs go wherever their descriptors say)
+ *   o     [hidden x hidden], x = a, y = o
+ *   gu    gate and up [inter x hidden], x = h1, y = g and u
+ *   down  [hidden x inter], x = act, y = d
+ * acc_out of any descriptor may be set (tests read the integer results).
+ */
+typedef struct tw_chain_layer {
+    const void *qkv_host, *qkv_dev;
+    const void *o_host, *o_dev;
+    const void *gu_host, *gu_dev;
+    const void *down_host, *down_dev;
+} tw_chain_layer;
+
+/* HOST-ONLY.  Scratch of tw_decoder_chain: the largest
+ * tw_sweep_workspace_bytes of the tables (the sweeps run one after another
+ * on one stream and share it; the same zero-fill rule applies).  0 if a
+ * table is missing or malformed. */
+TW_API size_t tw_chain_workspace_bytes(const tw_chain_layer *layers, int n_layers);
+
+/*
+ * Run n_layers layers (host array `layers`, host struct `buf`) in order on
+ * `stream`: per layer four sweeps and four element-wise launches (the
+ * attention stand-in, the two residual adds and SiLU * up).  Every
+ * table is checked on the host against `buf` first -- projection count, N
+ * and K, M, and the x and y pointers named above -- and nothing is launched
+ * if one does not match (TW_ERR_SHAPE, TW_ERR_NULL, TW_ERR_ALIGN,
+ * TW_ERR_CORRUPT or TW_ERR_BUFSIZE).
+ */
+TW_API int tw_decoder_chain(const tw_chain_layer *layers, int n_layers,
+                            const tw_chain_buffers *buf, void *ws, size_t ws_bytes,
+                            tw_stream_t stream);
+
+/* HOST-ONLY.  Kernel launches of one tw_decoder_chain call (0 if a table is
+ * missing or malformed). */
+TW_API int tw_chain_launches(const tw_chain_layer *layers, int n_layers);
+
 /* Wait for `stream`, then return and clear the device error word of the
  * current device (TW_OK if no kernel reported an error). */
 TW_API int tw_check(tw_stream_t stream);

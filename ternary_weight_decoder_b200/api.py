@@ -68,6 +68,9 @@ tw_sweep_launches = _sig("tw_sweep_launches", _int, [_p])
 tw_check = _sig("tw_check", _int, [_p])
 tw_last_error = _sig("tw_last_error", ctypes.c_char_p, [])
 tw_debug_wait_timeout = _sig("tw_debug_wait_timeout", _int, [ctypes.c_uint64, _p])
+tw_chain_workspace_bytes = _sig("tw_chain_workspace_bytes", _sz, [_p, _int])
+tw_decoder_chain = _sig("tw_decoder_chain", _int, [_p, _int, _p, _p, _sz, _p])
+tw_chain_launches = _sig("tw_chain_launches", _int, [_p, _int])
 
 
 class ProjDesc(ctypes.Structure):
@@ -212,7 +215,7 @@ class SweepTable:
     ``tw_sweep_table_encode`` and their device copy.  Keep the tensors named
     by the descriptors alive for as long as the table is used."""
 
-    def __init__(self, descs: Sequence[dict], M: int, device=None):
+    def __init__(self, descs: Sequence[dict], M: int, device=None, workspace: bool = True):
         n = len(descs)
         arr = (ProjDesc * n)()
         for i, d in enumerate(descs):
@@ -233,7 +236,7 @@ class SweepTable:
         # decode scratch: the quantised rows and their scales (rewritten by
         # every call)
         self.ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device=device) \
-            if device is not None else None
+            if device is not None and workspace else None
         self.ws_bytes = wsb
 
 
@@ -245,3 +248,79 @@ def decoder_projection_sweep(table: SweepTable, stream=None):
 
 def debug_wait_timeout(timeout_ns: int, stream=None):
     _raise(tw_debug_wait_timeout(timeout_ns, _stream(stream)))
+
+
+# ------------------------------------------------------ decoder-layer chain
+class ChainBuffers(ctypes.Structure):
+    """Mirror of ``tw_chain_buffers``."""
+    _fields_ = [("h", _p), ("v", _p), ("a", _p), ("o", _p), ("h1", _p), ("g", _p), ("u", _p),
+                ("act", _p), ("d", _p), ("M", _i64), ("hidden", _i64), ("kv_dim", _i64),
+                ("head_dim", _i64), ("inter", _i64)]
+
+
+class ChainLayer(ctypes.Structure):
+    """Mirror of ``tw_chain_layer``."""
+    _fields_ = [("qkv_host", _p), ("qkv_dev", _p), ("o_host", _p), ("o_dev", _p),
+                ("gu_host", _p), ("gu_dev", _p), ("down_host", _p), ("down_dev", _p)]
+
+
+CHAIN_PROJECTIONS = ("q", "k", "v", "o", "gate", "up", "down")
+
+
+class DecoderChain:
+    """The activation buffers and the four sweep tables per layer of a
+    decoder-layer chain over M tokens.
+
+    ``layers`` is a list with, per layer, a dict mapping each of
+    ``CHAIN_PROJECTIONS`` to ``(packed, wscale)`` from ``ternarize_pack``.
+    ``acc_out`` optionally maps (layer, name) to an int32 [M, N] tensor that
+    receives that projection's integer results.  The buffers are the
+    attributes named as in ``tw_chain_buffers`` plus ``q`` and ``k``; ``h``
+    is the input of the first layer and, after a run, the output of the
+    last."""
+
+    def __init__(self, layers, M: int, hidden: int, kv_dim: int, head_dim: int, inter: int,
+                 device, acc_out=None):
+        acc_out = acc_out or {}
+        f32 = dict(dtype=torch.float32, device=device)
+        self.M, self.hidden, self.kv_dim, self.head_dim, self.inter = M, hidden, kv_dim, head_dim, inter
+        for name, width in (("h", hidden), ("q", hidden), ("k", kv_dim), ("v", kv_dim),
+                            ("a", hidden), ("o", hidden), ("h1", hidden), ("g", inter),
+                            ("u", inter), ("act", inter), ("d", hidden)):
+            setattr(self, name, torch.zeros((M, width), **f32))
+        stages = (("qkv", (("q", self.h, self.q, hidden, hidden), ("k", self.h, self.k, kv_dim, hidden),
+                           ("v", self.h, self.v, kv_dim, hidden))),
+                  ("o", (("o", self.a, self.o, hidden, hidden),)),
+                  ("gu", (("gate", self.h1, self.g, inter, hidden), ("up", self.h1, self.u, inter, hidden))),
+                  ("down", (("down", self.act, self.d, hidden, inter),)))
+        self.tables = []
+        c_layers = (ChainLayer * len(layers))()
+        for li, layer in enumerate(layers):
+            row = {}
+            for stage, projs in stages:
+                descs = [dict(x=x, packed=layer[name][0], wscale=layer[name][1], y=y,
+                              acc_out=acc_out.get((li, name)), N=N, K=K)
+                         for name, x, y, N, K in projs]
+                row[stage] = SweepTable(descs, M, device=device, workspace=False)
+            self.tables.append(row)
+            c_layers[li] = ChainLayer(*[_ptr(t) for st in ("qkv", "o", "gu", "down")
+                                        for t in (row[st].host, row[st].device)])
+        self.c_layers = c_layers
+        self.c_buf = ChainBuffers(_ptr(self.h), _ptr(self.v), _ptr(self.a), _ptr(self.o),
+                                  _ptr(self.h1), _ptr(self.g), _ptr(self.u), _ptr(self.act),
+                                  _ptr(self.d), M, hidden, kv_dim, head_dim, inter)
+        self.n_layers = len(layers)
+        self.ws_bytes = int(tw_chain_workspace_bytes(c_layers, self.n_layers))
+        self.ws = torch.zeros(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
+        self.launches = int(tw_chain_launches(c_layers, self.n_layers))
+
+
+def decoder_chain(chain: DecoderChain, first: int = 0, count=None, stream=None):
+    """Run layers first .. first+count-1 of ``chain`` (all by default)."""
+    count = chain.n_layers - first if count is None else count
+    if not (0 <= first and count >= 1 and first + count <= chain.n_layers):
+        raise ValueError("layer range outside the chain")
+    layers = ctypes.cast(ctypes.addressof(chain.c_layers) + first * ctypes.sizeof(ChainLayer),
+                         ctypes.POINTER(ChainLayer))
+    _raise(tw_decoder_chain(layers, count, ctypes.byref(chain.c_buf), _ptr(chain.ws),
+                            chain.ws_bytes, _stream(stream)))

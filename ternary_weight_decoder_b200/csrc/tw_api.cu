@@ -109,6 +109,89 @@ int run_prefill_single(const int8_t *xq, const float *amax, const int32_t *qsum,
     return e == cudaSuccess ? TW_OK : cuda_fail(e, "prefill launch");
 }
 
+// ------------------------------------------------ decoder-layer chain
+// What one of a layer's four sweep tables must hold for the chain buffers.
+struct ChainStage {
+    const char *name;
+    int count;
+    int64_t N[3];
+    int64_t K;
+    const float *x;       // every projection's x
+    const float *y[3];    // required y per projection (null: any)
+};
+
+int check_chain_stage(const void *host, const void *dev, const ChainStage &st, int64_t M, int layer)
+{
+    if (!host || !dev)
+        return fail(TW_ERR_NULL, "chain layer %d: %s table missing", layer, st.name);
+    if ((reinterpret_cast<uintptr_t>(dev) & 63u) != 0)
+        return fail(TW_ERR_ALIGN, "chain layer %d: %s device table must be 64-byte aligned", layer,
+                    st.name);
+    const auto *hdr = static_cast<const tw::TableHeader *>(host);
+    if (hdr->magic != tw::kTableMagic)
+        return fail(TW_ERR_CORRUPT, "chain layer %d: %s table was not produced by "
+                    "tw_sweep_table_encode", layer, st.name);
+    if (hdr->count != st.count || hdr->M != M)
+        return fail(TW_ERR_SHAPE, "chain layer %d: %s table has %d projections at M=%lld, "
+                    "expected %d at M=%lld", layer, st.name, hdr->count, (long long)hdr->M,
+                    st.count, (long long)M);
+    const auto *r = reinterpret_cast<const tw::DescRecord *>(hdr + 1);
+    for (int i = 0; i < st.count; ++i) {
+        if (r[i].N != st.N[i] || r[i].K != st.K)
+            return fail(TW_ERR_SHAPE, "chain layer %d: %s projection %d is %lldx%lld, expected "
+                        "%lldx%lld", layer, st.name, i, (long long)r[i].N, (long long)r[i].K,
+                        (long long)st.N[i], (long long)st.K);
+        if (r[i].x != st.x)
+            return fail(TW_ERR_SHAPE, "chain layer %d: %s projection %d does not read its chain "
+                        "input buffer", layer, st.name, i);
+        if (st.y[i] && r[i].y != st.y[i])
+            return fail(TW_ERR_SHAPE, "chain layer %d: %s projection %d does not write its chain "
+                        "output buffer", layer, st.name, i);
+    }
+    return TW_OK;
+}
+
+// The four stages of one layer for the buffers b.
+void chain_stages(const tw_chain_buffers &b, ChainStage st[4])
+{
+    st[0] = ChainStage{"qkv", 3, {b.hidden, b.kv_dim, b.kv_dim}, b.hidden, b.h, {nullptr, nullptr, b.v}};
+    st[1] = ChainStage{"o", 1, {b.hidden, 0, 0}, b.hidden, b.a, {b.o, nullptr, nullptr}};
+    st[2] = ChainStage{"gate/up", 2, {b.inter, b.inter, 0}, b.hidden, b.h1, {b.g, b.u, nullptr}};
+    st[3] = ChainStage{"down", 1, {b.hidden, 0, 0}, b.inter, b.act, {b.d, nullptr, nullptr}};
+}
+
+void layer_tables(const tw_chain_layer &L, const void *host[4], const void *dev[4])
+{
+    host[0] = L.qkv_host, dev[0] = L.qkv_dev;
+    host[1] = L.o_host, dev[1] = L.o_dev;
+    host[2] = L.gu_host, dev[2] = L.gu_dev;
+    host[3] = L.down_host, dev[3] = L.down_dev;
+}
+
+int check_chain_buffers(const tw_chain_buffers *b)
+{
+    if (!b)
+        return fail(TW_ERR_NULL, "tw_decoder_chain: buffers required");
+    const void *ptrs[] = {b->h, b->v, b->a, b->o, b->h1, b->g, b->u, b->act, b->d};
+    for (const void *q : ptrs) {
+        if (!q)
+            return fail(TW_ERR_NULL, "tw_decoder_chain: every chain buffer is required");
+        if (!aligned16(q))
+            return fail(TW_ERR_ALIGN, "tw_decoder_chain: chain buffers must be 16-byte aligned");
+    }
+    if (b->M < 1 || b->M > tw::kDecodeMaxM)
+        return fail(TW_ERR_SHAPE, "tw_decoder_chain: M=%lld outside 1..%d (decode only)",
+                    (long long)b->M, tw::kDecodeMaxM);
+    if (b->hidden <= 0 || b->inter <= 0 || b->hidden % 128 || b->inter % 128)
+        return fail(TW_ERR_SHAPE, "tw_decoder_chain: hidden and inter must be positive "
+                    "multiples of 128");
+    if (b->head_dim <= 0 || b->kv_dim <= 0 || b->hidden % b->head_dim || b->kv_dim % b->head_dim ||
+        (b->hidden / b->head_dim) % (b->kv_dim / b->head_dim))
+        return fail(TW_ERR_SHAPE, "tw_decoder_chain: hidden and kv_dim must be whole heads of "
+                    "head_dim, the query heads an equal number per KV head");
+    return TW_OK;
+}
+
 }  // namespace
 
 namespace tw {
@@ -524,6 +607,93 @@ int tw_debug_wait_timeout(uint64_t timeout_ns, tw_stream_t stream)
         return rc;
     cudaError_t e = tw::launch_wait_probe(err, timeout_ns, stream);
     return e == cudaSuccess ? TW_OK : cuda_fail(e, "wait probe launch");
+}
+
+size_t tw_chain_workspace_bytes(const tw_chain_layer *layers, int n_layers)
+{
+    if (!layers || n_layers < 1)
+        return 0;
+    size_t need = 0;
+    for (int l = 0; l < n_layers; ++l) {
+        const void *host[4], *dev[4];
+        layer_tables(layers[l], host, dev);
+        for (int s = 0; s < 4; ++s) {
+            const auto *hdr = static_cast<const tw::TableHeader *>(host[s]);
+            if (!hdr || hdr->magic != tw::kTableMagic)
+                return 0;
+            need = std::max(need, (size_t)hdr->ws_bytes);
+        }
+    }
+    return need;
+}
+
+int tw_chain_launches(const tw_chain_layer *layers, int n_layers)
+{
+    if (!layers || n_layers < 1)
+        return 0;
+    int n = 0;
+    for (int l = 0; l < n_layers; ++l) {
+        const void *host[4], *dev[4];
+        layer_tables(layers[l], host, dev);
+        for (int s = 0; s < 4; ++s) {
+            const int k = host[s] ? tw_sweep_launches(host[s]) : 0;
+            if (k == 0)
+                return 0;
+            n += k;
+        }
+        n += 4;  // attention stand-in, two residual adds, SiLU * up
+    }
+    return n;
+}
+
+int tw_decoder_chain(const tw_chain_layer *layers, int n_layers, const tw_chain_buffers *buf,
+                     void *ws, size_t ws_bytes, tw_stream_t stream)
+{
+    t_last_error[0] = 0;
+    if (!layers || n_layers < 1)
+        return fail(TW_ERR_NULL, "tw_decoder_chain: at least one layer required");
+    if (int rc = check_chain_buffers(buf))
+        return rc;
+    const tw_chain_buffers &b = *buf;
+    ChainStage st[4];
+    chain_stages(b, st);
+    // Every table is checked before anything is launched.
+    for (int l = 0; l < n_layers; ++l) {
+        const void *host[4], *dev[4];
+        layer_tables(layers[l], host, dev);
+        for (int s = 0; s < 4; ++s)
+            if (int rc = check_chain_stage(host[s], dev[s], st[s], b.M, l))
+                return rc;
+    }
+    const size_t need = tw_chain_workspace_bytes(layers, n_layers);
+    if (!ws || ws_bytes < need)
+        return fail(TW_ERR_BUFSIZE, "tw_decoder_chain: workspace %zu < %zu bytes", ws_bytes, need);
+    if (!aligned16(ws))
+        return fail(TW_ERR_ALIGN, "tw_decoder_chain: workspace must be 16-byte aligned");
+
+    for (int l = 0; l < n_layers; ++l) {
+        const void *host[4], *dev[4];
+        layer_tables(layers[l], host, dev);
+        int rc = tw_decoder_projection_sweep(host[0], dev[0], ws, ws_bytes, stream);
+        if (rc)
+            return rc;
+        cudaError_t e = tw::launch_gqa_expand(b.v, b.a, b.M, b.kv_dim, b.hidden, b.head_dim, stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "chain attention launch");
+        if ((rc = tw_decoder_projection_sweep(host[1], dev[1], ws, ws_bytes, stream)))
+            return rc;
+        if ((e = tw::launch_add_f32(b.h, b.o, b.h1, b.M * b.hidden, stream)) != cudaSuccess)
+            return cuda_fail(e, "chain residual launch");
+        if ((rc = tw_decoder_projection_sweep(host[2], dev[2], ws, ws_bytes, stream)))
+            return rc;
+        if ((e = tw::launch_silu_mul(b.g, b.u, b.act, b.M * b.inter, stream)) != cudaSuccess)
+            return cuda_fail(e, "chain SiLU launch");
+        if ((rc = tw_decoder_projection_sweep(host[3], dev[3], ws, ws_bytes, stream)))
+            return rc;
+        if ((e = tw::launch_add_f32(b.h1, b.d, b.h, b.M * b.hidden, stream)) != cudaSuccess)
+            return cuda_fail(e, "chain residual launch");
+    }
+    return TW_OK;
 }
 
 }  // extern "C"

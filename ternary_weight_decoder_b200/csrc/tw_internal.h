@@ -55,6 +55,14 @@ static_assert(sizeof(TableHeader) == 64, "header size");
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Element-wise steps of the decoder-layer chain (tw_chain.cu).
+cudaError_t launch_gqa_expand(const float *v, float *a, int64_t M, int64_t kv_dim,
+                              int64_t hidden, int64_t head_dim, cudaStream_t stream);
+cudaError_t launch_add_f32(const float *x, const float *y, float *out, int64_t n,
+                           cudaStream_t stream);
+cudaError_t launch_silu_mul(const float *g, const float *u, float *out, int64_t n,
+                            cudaStream_t stream);
+
 // ------------------------------------------------------------ launchers
 // Each returns a cudaError_t from the launch.
 cudaError_t launch_ternarize(const float *W, int64_t N, int64_t K, uint8_t *packed,

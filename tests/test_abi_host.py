@@ -173,3 +173,108 @@ def test_sweep_launch_count_196(lib, M):
     # 8 for M <= 2, 4 for M = 3..4, 2 or 1 from M = 5 on
     quant = 1 if M <= 4 else 2
     assert api.tw_sweep_launches(buf.ctypes.data) == quant + 1
+
+
+# ------------------------------------------------------ decoder-layer chain
+CHAIN_BUFS = ("h", "v", "a", "o", "h1", "g", "u", "act", "d")
+
+
+def _fake_chain(M=1, hidden=256, kv=128, hd=128, inter=512, n_layers=2, tweak=None):
+    """Encoded tables of a chain over placeholder device addresses (nothing
+    is launched): per layer qkv, o, gate/up and down, as the chain wants
+    them unless `tweak(layer, stage, descs)` changes the descriptors."""
+    from ternary_weight_decoder_b200 import api
+    addr = {n: 0x7f0000000000 + 0x100000 * i for i, n in enumerate(CHAIN_BUFS + ("q", "k"))}
+    stages = {"qkv": [("h", "q", hidden, hidden), ("h", "k", kv, hidden), ("h", "v", kv, hidden)],
+              "o": [("a", "o", hidden, hidden)],
+              "gu": [("h1", "g", inter, hidden), ("h1", "u", inter, hidden)],
+              "down": [("act", "d", hidden, inter)]}
+    keep, layers = [], (api.ChainLayer * n_layers)()
+    for li in range(n_layers):
+        ptrs = []
+        for st in ("qkv", "o", "gu", "down"):
+            descs = stages[st]
+            arr = (api.ProjDesc * len(descs))()
+            for i, (x, y, N, K) in enumerate(descs):
+                w = 0x7d0000000000 + 0x1000000 * (8 * li + i)
+                arr[i] = api.ProjDesc(x=addr[x], xq=None, amax=None, qsum=None, packed=w,
+                                      wscale=w + 0x800000, y=addr[y], acc_out=None, N=N, K=K)
+            if tweak:
+                tweak(li, st, arr)
+            n = api.tw_sweep_table_bytes(len(descs))
+            buf = np.zeros(n, np.uint8)
+            assert api.tw_sweep_table_encode(arr, len(descs), M, buf.ctypes.data, n) == 0, \
+                api.tw_last_error()
+            keep.append(buf)
+            ptrs += [buf.ctypes.data, 0x7e0000000000 + 0x10000 * len(keep)]
+        layers[li] = api.ChainLayer(*ptrs)
+    cbuf = api.ChainBuffers(*[addr[n] for n in CHAIN_BUFS], M, hidden, kv, hd, inter)
+    return layers, cbuf, keep
+
+
+def test_chain_launch_count_and_workspace(lib):
+    """Per layer four sweeps of one quantisation and one decode launch each
+    (at M = 1) and four element-wise launches; the workspace is the largest
+    table's."""
+    from ternary_weight_decoder_b200 import api
+    layers, cbuf, keep = _fake_chain(n_layers=3)
+    assert api.tw_chain_launches(layers, 3) == 3 * (4 * 2 + 4)
+    per_table = [api.tw_sweep_workspace_bytes(b.ctypes.data) for b in keep]
+    assert api.tw_chain_workspace_bytes(layers, 3) == max(per_table)
+    assert api.tw_chain_launches(layers, 0) == 0
+    assert api.tw_chain_workspace_bytes(None, 1) == 0
+
+
+def test_chain_checks_every_table_before_launching(lib):
+    """A well-formed chain passes every host check and stops only at the
+    missing workspace (nothing launched)."""
+    from ternary_weight_decoder_b200 import api
+    import ctypes
+    layers, cbuf, keep = _fake_chain()
+    assert api.tw_decoder_chain(layers, 2, ctypes.byref(cbuf), None, 0, None) == 4
+    assert b"workspace" in api.tw_last_error()
+
+
+def _tw(arr, i, **kw):
+    for k, v in kw.items():
+        setattr(arr[i], k, v)
+
+
+@pytest.mark.parametrize("case,status", [
+    ("o_reads_wrong_buffer", 2), ("v_writes_wrong_buffer", 2), ("down_wrong_K", 2),
+    ("gate_wrong_N", 2), ("qkv_two_projections", 2), ("table_other_M", 2)])
+def test_chain_rejects_mismatched_tables(lib, case, status):
+    from ternary_weight_decoder_b200 import api
+    import ctypes
+    M = 1
+    tweaks = {
+        "o_reads_wrong_buffer": lambda l, st, a: st == "o" and l == 1 and _tw(a, 0, x=a[0].x + 0x100000),
+        "v_writes_wrong_buffer": lambda l, st, a: st == "qkv" and _tw(a, 2, y=a[2].y + 0x100000),
+        "down_wrong_K": lambda l, st, a: st == "down" and _tw(a, 0, K=256),
+        "gate_wrong_N": lambda l, st, a: st == "gu" and _tw(a, 0, N=384),
+    }
+    if case in tweaks:
+        layers, cbuf, keep = _fake_chain(tweak=tweaks[case])
+    elif case == "qkv_two_projections":
+        layers, cbuf, keep = _fake_chain()
+        other, _, keep2 = _fake_chain(tweak=None)
+        keep += keep2
+        # a two-projection table (gate/up of another chain) where qkv belongs
+        layers[0].qkv_host, layers[0].qkv_dev = other[0].gu_host, other[0].gu_dev
+    else:
+        layers, cbuf, keep = _fake_chain(M=2)
+        cbuf.M = M
+    assert api.tw_decoder_chain(layers, 2, ctypes.byref(cbuf), 0x7c0000000000, 1 << 30, None) == status
+    assert api.tw_last_error()
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("h", None, 1), ("act", 0x7f0000000008, 3), ("M", 33, 2), ("M", 0, 2),
+    ("hidden", 200, 2), ("head_dim", 96, 2), ("kv_dim", 384, 2)])
+def test_chain_rejects_bad_buffers(lib, field, value, status):
+    from ternary_weight_decoder_b200 import api
+    import ctypes
+    layers, cbuf, keep = _fake_chain()
+    setattr(cbuf, field, value)
+    assert api.tw_decoder_chain(layers, 2, ctypes.byref(cbuf), 0x7c0000000000, 1 << 30, None) == status
+    assert api.tw_last_error()
