@@ -212,8 +212,9 @@ def _dp(d, key):
 
 class SweepTable:
     """An encoded sweep over many projections: the host bytes written by
-    ``tw_sweep_table_encode`` and their device copy.  Keep the tensors named
-    by the descriptors alive for as long as the table is used."""
+    ``tw_sweep_table_encode`` and their device copy.  The table holds
+    references to the tensors its descriptors name (it stores their
+    addresses), so they stay allocated for as long as the table does."""
 
     def __init__(self, descs: Sequence[dict], M: int, device=None, workspace: bool = True):
         n = len(descs)
@@ -228,6 +229,7 @@ class SweepTable:
             if torch.cuda.is_available() else torch.empty(nbytes, dtype=torch.uint8)
         _raise(tw_sweep_table_encode(arr, n, M, _ptr(self.host), nbytes))
         self.count, self.M = n, M
+        self.descs = [dict(d) for d in descs]   # owns what the records point at
         self.device = None
         if device is not None:
             self.device = self.host.to(device, non_blocking=False)
@@ -281,7 +283,11 @@ class DecoderChain:
 
     def __init__(self, layers, M: int, hidden: int, kv_dim: int, head_dim: int, inter: int,
                  device, acc_out=None):
-        acc_out = acc_out or {}
+        acc_out = dict(acc_out or {})
+        # The tables store addresses only: hold the weights and integer
+        # outputs here so that they outlive every run of the chain.
+        self.layers = [dict(layer) for layer in layers]
+        self.acc_out = acc_out
         f32 = dict(dtype=torch.float32, device=device)
         self.M, self.hidden, self.kv_dim, self.head_dim, self.inter = M, hidden, kv_dim, head_dim, inter
         for name, width in (("h", hidden), ("q", hidden), ("k", kv_dim), ("v", kv_dim),

@@ -278,3 +278,34 @@ def test_chain_rejects_bad_buffers(lib, field, value, status):
     setattr(cbuf, field, value)
     assert api.tw_decoder_chain(layers, 2, ctypes.byref(cbuf), 0x7c0000000000, 1 << 30, None) == status
     assert api.tw_last_error()
+
+
+def test_chain_binding_owns_the_tensors_it_points_at(lib):
+    """The tables hold raw addresses; the binding must keep the weights and
+    integer outputs alive after the caller drops them (a freed weight scale
+    reused by a later allocation would silently change the outputs)."""
+    import gc
+    import weakref
+    import torch
+    from ternary_weight_decoder_b200 import api
+    hidden, kv, hd, inter = 256, 128, 128, 512
+    shapes = {"q": (hidden, hidden), "k": (kv, hidden), "v": (kv, hidden), "o": (hidden, hidden),
+              "gate": (inter, hidden), "up": (inter, hidden), "down": (hidden, inter)}
+    layers = [{n: (torch.zeros(api.packed_bytes(N, K), dtype=torch.uint8), torch.ones(4))
+               for n, (N, K) in shapes.items()} for _ in range(2)]
+    acc = {(1, "k"): torch.zeros((1, kv), dtype=torch.int32)}
+    refs = [weakref.ref(t) for layer in layers for pair in layer.values() for t in pair]
+    refs.append(weakref.ref(acc[(1, "k")]))
+    chain = api.DecoderChain(layers, 1, hidden, kv, hd, inter, torch.device("cpu"), acc_out=acc)
+    del layers, acc
+    gc.collect()
+    assert all(r() is not None for r in refs)
+    assert chain.launches == 2 * (4 * 2 + 4)
+    # a sweep table alone owns its descriptors' tensors too
+    x = torch.zeros((1, 128))
+    t = api.SweepTable([dict(x=x, packed=torch.zeros(api.packed_bytes(16, 128), dtype=torch.uint8),
+                             wscale=torch.ones(4), y=torch.zeros((1, 16)), N=16, K=128)], 1)
+    r = weakref.ref(x)
+    del x
+    gc.collect()
+    assert r() is not None and t.count == 1
