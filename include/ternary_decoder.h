@@ -303,7 +303,10 @@ TW_API size_t tw_chain_workspace_bytes(const tw_chain_layer *layers, int n_layer
  * table is checked on the host against `buf` first -- projection count, N
  * and K, M, and the x and y pointers named above -- and nothing is launched
  * if one does not match (TW_ERR_SHAPE, TW_ERR_NULL, TW_ERR_ALIGN,
- * TW_ERR_CORRUPT or TW_ERR_BUFSIZE).
+ * TW_ERR_CORRUPT or TW_ERR_BUFSIZE).  A launch that fails part-way returns
+ * TW_ERR_CUDA with the earlier steps already enqueued; the buffers then hold
+ * a partial result.  The caller keeps the tables, buffers, weights and `ws`
+ * allocated until the stream has finished the call.
  */
 TW_API int tw_decoder_chain(const tw_chain_layer *layers, int n_layers,
                             const tw_chain_buffers *buf, void *ws, size_t ws_bytes,
