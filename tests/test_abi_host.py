@@ -301,6 +301,11 @@ def test_chain_binding_owns_the_tensors_it_points_at(lib):
     gc.collect()
     assert all(r() is not None for r in refs)
     assert chain.launches == 2 * (4 * 2 + 4)
+    # the binding's tables pass every host check of the chain; with no
+    # workspace the call stops there, before any launch
+    import ctypes
+    assert api.tw_decoder_chain(chain.c_layers, 2, ctypes.byref(chain.c_buf), None, 0, None) == 4
+    assert b"workspace" in api.tw_last_error()
     # a sweep table alone owns its descriptors' tensors too
     x = torch.zeros((1, 128))
     t = api.SweepTable([dict(x=x, packed=torch.zeros(api.packed_bytes(16, 128), dtype=torch.uint8),
