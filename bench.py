@@ -1,20 +1,30 @@
 """Benchmark of the ternary-weight decoder projections on B200.
 
-Default workload: the full decode sweep — 28 layers x 7 projections = 196
+Headline workload: the full decode sweep -- 28 layers x 7 projections = 196
 ternary matrices of a Qwen2.5-1.5B-shaped decoder (q/o 1536x1536, k/v
 256x1536, gate/up 8960x1536, down 1536x8960; 1,310,195,712 weights,
 327,548,928 bytes of 2-bit codes), one token (M = 1), seeded synthetic
 weights N(0, 0.02^2) and activations N(0, 1) with 1% outlier channels x20.
 A step is one pass of the whole hot path over every projection: activation
-quantisation (one launch), then ternary product and rescale (one persistent
-launch per token group, started early by programmatic dependent launch).
-Prefill sizes (--m > 32) take int8 activations quantised beforehand and run
-the tensor-core kernel (one persistent launch).
+quantisation, then ternary product and rescale (one persistent launch per
+token group, started early by programmatic dependent launch).
 
---chain times the decoder-layer chain instead: the layers' projections in
-dependency order (q/k/v on one input, identity attention, o and a residual,
-gate/up, SiLU * up, down and a residual), each step all layers from one
-token state, under its own metric name.
+The same JSON line carries a ``configs`` object with every workload of the
+benchmark definition, measured in the same run on the same weights:
+
+  1. one 1536x1536 GEMV at M = 1 (x without outliers), L2 flushed before
+     every call: us per call, median and p10/p90;
+  2. one decoder layer's 7 projections at M = 1 as one sweep call, L2
+     flushed before every call: us per matrix;
+  3. the headline (196 projections, M = 1);
+  4. the 196-projection sweep at M = 4, 8, 16, 32 (fraction of HBM);
+  5. the 196-projection prefill sweep at M = 256, 1024, 4096 on int8
+     activations quantised beforehand (fraction of the int8 tensor peak);
+  and the decoder-layer chain (28 dependent layers at M = 1).
+Each decode/prefill entry also carries the oracle timed on the host's cores
+on a bounded sample (labelled, extrapolated by weight count and tokens).
+
+--chain times only the decoder-layer chain, under its own metric name.
 
 Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own
 replica of the sweep on its own token (data-parallel decode; no collective
@@ -25,6 +35,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -39,56 +50,92 @@ METRIC = "196-matrix ternary decode sweep tokens/s & weight GB/s (% of HBM roofl
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+DTYPE = "int8xternary->int32, f32 in/out"
+DECODE_MS = (4, 8, 16, 32)
+PREFILL_MS = (256, 1024, 4096)
+L2_FLUSH_BYTES = 256 << 20   # > 2 x the 126 MB L2
+PREFILL_DISTINCT_ROWS = 256  # distinct generated token rows per projection (tiled up to M)
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--m", type=int, default=1, help="tokens per step (decode: 1..32)")
+    ap.add_argument("--m", type=int, default=1, help="tokens per step of the headline sweep")
     ap.add_argument("--layers", type=int, default=28)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="headline only (no configs object)")
+    ap.add_argument("--configs", default="1,2,4,5,chain",
+                    help="comma list of the extra workloads to measure")
     ap.add_argument("--chain", action="store_true",
                     help="time the dependent decoder-layer chain instead of the sweep")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def peaks():
+    """(HBM GB/s, int8 dense TOP/s, source).  The int8 peak is 2 x the
+    measured bf16 burst (the nominal int8 : bf16 dense ratio, 4.5 : 2.25)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return d.get("hbm_gbs", FALLBACK_HBM_GBS), "measured"
-    return FALLBACK_HBM_GBS, "fallback"
+        return (d.get("hbm_gbs", FALLBACK_HBM_GBS),
+                2 * d.get("bf16_tflops", FALLBACK_BF16_TFLOPS), "measured")
+    return FALLBACK_HBM_GBS, 2 * FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def peak_source(src):
+    return ("measured (MEASURED_PEAKS.json hbm_gbs; int8 = 2 x bf16_tflops)"
+            if src == "measured" else "fallback 6650 GB/s; int8 = 2 x 1590 TFLOP/s")
 
 
 def _strip_comments(text):
     """C/C++/CUDA source without comments, trailing blanks or empty lines."""
-    import re
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     text = re.sub(r"//[^\n]*", "", text)
     return "\n".join(l.rstrip() for l in text.splitlines() if l.strip())
 
 
-def code_digest(kernel_src, read=None):
-    """sha256 over the code of one kernel source file and of the library's
-    headers (comments and blank lines removed): an ncu capture stays valid
-    across comment edits and stops applying on any change of code.
-    `read(relpath)` returns a file's text (default: the working tree)."""
-    import glob
-    import hashlib
+# The public C header declares host entry points only; no kernel's device
+# code depends on it, so an edit there keeps a capture valid.
+_HOST_ONLY_HEADERS = (os.path.join("include", "ternary_decoder.h"),)
+
+
+def kernel_sources(kernel_src, read=None):
+    """The kernel's source file and every local header it includes,
+    transitively (quoted includes), minus the host-only public header."""
     if read is None:
         def read(rel):
             with open(os.path.join(ROOT, rel)) as f:
                 return f.read()
     csrc = os.path.join("ternary_weight_decoder_b200", "csrc")
-    rels = [os.path.join(csrc, kernel_src)]
-    for pat in (os.path.join(csrc, "*.cuh"), os.path.join(csrc, "*.h"), os.path.join("include", "*.h")):
-        rels += sorted(os.path.relpath(q, ROOT) for q in glob.glob(os.path.join(ROOT, pat)))
+    todo, seen = [os.path.join(csrc, kernel_src)], []
+    while todo:
+        rel = os.path.normpath(todo.pop(0))
+        if rel in seen or rel in _HOST_ONLY_HEADERS:
+            continue
+        seen.append(rel)
+        for inc in re.findall(r'^\s*#\s*include\s+"([^"]+)"', _strip_comments(read(rel)), re.M):
+            todo.append(os.path.join(os.path.dirname(rel), inc))
+    return seen
+
+
+def code_digest(kernel_src, read=None):
+    """sha256 over the code of one kernel source file and of the local
+    headers it includes (comments and blank lines removed): an ncu capture
+    stays valid across comment edits and stops applying on any change of
+    the code the kernel is compiled from.  `read(relpath)` returns a file's
+    text (default: the working tree)."""
+    import hashlib
+    if read is None:
+        def read(rel):
+            with open(os.path.join(ROOT, rel)) as f:
+                return f.read()
     h = hashlib.sha256()
-    for rel in rels:
+    for rel in kernel_sources(kernel_src, read):
         h.update(rel.encode() + b"\0" + _strip_comments(read(rel)).encode() + b"\0")
     return h.hexdigest()
 
@@ -109,12 +156,45 @@ def profiled_traffic(kernel_src, M, layers):
     return None
 
 
+def decode_kernel_src(M):
+    """Source file of the dominant kernel of a sweep of M tokens."""
+    return "tw_prefill.cu" if M > 32 else "tw_decode_tc.cu" if M > 16 else "tw_decode.cu"
+
+
 def sweep_bytes(shapes, M):
     codes = sum((-(-N // 16) * 16) * K // 4 for (_, _, _, N, K) in shapes)
     algo_codes = sum(N * K // 4 for (_, _, _, N, K) in shapes)
     xin = sum(M * K * 4 for (_, _, _, N, K) in shapes)
     yout = sum(M * N * 4 for (_, _, _, N, K) in shapes)
     return algo_codes + xin + yout, algo_codes, codes
+
+
+def sweep_ops(shapes, M):
+    return sum(2 * M * N * K for (_, _, _, N, K) in shapes)
+
+
+def dist_summary(per_ms):
+    """Median and 10th/90th percentiles (us) of per-step times in ms."""
+    a = np.asarray(per_ms, np.float64) * 1e3
+    return {"median_us": float(np.median(a)), "p10_us": float(np.percentile(a, 10)),
+            "p90_us": float(np.percentile(a, 90)), "samples": int(a.size)}
+
+
+def cpu_info():
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except AttributeError:
+        avail = os.cpu_count()
+    return {"cpu_model": model, "nproc": os.cpu_count(), "cpus_available": avail}
 
 
 class ClockSampler:
@@ -132,7 +212,7 @@ class ClockSampler:
         except Exception as e:  # no NVML: report that instead of clocks
             self.nv, self.err = None, str(e)
 
-    def _run(self):
+    def _sample(self):
         nv = self.nv
         names = {
             "hw_slowdown": getattr(nv, "nvmlClocksThrottleReasonHwSlowdown", 0x8),
@@ -140,20 +220,24 @@ class ClockSampler:
             "sw_thermal_slowdown": getattr(nv, "nvmlClocksThrottleReasonSwThermalSlowdown", 0x20),
             "sw_power_cap": getattr(nv, "nvmlClocksThrottleReasonSwPowerCap", 0x4),
         }
+        try:
+            mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+            self.samples.append(mhz)
+            for k, bit in names.items():
+                if r & bit:
+                    self.reasons.add(k)
+        except Exception:
+            pass
+
+    def _run(self):
         while not self.stop_ev.is_set():
-            try:
-                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
-                r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
-                self.samples.append(mhz)
-                for k, bit in names.items():
-                    if r & bit:
-                        self.reasons.add(k)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(0.002)
 
     def __enter__(self):
         if self.nv:
+            self._sample()   # at least one sample inside the region
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         return self
@@ -162,6 +246,7 @@ class ClockSampler:
         if self.nv:
             self.stop_ev.set()
             self.t.join()
+            self._sample()
 
     def summary(self):
         if not self.nv:
@@ -192,25 +277,19 @@ def job_value(M, world, steps, max_ms):
     return M * world * steps / (max_ms / 1e3)
 
 
-def build_workload(api, torch, dev, M, layers, rank):
-    """Generate, upload and ternarise the sweep; return descriptors and buffers."""
+def _pool():
+    import concurrent.futures as cf
+    return cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 4))
+
+
+def build_weights(api, torch, dev, layers):
+    """Generate and ternarise the 196 (7 x layers) projections on the GPU:
+    [(layer, proj, name, N, K)] and [(packed, wscale)]."""
     from ternary_weight_decoder_b200 import synth
     shapes = synth.sweep_shapes(layers)
-    x_off, y_off, xo, yo = [], [], 0, 0
-    for (_, _, _, N, K) in shapes:
-        x_off.append(xo)
-        y_off.append(yo)
-        xo += M * K
-        yo += M * N
-    x_host = torch.empty(xo, dtype=torch.float32).pin_memory()
-    xn = x_host.numpy()
-    descs = []
-    x_all = torch.empty(xo, dtype=torch.float32, device=dev)
-    y_all = torch.empty(yo, dtype=torch.float32, device=dev)
-    import concurrent.futures as cf
-    pool = cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 4))
+    pool = _pool()
     window = 16   # bounds host memory: at most this many fp32 matrices alive
-    futs = {}
+    futs, weights = {}, []
     for i, (l, p, name, N, K) in enumerate(shapes):
         for j in range(i, min(i + window, len(shapes))):
             if j not in futs:
@@ -218,18 +297,105 @@ def build_workload(api, torch, dev, M, layers, rank):
                 futs[j] = pool.submit(synth.weights, lj, pj, Nj, Kj)
         W = futs.pop(i).result()
         Wd = torch.from_numpy(W).to(dev)
-        packed, mean_abs, wscale = api.ternarize_pack(Wd)
+        packed, _, wscale = api.ternarize_pack(Wd)
         del Wd, W
-        # each rank decodes its own token stream
-        xn[x_off[i]:x_off[i] + M * K] = synth.activations(rank_layer_seed(l, rank), p, M, K).ravel()
+        weights.append((packed, wscale))
+    api.check()
+    pool.shutdown()
+    return shapes, weights
+
+
+def decode_inputs(api, torch, dev, shapes, weights, M, rank, with_host=False):
+    """Decode-sweep descriptors over M tokens: per projection its own seeded
+    x (one contiguous device buffer) and y.  Returns (descs, x_host, x_all,
+    y_all); x_host (pinned) only when with_host."""
+    from ternary_weight_decoder_b200 import synth
+    x_off, y_off, xo, yo = [], [], 0, 0
+    for (_, _, _, N, K) in shapes:
+        x_off.append(xo)
+        y_off.append(yo)
+        xo += M * K
+        yo += M * N
+    x_host = torch.empty(xo, dtype=torch.float32)
+    if with_host:
+        x_host = x_host.pin_memory()
+    xn = x_host.numpy()
+    pool = _pool()
+    futs = [pool.submit(synth.activations, rank_layer_seed(l, rank), p, M, K)
+            for (l, p, _, _, K) in shapes]
+    for i, f in enumerate(futs):
+        K = shapes[i][4]
+        xn[x_off[i]:x_off[i] + M * K] = f.result().ravel()
+    pool.shutdown()
+    x_all = x_host.to(dev)
+    y_all = torch.empty(yo, dtype=torch.float32, device=dev)
+    descs = []
+    for i, (_, _, _, N, K) in enumerate(shapes):
+        packed, wscale = weights[i]
         descs.append(dict(x=x_all[x_off[i]:x_off[i] + M * K].view(M, K), packed=packed,
                           wscale=wscale, y=y_all[y_off[i]:y_off[i] + M * N].view(M, N),
                           N=N, K=K))
-    api.check()
-    pool.shutdown()
-    x_all.copy_(x_host)
     torch.cuda.synchronize()
-    return shapes, descs, x_host, x_all, y_all
+    return descs, (x_host if with_host else None), x_all, y_all
+
+
+def prefill_inputs(api, torch, dev, shapes, weights, M, rank):
+    """Prefill-sweep descriptors over M tokens: per projection
+    PREFILL_DISTINCT_ROWS seeded token rows (with outliers) tiled up to M,
+    quantised once by tw_quantize_act; y [M x N] per projection."""
+    from ternary_weight_decoder_b200 import synth
+    R = min(M, PREFILL_DISTINCT_ROWS)
+    pool = _pool()
+    futs = [pool.submit(synth.activations, rank_layer_seed(l, rank), p, R, K)
+            for (l, p, _, _, K) in shapes]
+    descs = []
+    for i, (_, _, _, N, K) in enumerate(shapes):
+        xr = torch.from_numpy(futs[i].result()).to(dev)
+        x = xr.repeat((M + R - 1) // R, 1)[:M].contiguous()
+        xq, amax, qsum = api.quantize_act(x)
+        del x, xr
+        packed, wscale = weights[i]
+        descs.append(dict(xq=xq, amax=amax, qsum=qsum, packed=packed, wscale=wscale,
+                          y=torch.empty((M, N), dtype=torch.float32, device=dev), N=N, K=K))
+    pool.shutdown()
+    api.check()
+    return descs
+
+
+def timed_steps(torch, stream, fn, steps, barrier):
+    """Run fn `steps` times between a barrier + synchronize on each side;
+    an event at every step boundary on `stream`.  Returns (total ms, per-step
+    ms list)."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    barrier()
+    evs[0].record(stream)
+    for i in range(steps):
+        fn()
+        evs[i + 1].record(stream)
+    barrier()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+    return evs[0].elapsed_time(evs[steps]), per
+
+
+def cold_calls(torch, stream, fn, n, flush, batch=32, sleep_cycles=40_000_000):
+    """Device time of `n` calls of fn, each after an L2 flush (`flush()`
+    writes more than the L2 holds; it is not timed).  A spin kernel at the
+    head of every batch lets the host queue the whole batch, so the events
+    bracket device work and not host launch gaps.  Returns per-call ms."""
+    per = []
+    for b0 in range(0, n, batch):
+        nb = min(batch, n - b0)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(nb)]
+        torch.cuda._sleep(sleep_cycles)
+        for a, b in evs:
+            flush()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        per += [a.elapsed_time(b) for a, b in evs]
+    return per
 
 
 CHAIN_METRIC = "decoder-layer chain tokens/s (28 dependent layers; % of HBM roofline)"
@@ -248,18 +414,22 @@ def chain_bytes(shapes, M, dims=CHAIN_DIMS):
     return algo + layers * ew, codes
 
 
+def make_chain(api, torch, dev, shapes, weights, M, layers):
+    per_layer = [dict() for _ in range(layers)]
+    for (l, _, name, _, _), w in zip(shapes, weights):
+        per_layer[l][name] = w
+    hidden, kv, hd, inter = CHAIN_DIMS
+    return api.DecoderChain(per_layer, M, hidden, kv, hd, inter, dev)
+
+
 def run_chain(args, api, torch, dev, rank, world, dist, local):
     from ternary_weight_decoder_b200 import synth
     M = args.m
     if not 1 <= M <= 32:
         raise SystemExit("--chain runs decode token counts only (1..32)")
-    shapes, descs, _, x_all, y_all = build_workload(api, torch, dev, M, args.layers, rank)
-    layers = [dict() for _ in range(args.layers)]
-    for (l, _, name, _, _), d in zip(shapes, descs):
-        layers[l][name] = (d["packed"], d["wscale"])
-    del descs, x_all, y_all
-    hidden, kv, hd, inter = CHAIN_DIMS
-    chain = api.DecoderChain(layers, M, hidden, kv, hd, inter, dev)
+    shapes, weights = build_weights(api, torch, dev, args.layers)
+    chain = make_chain(api, torch, dev, shapes, weights, M, args.layers)
+    hidden = CHAIN_DIMS[0]
     h0_host = torch.from_numpy(synth.activations(rank_layer_seed(0, rank), 0, M, hidden)).pin_memory()
     h0 = h0_host.to(dev)
     stream = torch.cuda.current_stream()
@@ -277,19 +447,13 @@ def run_chain(args, api, torch, dev, rank, world, dist, local):
             dist.barrier()
         torch.cuda.synchronize()
 
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        barrier()
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        barrier()
+        ms, per = timed_steps(torch, stream, step, args.steps, barrier)
     api.check()
-    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    ms = max_over_ranks(ms, dist, dev)
     ms_per_step = ms / args.steps
     algo, codes = chain_bytes(shapes, M)
-    hbm, src = peaks()
+    hbm, _, src = peaks()
     achieved = algo / (ms_per_step / 1e3) / 1e9
 
     e2e = None
@@ -314,39 +478,47 @@ def run_chain(args, api, torch, dev, rank, world, dist, local):
         dist.destroy_process_group()
     if rank != 0:
         return
+    hidden, kv, hd, inter = CHAIN_DIMS
     print(json.dumps({
         "metric": CHAIN_METRIC, "value": job_value(M, world, args.steps, ms), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8xternary->int32, f32 in/out", "data": "synthetic",
+        "dtype": DTYPE, "data": "synthetic",
         "config": {"workload": f"decoder_chain_{args.layers}L_M{M}", "M": M,
                    "layers": args.layers, "hidden": hidden, "kv_dim": kv, "head_dim": hd,
                    "inter": inter, "parallelism": f"dp{world} (independent replicas)",
                    "l2": f"codes {codes / 1e6:.0f} MB > 126 MB L2; no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None,
-                     "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured"
-                     else "fallback 6650 GB/s",
-                     "algorithmic_bytes_per_step": algo, "weight_bytes_per_step": codes,
-                     "note": "step = all layers: per layer 4 sweeps + 4 element-wise launches"},
+                     "frac": achieved / hbm, "traffic": None, "peak_source": peak_source(src),
+                     "algorithmic_bytes_per_step": algo, "weight_bytes_per_step": codes},
+        "step_times": dist_summary(per),
         "cpu_baseline": None, "e2e": e2e,
         "gpu_launches": chain.launches * args.steps, "clocks": clk.summary(),
     }))
 
 
-def cpu_oracle_sample(M, budget_s=10.0, sample_layers=4, layers=28):
-    """Time the reference oracle, as it stands, on one host core: repeated
-    passes over the projections of the first `sample_layers` layers until
-    about budget_s of timed work; tokens/s is scaled to the full sweep by
-    weight count."""
+# ------------------------------------------------------------ oracle timing
+_ORACLE_CODES = {}
+
+
+def _oracle_sample(M, rows_cap, token_cap, budget_s, layers=28, sample_layers=1):
+    """Time the oracle, as it stands, on one host core over the first
+    `rows_cap` weight rows of each projection of the first `sample_layers`
+    layers and min(M, token_cap) token rows, repeated for about budget_s;
+    tokens/s of the full sweep extrapolated by weight count (and by tokens
+    when fewer than M were run)."""
     from oracle import oracle as orc
     from ternary_weight_decoder_b200 import synth
     shapes = synth.sweep_shapes(layers)
     total_w = sum(N * K for (_, _, _, N, K) in shapes)
+    toks = min(M, token_cap)
     sample = []
     for (l, p, name, N, K) in synth.sweep_shapes(min(sample_layers, layers)):
-        codes, mean = orc.ternarize(synth.weights(l, p, N, K))
-        sample.append((synth.activations(l, p, M, K), codes, mean))
+        r = min(rows_cap, N)
+        if (l, p) not in _ORACLE_CODES:   # the oracle's ternarisation, done once per run
+            _ORACLE_CODES[(l, p)] = orc.ternarize(synth.weights(l, p, N, K))
+        codes, mean = _ORACLE_CODES[(l, p)]
+        sample.append((synth.activations(l, p, toks, K), np.ascontiguousarray(codes[:r]), mean))
     sample_w = sum(c.size for _, c, _ in sample)
     timed, passes = 0.0, 0
     while timed < budget_s or passes == 0:
@@ -355,12 +527,20 @@ def cpu_oracle_sample(M, budget_s=10.0, sample_layers=4, layers=28):
             orc.ternary_linear(x, codes, mean)
         timed += time.perf_counter() - t0
         passes += 1
-    sweep_s = timed / passes * total_w / sample_w
+    sweep_s = timed / passes * (total_w / sample_w) * (M / toks)
+    desc = (f"{len(sample)} of {len(shapes)} projections, {'all rows' if rows_cap >= 8960 else f'first {rows_cap} rows each'} "
+            f"({sample_w / total_w:.4f} of the weights), {toks} of {M} tokens, {passes} passes, "
+            f"{timed:.1f} s timed; extrapolated to the full sweep by weight count"
+            + (" and token count" if toks < M else ""))
     return {"value": M / sweep_s, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": (f"{len(sample)} of {len(shapes)} projections (layers 0-"
-                       f"{min(sample_layers, layers) - 1}, {sample_w / total_w:.3f} of the "
-                       f"weights) at M={M}, {passes} passes, {timed:.1f} s timed, scaled to "
-                       f"the full sweep by weight count")}
+            "sample": desc, **cpu_info()}
+
+
+def cpu_oracle_sample(M, budget_s=10.0, sample_layers=4, layers=28):
+    """Headline CPU baseline: the oracle over all rows of the projections
+    of the first `sample_layers` layers at M tokens."""
+    return _oracle_sample(M, rows_cap=1 << 30, token_cap=M, budget_s=budget_s, layers=layers,
+                          sample_layers=sample_layers)
 
 
 def run_reference(args):
@@ -406,14 +586,159 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8xternary->int32, f32 in/out", "data": "synthetic",
+        "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
         "config": {"workload": f"decode_sweep_196x_M{M}", "M": M,
                    "projections": len(shapes)},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": samp},
+                         "sample": samp, **cpu_info()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }))
+
+
+# ------------------------------------------------------------ configs
+def measure_configs(args, api, torch, dev, rank, shapes, weights, descs_m1, want, cpu_ok):
+    """The benchmark definition's other workloads on the same weights."""
+    from ternary_weight_decoder_b200 import synth
+    hbm, int8_peak, src = peaks()
+    stream = torch.cuda.current_stream()
+    out = {}
+    csteps = max(3, min(args.steps, 200))
+    psteps = max(3, min(args.steps, 20))
+    cwarm = max(3, min(args.warmup, 10))
+
+    def barrier():
+        torch.cuda.synchronize()
+
+    flush_buf = None
+    if "1" in want or "2" in want:
+        flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_ctr = [0]
+
+    def flush():
+        flush_ctr[0] += 1
+        flush_buf.fill_(flush_ctr[0])
+
+    if "1" in want:
+        # layer 0's q projection, x ~ N(0, 1) without outliers
+        N = K = 1536
+        assert shapes[0][3:] == (N, K)
+        packed, wscale = weights[0]
+        x = torch.from_numpy(synth.activations(rank_layer_seed(0, rank), 0, 1, K,
+                                               outliers=False)).to(dev)
+        y = torch.empty((1, N), dtype=torch.float32, device=dev)
+        ws = torch.zeros(api.linear_workspace_bytes(1, N, K), dtype=torch.uint8, device=dev)
+
+        def one():
+            api.ternary_linear(x, packed, wscale, N, y=y, ws=ws)
+        for _ in range(cwarm):
+            one()
+        api.check()
+        per = cold_calls(torch, stream, one, max(32, min(args.steps, 512)), flush)
+        api.check()
+        s = dist_summary(per)
+        nbytes = N * K // 4 + K * 4 + N * 4
+        out["1_gemv_1536x1536_M1"] = {
+            "us_per_call": s, "algorithmic_bytes": nbytes,
+            "gbs_at_median": nbytes / (s["median_us"] * 1e-6) / 1e9,
+            "frac_hbm_at_median": nbytes / (s["median_us"] * 1e-6) / 1e9 / hbm,
+            "launches_per_call": 2, "l2": "flushed (256 MB written) before every call",
+            "note": "launch-latency bound: the 0.6 MB of work is 0.09 us of HBM time"}
+
+    if "2" in want:
+        layer0 = descs_m1[:7]
+        t1 = api.SweepTable(layer0, 1, device=dev)
+        for _ in range(cwarm):
+            api.decoder_projection_sweep(t1)
+        api.check()
+        per = cold_calls(torch, stream, lambda: api.decoder_projection_sweep(t1),
+                         max(32, min(args.steps, 512)), flush)
+        api.check()
+        s = dist_summary(per)
+        nbytes, _, _ = sweep_bytes(shapes[:7], 1)
+        out["2_layer_7proj_M1"] = {
+            "us_per_sweep": s, "us_per_matrix_median": s["median_us"] / 7,
+            "algorithmic_bytes": nbytes,
+            "frac_hbm_at_median": nbytes / (s["median_us"] * 1e-6) / 1e9 / hbm,
+            "launches_per_call": t1.launches, "l2": "flushed (256 MB written) before every call"}
+        del t1
+    del flush_buf
+
+    if "4" in want:
+        for M in DECODE_MS:
+            descs, _, x_all, y_all = decode_inputs(api, torch, dev, shapes, weights, M, rank)
+            table = api.SweepTable(descs, M, device=dev)
+            for _ in range(cwarm):
+                api.decoder_projection_sweep(table)
+            api.check()
+            ms, per = timed_steps(torch, stream, lambda: api.decoder_projection_sweep(table),
+                                  csteps, barrier)
+            api.check()
+            algo, codes, _ = sweep_bytes(shapes, M)
+            step_s = ms / csteps / 1e3
+            e = {"M": M, "tokens_per_s": M / step_s, "us_per_step": step_s * 1e6,
+                 "step_times": dist_summary(per), "algorithmic_bytes": algo,
+                 "achieved_gbs": algo / step_s / 1e9, "frac_hbm": algo / step_s / 1e9 / hbm,
+                 "weight_gbs": codes / step_s / 1e9, "launches_per_step": table.launches,
+                 "dominant_kernel_src": decode_kernel_src(M),
+                 "traffic": profiled_traffic(decode_kernel_src(M), M, args.layers)}
+            if cpu_ok:
+                e["oracle"] = _oracle_sample(M, rows_cap=512, token_cap=M, budget_s=2.5,
+                                             layers=args.layers)
+            out[f"4_decode_sweep_196x_M{M}"] = e
+            del table, descs, x_all, y_all
+            torch.cuda.empty_cache()
+
+    if "5" in want:
+        for M in PREFILL_MS:
+            descs = prefill_inputs(api, torch, dev, shapes, weights, M, rank)
+            table = api.SweepTable(descs, M, device=dev)
+            for _ in range(cwarm):
+                api.decoder_projection_sweep(table)
+            api.check()
+            ms, per = timed_steps(torch, stream, lambda: api.decoder_projection_sweep(table),
+                                  psteps, barrier)
+            api.check()
+            step_s = ms / psteps / 1e3
+            ops = sweep_ops(shapes, M)
+            e = {"M": M, "tokens_per_s": M / step_s, "us_per_step": step_s * 1e6,
+                 "step_times": dist_summary(per), "int8_ops": ops,
+                 "achieved_tops": ops / step_s / 1e12, "peak_tops": int8_peak,
+                 "frac_int8": ops / step_s / 1e12 / int8_peak,
+                 "launches_per_step": table.launches,
+                 "inputs": f"{min(M, PREFILL_DISTINCT_ROWS)} distinct seeded token rows per "
+                           f"projection tiled to {M}, quantised before the timed region",
+                 "traffic": profiled_traffic("tw_prefill.cu", M, args.layers)}
+            if cpu_ok:
+                e["oracle"] = _oracle_sample(M, rows_cap=64, token_cap=256, budget_s=3.0,
+                                             layers=args.layers)
+            out[f"5_prefill_sweep_196x_M{M}"] = e
+            del table, descs
+            torch.cuda.empty_cache()
+
+    if "chain" in want:
+        M = 1
+        chain = make_chain(api, torch, dev, shapes, weights, M, args.layers)
+        h0 = torch.from_numpy(synth.activations(rank_layer_seed(0, rank), 0, M,
+                                                CHAIN_DIMS[0])).to(dev)
+
+        def cstep():
+            chain.h.copy_(h0, non_blocking=True)
+            api.decoder_chain(chain)
+        for _ in range(cwarm):
+            cstep()
+        api.check()
+        ms, per = timed_steps(torch, stream, cstep, csteps, barrier)
+        api.check()
+        algo, codes = chain_bytes(shapes, M)
+        step_s = ms / csteps / 1e3
+        out["chain_28L_M1"] = {
+            "M": M, "tokens_per_s": M / step_s, "us_per_step": step_s * 1e6,
+            "step_times": dist_summary(per), "algorithmic_bytes": algo,
+            "frac_hbm": algo / step_s / 1e9 / hbm, "launches_per_step": chain.launches + 1,
+            "note": "28 dependent layers from one token state (the +1 launch copies it in)"}
+        del chain
+    return out
 
 
 def main():
@@ -440,10 +765,14 @@ def main():
     if args.chain:
         return run_chain(args, api, torch, dev, rank, world, dist, local)
     M = args.m
-    shapes, descs, x_host, x_all, y_all = build_workload(api, torch, dev, M, args.layers, rank)
-    if M > 32:   # prefill sweeps consume int8 activations quantised beforehand
-        for d in descs:
-            d["xq"], d["amax"], d["qsum"] = api.quantize_act(d["x"])
+    shapes, weights = build_weights(api, torch, dev, args.layers)
+    if M > 32:
+        descs = prefill_inputs(api, torch, dev, shapes, weights, M, rank)
+        x_host = x_all = None
+        y_all = None
+    else:
+        descs, x_host, x_all, y_all = decode_inputs(api, torch, dev, shapes, weights, M, rank,
+                                                    with_host=True)
     table = api.SweepTable(descs, M, device=dev)
     algo_bytes, algo_codes, _ = sweep_bytes(shapes, M)
     launches_per_step = table.launches
@@ -458,45 +787,34 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        barrier()
-        e0.record(stream)
-        for _ in range(args.steps):
-            api.decoder_projection_sweep(table)
-        e1.record(stream)
-        barrier()
+        ms, per = timed_steps(torch, stream, lambda: api.decoder_projection_sweep(table),
+                              args.steps, barrier)
     api.check()
-    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    ms = max_over_ranks(ms, dist, dev)
     ms_per_step = ms / args.steps
     value = job_value(M, world, args.steps, ms)
 
-    hbm, src = peaks()
+    hbm, int8_peak, src = peaks()
     if M <= 32:
         # decode: HBM-bound; algorithmic bytes = 2-bit codes + fp32 x + fp32 y
         achieved = algo_bytes / (ms_per_step / 1e3) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                     "frac": achieved / hbm,
-                    # sweeps of more than 16 tokens run the tensor-core decode kernel
-                    "traffic": profiled_traffic("tw_decode_tc.cu" if M > 16 else "tw_decode.cu",
-                                                M, args.layers),
-                    "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured"
-                    else "fallback 6650 GB/s",
+                    "traffic": profiled_traffic(decode_kernel_src(M), M, args.layers),
+                    "peak_source": peak_source(src),
                     "algorithmic_bytes_per_step": algo_bytes,
                     "weight_bytes_per_step": algo_codes,
                     "weight_gbs": algo_codes / (ms_per_step / 1e3) / 1e9,
                     "note": "step = quantise launch + decode launch; time of the whole step"}
     else:
         # prefill: int8 tensor-core bound; 2*M*N*K ops per projection
-        ops = sum(2 * M * N * K for (_, _, _, N, K) in shapes)
+        ops = sweep_ops(shapes, M)
         tops = ops / (ms_per_step / 1e3) / 1e12
-        pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))).get("bf16_tflops") \
-            if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else FALLBACK_BF16_TFLOPS
-        roofline = {"bound": "tensor", "achieved": tops, "peak": 2 * pk, "unit": "TOP/s",
-                    "frac": tops / (2 * pk),
+        roofline = {"bound": "tensor", "achieved": tops, "peak": int8_peak, "unit": "TOP/s",
+                    "frac": tops / int8_peak,
                     "traffic": profiled_traffic("tw_prefill.cu", M, args.layers),
-                    "peak_source": "2 x measured bf16 burst (int8 dense = 2 x bf16 nominal)",
-                    "ops_per_step": ops}
+                    "peak_source": peak_source(src), "ops_per_step": ops}
 
     e2e = None
     if not args.no_e2e and M <= 32:
@@ -524,28 +842,40 @@ def main():
                "h2d_bytes_per_step": x_all.numel() * 4, "d2h_bytes_per_step": y_all.numel() * 4,
                "steps": k2, "ms_per_step": ems / k2, "host_wall_ms_per_step": wall * 1e3 / k2}
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_oracle_sample(M, layers=args.layers)
+    cpu_ok = rank == 0 and world == 1 and not args.no_cpu
+    cpu = cpu_oracle_sample(M, layers=args.layers) if cpu_ok and M <= 32 else None
+
+    configs, cclk = None, None
+    if not args.no_configs and M == 1 and args.layers == 28:
+        want = set(w.strip() for w in args.configs.split(",") if w.strip())
+        del table
+        with ClockSampler(local) as cs:
+            configs = measure_configs(args, api, torch, dev, rank, shapes, weights, descs,
+                                      want, cpu_ok)
+        cclk = cs.summary()
 
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return
-    print(json.dumps({
+    line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8xternary->int32, f32 in/out", "data": "synthetic",
-        "config": {"workload": f"decode_sweep_196x_M{M}" if args.layers == 28
-                   else f"decode_sweep_{7 * args.layers}x_M{M}",
+        "scaling": "weak", "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
+        "config": {"workload": (f"decode_sweep_196x_M{M}" if args.layers == 28
+                                else f"decode_sweep_{7 * args.layers}x_M{M}") if M <= 32
+                   else f"prefill_sweep_{7 * args.layers}x_M{M}",
                    "M": M, "projections": len(shapes), "layers": args.layers,
                    "parallelism": f"dp{world} (independent replicas, no collective)",
                    "l2": f"inputs {algo_bytes / 1e6:.0f} MB > 126 MB L2; no flush"},
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "roofline": roofline, "step_times": dist_summary(per), "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
-    }))
+    }
+    if configs is not None:
+        line["configs"] = configs
+        line["configs_clocks"] = cclk
+    print(json.dumps(line))
 
 
 if __name__ == "__main__":

@@ -6,6 +6,7 @@
 #include <cstring>
 #include <algorithm>
 #include <mutex>
+#include <cuda.h>
 
 #include "tw_device.cuh"
 #include "tw_internal.h"
@@ -33,33 +34,63 @@ int cuda_fail(cudaError_t e, const char *what)
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Address of g_tw_err on the current device (looked up once per device).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// Id of the calling thread's current CUDA context, or 0 when there is none
+// (or the driver cannot say).  Context ids are unique for the life of the
+// process, so a context created after cudaDeviceReset gets a new one.
+unsigned long long current_context_id()
+{
+    static CtxGetCurrentFn get_cur = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess && f)
+            get_cur = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess && f)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+    });
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (!get_cur || !get_id || get_cur(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Address of g_tw_err on the current device.  Looked up once per device and
+// context: a device reset (a new context) makes the lookup run again.
 int err_word(uint32_t **out)
 {
-    static std::mutex mu;
-    static uint32_t *cache[64] = {};
+    static tw::SymbolCache cache;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaGetDevice");
-    if (dev < 0 || dev >= 64)
+    if (dev < 0 || dev >= tw::SymbolCache::kDevices)
         return fail(TW_ERR_UNSUPPORTED, "device index %d out of range", dev);
-    std::lock_guard<std::mutex> lk(mu);
-    if (!cache[dev]) {
-        int major = 0;
-        e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "cudaDeviceGetAttribute");
-        if (major != 10)
-            return fail(TW_ERR_UNSUPPORTED, "device %d is sm_%d0, this library is built for sm_100a",
-                        dev, major);
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_tw_err);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "cudaGetSymbolAddress(error word)");
-        cache[dev] = static_cast<uint32_t *>(p);
+    {
+        std::lock_guard<std::mutex> lk(cache.mu);
+        if (!cache.addr[dev]) {   // first use of this device: check what it is
+            int major = 0;
+            e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "cudaDeviceGetAttribute");
+            if (major != 10)
+                return fail(TW_ERR_UNSUPPORTED,
+                            "device %d is sm_%d0, this library is built for sm_100a", dev, major);
+        }
     }
-    *out = cache[dev];
+    void *p = nullptr;
+    if (int rc = tw::symbol_address(reinterpret_cast<const void *>(&g_tw_err), cache,
+                                    "the error word", &p))
+        return rc;
+    *out = static_cast<uint32_t *>(p);
     return TW_OK;
 }
 
@@ -120,7 +151,36 @@ struct ChainStage {
     const float *y[3];    // required y per projection (null: any)
 };
 
-int check_chain_stage(const void *host, const void *dev, const ChainStage &st, int64_t M, int layer)
+// The nine chain buffers as byte ranges.
+struct ChainRange {
+    const char *name;
+    uintptr_t lo, hi;
+};
+
+void chain_ranges(const tw_chain_buffers &b, ChainRange r[9])
+{
+    const int64_t f = 4 * b.M;
+    const struct { const char *n; const float *p; int64_t w; } bufs[9] = {
+        {"h", b.h, b.hidden}, {"v", b.v, b.kv_dim}, {"a", b.a, b.hidden},
+        {"o", b.o, b.hidden}, {"h1", b.h1, b.hidden}, {"g", b.g, b.inter},
+        {"u", b.u, b.inter}, {"act", b.act, b.inter}, {"d", b.d, b.hidden}};
+    for (int i = 0; i < 9; ++i) {
+        const uintptr_t lo = reinterpret_cast<uintptr_t>(bufs[i].p);
+        r[i] = ChainRange{bufs[i].n, lo, lo + (uintptr_t)(f * bufs[i].w)};
+    }
+}
+
+// Name of the first chain buffer that [lo, hi) overlaps, or null.
+const char *overlaps_chain(uintptr_t lo, uintptr_t hi, const ChainRange r[9])
+{
+    for (int i = 0; i < 9; ++i)
+        if (lo < r[i].hi && r[i].lo < hi)
+            return r[i].name;
+    return nullptr;
+}
+
+int check_chain_stage(const void *host, const void *dev, const ChainStage &st, int64_t M, int layer,
+                      const ChainRange ranges[9])
 {
     if (!host || !dev)
         return fail(TW_ERR_NULL, "chain layer %d: %s table missing", layer, st.name);
@@ -147,6 +207,19 @@ int check_chain_stage(const void *host, const void *dev, const ChainStage &st, i
         if (st.y[i] && r[i].y != st.y[i])
             return fail(TW_ERR_SHAPE, "chain layer %d: %s projection %d does not write its chain "
                         "output buffer", layer, st.name, i);
+        // An output that is not the projection's own chain buffer must lie
+        // outside all of them: the chain reads those while the sweep writes.
+        const uintptr_t bytes = (uintptr_t)(4 * M * r[i].N);
+        const uintptr_t ylo = reinterpret_cast<uintptr_t>(r[i].y);
+        if (!st.y[i])
+            if (const char *hit = overlaps_chain(ylo, ylo + bytes, ranges))
+                return fail(TW_ERR_SHAPE, "chain layer %d: %s projection %d writes into chain "
+                            "buffer %s", layer, st.name, i, hit);
+        const uintptr_t alo = reinterpret_cast<uintptr_t>(r[i].acc_out);
+        if (r[i].acc_out)
+            if (const char *hit = overlaps_chain(alo, alo + bytes, ranges))
+                return fail(TW_ERR_SHAPE, "chain layer %d: %s projection %d has its integer "
+                            "outputs in chain buffer %s", layer, st.name, i, hit);
     }
     return TW_OK;
 }
@@ -189,6 +262,13 @@ int check_chain_buffers(const tw_chain_buffers *b)
         (b->hidden / b->head_dim) % (b->kv_dim / b->head_dim))
         return fail(TW_ERR_SHAPE, "tw_decoder_chain: hidden and kv_dim must be whole heads of "
                     "head_dim, the query heads an equal number per KV head");
+    ChainRange r[9];
+    chain_ranges(*b, r);
+    for (int i = 0; i < 9; ++i)
+        for (int j = i + 1; j < 9; ++j)
+            if (r[i].lo < r[j].hi && r[j].lo < r[i].hi)
+                return fail(TW_ERR_SHAPE, "tw_decoder_chain: chain buffers %s and %s overlap",
+                            r[i].name, r[j].name);
     return TW_OK;
 }
 
@@ -197,6 +277,30 @@ int check_chain_buffers(const tw_chain_buffers *b)
 namespace tw {
 int error_word(uint32_t **out) { return err_word(out); }
 int record_error(int code, const char *msg) { return fail(code, "%s", msg); }
+void clear_error() { t_last_error[0] = 0; }
+
+int symbol_address(const void *symbol, SymbolCache &c, const char *what, void **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= SymbolCache::kDevices)
+        return fail(TW_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    const unsigned long long id = current_context_id();
+    std::lock_guard<std::mutex> lk(c.mu);
+    if (!c.addr[dev] || id == 0 || c.ctx[dev] != id) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, symbol);
+        if (e != cudaSuccess || !p)
+            return fail(TW_ERR_CUDA, "cudaGetSymbolAddress(%s): %s", what,
+                        e != cudaSuccess ? cudaGetErrorString(e) : "null address");
+        c.addr[dev] = p;
+        c.ctx[dev] = id ? id : current_context_id();   // the lookup made a context current
+    }
+    *out = c.addr[dev];
+    return TW_OK;
+}
 }  // namespace tw
 
 extern "C" {
@@ -657,12 +761,14 @@ int tw_decoder_chain(const tw_chain_layer *layers, int n_layers, const tw_chain_
     const tw_chain_buffers &b = *buf;
     ChainStage st[4];
     chain_stages(b, st);
+    ChainRange ranges[9];
+    chain_ranges(b, ranges);
     // Every table is checked before anything is launched.
     for (int l = 0; l < n_layers; ++l) {
         const void *host[4], *dev[4];
         layer_tables(layers[l], host, dev);
         for (int s = 0; s < 4; ++s)
-            if (int rc = check_chain_stage(host[s], dev[s], st[s], b.M, l))
+            if (int rc = check_chain_stage(host[s], dev[s], st[s], b.M, l, ranges))
                 return rc;
     }
     const size_t need = tw_chain_workspace_bytes(layers, n_layers);

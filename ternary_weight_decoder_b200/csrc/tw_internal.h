@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "../../include/ternary_decoder.h"
@@ -166,5 +167,22 @@ cudaError_t launch_wait_probe(uint32_t *err, uint64_t timeout_ns, cudaStream_t s
 int error_word(uint32_t **out);
 // Record a message for tw_last_error() and return `code`.
 int record_error(int code, const char *msg);
+// Clear this host thread's last-error message (every entry point does so
+// first).
+void clear_error();
+
+// Device addresses of a __device__ variable, one per device, each valid
+// for the context it was looked up in (re-resolved when the current
+// context's id changes, as after cudaDeviceReset).
+struct SymbolCache {
+    static constexpr int kDevices = 64;
+    std::mutex mu;
+    void *addr[kDevices] = {};
+    unsigned long long ctx[kDevices] = {};
+};
+// `symbol` is the address of the __device__ variable as host code sees it
+// (a host-side stand-in); *out receives its device address on the current
+// device.  `what` names it in the error message.
+int symbol_address(const void *symbol, SymbolCache &cache, const char *what, void **out);
 
 }  // namespace tw

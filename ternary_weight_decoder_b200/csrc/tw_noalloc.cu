@@ -26,28 +26,13 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 // Device address of g_noalloc_scratch for the current device.  Host code
 // must not pass the symbol itself to a kernel: on the host it names a
-// stand-in object, not device memory.  Looked up once per device.
+// stand-in object, not device memory.  Looked up once per device and
+// context (again after a device reset, which creates a new context).
 int scratch_address(void **out)
 {
-    static std::mutex mu;
-    static void *cache[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return tw::record_error(TW_ERR_CUDA, "cudaGetDevice failed");
-    if (dev < 0 || dev >= 64)
-        return tw::record_error(TW_ERR_UNSUPPORTED, "device index out of range");
-    std::lock_guard<std::mutex> lk(mu);
-    if (!cache[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess || !p)
-            return tw::record_error(TW_ERR_CUDA,
-                                    "cudaGetSymbolAddress(no-alloc scratch) failed");
-        cache[dev] = p;
-    }
-    *out = cache[dev];
-    return TW_OK;
+    static tw::SymbolCache cache;
+    return tw::symbol_address(reinterpret_cast<const void *>(&g_noalloc_scratch), cache,
+                              "no-alloc scratch", out);
 }
 
 }  // namespace
@@ -57,6 +42,7 @@ extern "C" TW_API int tw_ternarize_pack_noalloc(const float *W, int64_t N, int64
                                                 double *mean_abs, float *wscale,
                                                 tw_stream_t stream)
 {
+    tw::clear_error();
     if (!W || !packed || !wscale)
         return tw::record_error(TW_ERR_NULL,
                                 "tw_ternarize_pack_noalloc: W, packed and wscale are required");

@@ -150,6 +150,14 @@ def test_layout_spec_round_trip():
         assert dec == c[0, :16].tolist()
 
 
+def test_layout_spec_fast_pack_matches_the_statement():
+    """pack_fast (used at full size) writes the same bytes as pack."""
+    rng = np.random.default_rng(1)
+    for N, K in [(16, 128), (37, 256), (5, 384), (1, 128), (48, 1152)]:
+        c = rng.integers(-1, 2, (N, K)).astype(np.int8)
+        assert (layout_spec.pack_fast(c) == layout_spec.pack(c)).all(), (N, K)
+
+
 QWEN_LAYER = [(1536, 1536), (256, 1536), (256, 1536), (1536, 1536),
               (8960, 1536), (8960, 1536), (1536, 8960)]
 
@@ -179,12 +187,15 @@ def test_sweep_launch_count_196(lib, M):
 CHAIN_BUFS = ("h", "v", "a", "o", "h1", "g", "u", "act", "d")
 
 
+CHAIN_ADDR = {n: 0x7f0000000000 + 0x100000 * i for i, n in enumerate(CHAIN_BUFS + ("q", "k"))}
+
+
 def _fake_chain(M=1, hidden=256, kv=128, hd=128, inter=512, n_layers=2, tweak=None):
     """Encoded tables of a chain over placeholder device addresses (nothing
     is launched): per layer qkv, o, gate/up and down, as the chain wants
     them unless `tweak(layer, stage, descs)` changes the descriptors."""
     from ternary_weight_decoder_b200 import api
-    addr = {n: 0x7f0000000000 + 0x100000 * i for i, n in enumerate(CHAIN_BUFS + ("q", "k"))}
+    addr = CHAIN_ADDR
     stages = {"qkv": [("h", "q", hidden, hidden), ("h", "k", kv, hidden), ("h", "v", kv, hidden)],
               "o": [("a", "o", hidden, hidden)],
               "gu": [("h1", "g", inter, hidden), ("h1", "u", inter, hidden)],
@@ -242,7 +253,9 @@ def _tw(arr, i, **kw):
 
 @pytest.mark.parametrize("case,status", [
     ("o_reads_wrong_buffer", 2), ("v_writes_wrong_buffer", 2), ("down_wrong_K", 2),
-    ("gate_wrong_N", 2), ("qkv_two_projections", 2), ("table_other_M", 2)])
+    ("gate_wrong_N", 2), ("qkv_two_projections", 2), ("table_other_M", 2),
+    ("q_writes_into_h", 2), ("k_writes_into_a", 2), ("acc_out_in_h1", 2),
+    ("acc_out_in_act", 2)])
 def test_chain_rejects_mismatched_tables(lib, case, status):
     from ternary_weight_decoder_b200 import api
     import ctypes
@@ -252,6 +265,11 @@ def test_chain_rejects_mismatched_tables(lib, case, status):
         "v_writes_wrong_buffer": lambda l, st, a: st == "qkv" and _tw(a, 2, y=a[2].y + 0x100000),
         "down_wrong_K": lambda l, st, a: st == "down" and _tw(a, 0, K=256),
         "gate_wrong_N": lambda l, st, a: st == "gu" and _tw(a, 0, N=384),
+        # q's output inside h: the sweep would overwrite h while k and v read it
+        "q_writes_into_h": lambda l, st, a: st == "qkv" and _tw(a, 0, y=CHAIN_ADDR["h"] + 256),
+        "k_writes_into_a": lambda l, st, a: st == "qkv" and _tw(a, 1, y=CHAIN_ADDR["a"]),
+        "acc_out_in_h1": lambda l, st, a: st == "o" and _tw(a, 0, acc_out=CHAIN_ADDR["h1"]),
+        "acc_out_in_act": lambda l, st, a: st == "gu" and l == 1 and _tw(a, 1, acc_out=CHAIN_ADDR["act"] + 512),
     }
     if case in tweaks:
         layers, cbuf, keep = _fake_chain(tweak=tweaks[case])
@@ -270,7 +288,8 @@ def test_chain_rejects_mismatched_tables(lib, case, status):
 
 @pytest.mark.parametrize("field,value,status", [
     ("h", None, 1), ("act", 0x7f0000000008, 3), ("M", 33, 2), ("M", 0, 2),
-    ("hidden", 200, 2), ("head_dim", 96, 2), ("kv_dim", 384, 2)])
+    ("hidden", 200, 2), ("head_dim", 96, 2), ("kv_dim", 384, 2),
+    ("h1", CHAIN_ADDR["h"] + 512, 2), ("d", CHAIN_ADDR["act"], 2)])
 def test_chain_rejects_bad_buffers(lib, field, value, status):
     from ternary_weight_decoder_b200 import api
     import ctypes

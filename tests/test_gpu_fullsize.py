@@ -3,11 +3,14 @@ times: the 196-projection decode sweep (M = 1 and M = 4, 8, 16, 32) and the
 196-projection prefill sweep (M = 256, 1024, 4096), checked on sampled
 outputs against the oracle.
 
-Every projection is ternarised on the GPU and its mean|W| and scale checked
-bit-exact against the oracle over the whole matrix; then for a seeded sample
-of weight rows (and, for prefill, of token rows) the oracle recomputes the
-codes, activations and accumulators one by one: accumulators bit-exact,
-outputs within 1e-6 relative.
+Every projection is ternarised on the GPU; its packed bytes (the whole
+matrix, all 196 of them), mean|W| and scale are compared bit for bit with
+the oracle's codes laid out by the layout statement in tests/layout_spec.py.
+Then for a seeded sample of 64 weight rows per projection (and, for prefill,
+16 token rows including the first and last 128-token tile) the oracle
+recomputes the activations and accumulators one by one: accumulators
+bit-exact, outputs within 1e-6 relative.  Every output of every projection
+is poisoned before the call and checked to have been written.
 """
 import concurrent.futures as cf
 import os
@@ -17,17 +20,20 @@ import pytest
 
 from oracle import oracle as orc
 from tests import gpu_util as G
+from tests import layout_spec
 from ternary_weight_decoder_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-ROWS_PER_PROJ = 8
+ROWS_PER_PROJ = 64
+TOKENS_PER_PREFILL = 16
 
 
 @pytest.fixture(scope="module")
 def model():
-    """All 196 projections ternarised on the GPU, with oracle references for
-    a seeded sample of rows of each."""
+    """All 196 projections ternarised on the GPU, each compared whole with
+    the oracle (packed bytes, mean, scale), with oracle codes kept for a
+    seeded sample of rows of each."""
     dev = G.torch_dev()
     api = G.api()
     shapes = synth.sweep_shapes()
@@ -43,6 +49,11 @@ def model():
         W = futs.pop(i).result()
         packed, mean_abs, wscale = api.ternarize_pack(G.to_dev(W, dev))
         codes, mean = orc.ternarize(W)
+        want = layout_spec.pack_fast(codes)
+        got = packed.cpu().numpy()
+        assert got.size >= want.size and (got[:want.size] == want).all(), \
+            f"packed codes of L{l}.{name} ({N}x{K}) differ from the oracle's"
+        del want, got
         rows = np.sort(rng.choice(N, size=min(ROWS_PER_PROJ, N), replace=False))
         projs.append(dict(l=l, p=p, name=name, N=N, K=K, packed=packed, mean_abs=mean_abs,
                           wscale=wscale, mean=mean, rows=rows, codes=codes[rows].copy()))
@@ -94,7 +105,11 @@ def test_prefill_sweep_full_size(model, M):
         xd = G.to_dev(x, dev)
         xq, amax, qsum = api.quantize_act(xd)
         del xd
-        toks = np.sort(rng.choice(M, size=6, replace=False))
+        # the first and last token of the first and last 128-token tile, the
+        # rest seeded
+        fixed = {0, 1, M - 1, M - 2, (M - 1) // 128 * 128}
+        rest = [t for t in rng.permutation(M) if t not in fixed]
+        toks = np.sort(np.array(sorted(fixed) + rest[:TOKENS_PER_PREFILL - len(fixed)]))
         keep.append((toks, x[toks].copy()))
         descs.append(dict(xq=xq, amax=amax, qsum=qsum, packed=d["packed"],
                           wscale=d["wscale"],

@@ -170,7 +170,8 @@ def test_decode_k_permutation_detector(dev, api):
 @pytest.mark.parametrize("M,N,K", [(33, 80, 640), (128, 256, 128), (129, 257, 256),
                                    (255, 1536, 1536), (256, 1536, 1536), (257, 300, 1152),
                                    (1024, 256, 1536), (300, 8960, 1536), (64, 1536, 8960),
-                                   (40, 1, 128), (200, 30, 384)])
+                                   (40, 1, 128), (200, 30, 384), (1023, 1536, 1536),
+                                   (4095, 300, 1536)])
 def test_prefill_linear_shapes(dev, api, M, N, K):
     W = _weights(N, K, 7 * M + N + K)
     x = _acts(M, K, 11 * M + K)

@@ -45,3 +45,7 @@ def test_noalloc_rejects_rows_beyond_its_scratch():
     with pytest.raises(api.TernaryError) as e:
         api.ternarize_pack_noalloc(W)
     assert e.value.status == 2 and "TW_NOALLOC_MAX_N" in str(e.value)
+    # a successful call after the failure leaves no stale message behind
+    api.ternarize_pack_noalloc(W[:16].contiguous())
+    assert api.tw_last_error() == b""
+    api.check()
