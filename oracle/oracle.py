@@ -52,6 +52,10 @@ def _bind(lib):
     lib.orc_add_f32.argtypes = [p, p, i64, p]
     lib.orc_silu_mul.restype = None
     lib.orc_silu_mul.argtypes = [p, p, i64, p]
+    lib.orc_i8_quantize_weights.restype = None
+    lib.orc_i8_quantize_weights.argtypes = [p, i64, i64, p, p]
+    lib.orc_i8_epilogue.restype = None
+    lib.orc_i8_epilogue.argtypes = [p, i64, i64, p, ctypes.c_float, p, ctypes.c_int, p]
     return lib
 
 
@@ -202,3 +206,37 @@ def decoder_layer(h, layer, head_dim: int = 128):
     d = proj(act, "down")
     return {"q": q, "k": k, "v": v, "a": a, "o": o, "h1": h1, "g": g, "u": u,
             "act": act, "d": d, "h_next": add_f32(h1, d)}
+
+
+# ------------------------------------------------ I8_S linear (R17-R19)
+def i8_quantize_weights(W):
+    """R17: (wq int8 [N,K], amax_w float32) -- one absmax scale per tensor."""
+    W, pw = _c(W, np.float32)
+    N, K = W.shape
+    wq = np.empty((N, K), np.int8)
+    amax = np.empty(1, np.float32)
+    _load().orc_i8_quantize_weights(pw, N, K, wq.ctypes.data, amax.ctypes.data)
+    return wq, np.float32(amax[0])
+
+
+def i8_epilogue(acc, amax_x, amax_w, bias=None, relu=True):
+    """R19: y float64 [M,N] = relu?(acc * amax_x/127 * amax_w/127 + bias)."""
+    acc, pa = _c(acc, np.int32)
+    amax_x, px = _c(amax_x, np.float32)
+    M, N = acc.shape
+    pb = None
+    if bias is not None:
+        bias, pb = _c(bias, np.float32)
+        assert bias.shape == (N,)
+    y = np.empty((M, N), np.float64)
+    _load().orc_i8_epilogue(pa, M, N, px, float(amax_w), pb, int(bool(relu)), y.ctypes.data)
+    return y
+
+
+def i8_linear(x, wq, amax_w, bias=None, relu=True):
+    """The I8_S layer on quantised weights: quantise x per token (R18),
+    int8 dot products (exact), rescale + bias + ReLU.  dict(q, amax, acc, y)."""
+    q, amax = quantize_act(x)
+    acc = ternary_acc(wq, q)       # an exact int8 dot product for any int8 weights
+    y = i8_epilogue(acc, amax, amax_w, bias, relu)
+    return {"q": q, "amax": amax, "acc": acc, "y": y}

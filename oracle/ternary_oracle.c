@@ -207,3 +207,51 @@ void orc_silu_mul(const float *g, const float *u, int64_t n, double *out)
         out[i] = z / (1.0 + exp(-z)) * (double)u[i];
     }
 }
+
+/* ------------------------------------------------------------------------
+ * I8_S linear with fused bias and ReLU: the int8 side of the model.
+ *
+ * The audio encoder (VAE tokenizer) keeps int8 weights and int8 activations
+ * and replaces GELU by ReLU ("VibeVoice-ASR-BitNet-ONNX" model page,
+ * "Quantization" table, row "VAE encoders": I8_S); its fused int8 routines
+ * join matmul, bias and ReLU in one pass (aitrends summary, technical
+ * features); it is bound by data movement, activations outweighing weights
+ * 16 to 1 ("The Paper Says ARM Support" post, "What the model is trying to
+ * do").  The pages fix neither the weight scale's granularity nor the
+ * rounding; readings taken here:
+ *   R17 I8_S weights carry one scale per tensor (the "_S" format of the
+ *       ternary weights is per tensor too, and the ONNX page contrasts its
+ *       own per-channel int8 weights with it): wq = the absmax int8
+ *       quantisation of the whole tensor, the same rule as R4 applied to W
+ *       as one row, amax_w = max|W|.
+ *   R18 activations are quantised per token as in R4.
+ *   R19 y = acc * (amax_x/127) * (amax_w/127) + bias, then ReLU when asked
+ *       (max(0, y)); evaluated here in fp64.  A missing bias is zero.
+ * ---------------------------------------------------------------------- */
+
+/* R17: wq [N x K] and amax_w of W [N x K]. */
+void orc_i8_quantize_weights(const float *W, int64_t N, int64_t K, int8_t *wq,
+                             float *amax_w)
+{
+    orc_quantize_act(W, 1, N * K, wq, amax_w);
+}
+
+/* R19: y[m*N+n] from the exact accumulators (orc_ternary_acc computes the
+ * int8 dot products for any int8 weights). */
+void orc_i8_epilogue(const int32_t *acc, int64_t M, int64_t N,
+                     const float *amax_x, float amax_w, const float *bias,
+                     int relu, double *y)
+{
+    const double w = (double)amax_w / 127.0;
+    for (int64_t m = 0; m < M; ++m) {
+        const double a = (double)amax_x[m] / 127.0;
+        for (int64_t n = 0; n < N; ++n) {
+            double v = (double)acc[m * N + n] * a * w;
+            if (bias)
+                v += (double)bias[n];
+            if (relu && v < 0.0)
+                v = 0.0;
+            y[m * N + n] = v;
+        }
+    }
+}

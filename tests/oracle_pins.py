@@ -391,5 +391,108 @@ def pin_decoder_layer_attention_reads_v():
     assert not np.array_equal(with_v["h1"], h)
 
 
+# ------------------------------------------------ I8_S linear (R17-R19)
+def pin_i8_hand_3x8():
+    """Hand-worked I8_S case: ties pin half-even for weights and tokens, the
+    dyadic scales pin both /127 factors, the bias signs pin ReLU."""
+    g = _golden("hand_i8_3x8.json")
+    W = (np.array(g["W128"], np.float64) / 128.0).astype(np.float32)
+    wq, amax_w = orc.i8_quantize_weights(W)
+    assert float(amax_w) == g["amax_w"], amax_w
+    assert wq.tolist() == g["wq"], wq
+    assert wq.tolist() != g["wq_half_away"]
+    x = np.array(g["x"], np.float32)
+    bias = np.array(g["bias"], np.float32)
+    out = orc.i8_linear(x, wq, amax_w, bias, relu=True)
+    assert out["amax"].tolist() == g["amax_x"]
+    assert out["q"].tolist() == g["q"], out["q"]
+    assert out["acc"].tolist() == g["acc"], out["acc"]
+    assert out["y"].tolist() == g["y_relu"], out["y"]
+    lin = orc.i8_linear(x, wq, amax_w, bias, relu=False)
+    assert lin["y"].tolist() == g["y_linear"], lin["y"]
+
+
+def pin_i8_weight_quant_is_the_fp32_rule():
+    """wq = half-even(fl(W * fl(127 / max|W|))) with IEEE fp32 operations
+    (numpy's float32 arithmetic and rint), amax_w = max|W| exactly; |wq| <= 127."""
+    rng = np.random.default_rng(17)
+    for shape in [(7, 40), (1, 128), (33, 96)]:
+        W = (rng.standard_normal(shape) * 0.05).astype(np.float32)
+        W[rng.integers(shape[0]), rng.integers(shape[1])] = -0.25   # the extreme is negative
+        wq, amax_w = orc.i8_quantize_weights(W)
+        a = np.float32(np.abs(W).max())
+        assert amax_w == a
+        scale = np.float32(127.0) / a
+        want = np.clip(np.rint(W * scale), -128, 127).astype(np.int8)
+        assert (wq == want).all()
+        assert np.abs(wq.astype(np.int32)).max() == 127
+
+
+def pin_i8_acc_numpy_matmul():
+    """acc of full-range int8 weights and tokens equals numpy's int64 matmul."""
+    rng = np.random.default_rng(18)
+    wq = rng.integers(-127, 128, (9, 200)).astype(np.int8)
+    q = rng.integers(-128, 128, (5, 200)).astype(np.int8)
+    acc = orc.ternary_acc(wq, q)
+    assert (acc == q.astype(np.int64) @ wq.astype(np.int64).T).all()
+
+
+def pin_i8_epilogue_closed_forms():
+    """Zero weights give relu(bias); no bias equals a zero bias; ReLU is
+    max(0, linear); a bias far below the products zeroes every output."""
+    rng = np.random.default_rng(19)
+    M, N, K = 4, 6, 64
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    bias = np.array([-2.0, -0.5, 0.0, 0.25, 1.0, 3.0], np.float32)
+    z = orc.i8_linear(x, np.zeros((N, K), np.int8), np.float32(0.5), bias, relu=True)
+    assert (z["y"] == np.maximum(0.0, bias.astype(np.float64))[None, :]).all()
+    zl = orc.i8_linear(x, np.zeros((N, K), np.int8), np.float32(0.5), bias, relu=False)
+    assert (zl["y"] == bias.astype(np.float64)[None, :]).all()
+    wq = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    a = orc.i8_linear(x, wq, np.float32(0.3), None, relu=False)["y"]
+    b = orc.i8_linear(x, wq, np.float32(0.3), np.zeros(N, np.float32), relu=False)["y"]
+    assert (a == b).all()
+    r = orc.i8_linear(x, wq, np.float32(0.3), bias, relu=True)["y"]
+    l = orc.i8_linear(x, wq, np.float32(0.3), bias, relu=False)["y"]
+    assert (r == np.maximum(0.0, l)).all() and (l < 0).any() and (l > 0).any()
+    low = orc.i8_linear(x, wq, np.float32(0.3), np.full(N, -1e6, np.float32), relu=True)["y"]
+    assert not low.any()
+
+
+def pin_i8_linear_exact_fraction():
+    """y against exact rational arithmetic on a tiny case: within 1e-15 of
+    the magnitudes summed (|product| + |bias|; the bias may cancel)."""
+    rng = np.random.default_rng(20)
+    W = (rng.standard_normal((3, 16)) * 0.03).astype(np.float32)
+    x = rng.standard_normal((2, 16)).astype(np.float32)
+    bias = np.array([0.125, -0.03, 0.0], np.float32)
+    wq, aw = orc.i8_quantize_weights(W)
+    out = orc.i8_linear(x, wq, aw, bias, relu=False)
+    for m in range(2):
+        for n in range(3):
+            acc = sum(int(out["q"][m, k]) * int(wq[n, k]) for k in range(16))
+            assert acc == out["acc"][m, n]
+            prod = F(acc) * F(float(out["amax"][m])) / 127 * F(float(aw)) / 127
+            exact = prod + F(float(bias[n]))
+            got = out["y"][m, n]
+            bound = F(1, 10**15) * (abs(prod) + abs(F(float(bias[n]))))
+            assert abs(F(got) - exact) <= bound, (m, n, got, float(exact))
+
+
+def pin_i8_scale_invariance():
+    """Scaling W by 2^j leaves wq unchanged and scales amax_w, and the
+    bias-free outputs, by exactly 2^j."""
+    rng = np.random.default_rng(21)
+    W = (rng.standard_normal((5, 48)) * 0.02).astype(np.float32)
+    x = rng.standard_normal((3, 48)).astype(np.float32)
+    wq, aw = orc.i8_quantize_weights(W)
+    y = orc.i8_linear(x, wq, aw, None, relu=False)["y"]
+    for j in (-3, 5):
+        wq2, aw2 = orc.i8_quantize_weights((W * np.float32(2.0 ** j)).astype(np.float32))
+        assert (wq2 == wq).all() and aw2 == np.float32(aw * 2.0 ** j)
+        y2 = orc.i8_linear(x, wq2, aw2, None, relu=False)["y"]
+        assert (y2 == y * 2.0 ** j).all()
+
+
 ALL_PINS = {name: fn for name, fn in sorted(globals().items())
             if name.startswith("pin_") and callable(fn)}

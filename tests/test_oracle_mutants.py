@@ -42,6 +42,15 @@ MUTANTS = {
     "add_subtracts": ("out[i] = x[i] + y[i];", "out[i] = x[i] - y[i];"),
     "silu_sign": ("z / (1.0 + exp(-z))", "z / (1.0 + exp(z))"),
     "silu_drops_u": ("exp(-z)) * (double)u[i];", "exp(-z));"),
+    "i8_no_relu": ("if (relu && v < 0.0)", "if (0 && v < 0.0)"),
+    "i8_bias_subtracted": ("v += (double)bias[n];", "v -= (double)bias[n];"),
+    "i8_bias_first_only": ("v += (double)bias[n];", "v += (double)bias[0];"),
+    "i8_weight_scale_no_127": ("const double w = (double)amax_w / 127.0;",
+                               "const double w = (double)amax_w;"),
+    "i8_token_scale_no_127": ("const double a = (double)amax_x[m] / 127.0;",
+                              "const double a = (double)amax_x[m] / 128.0;"),
+    "i8_relu_clamps_above": ("if (relu && v < 0.0)\n                v = 0.0;",
+                             "if (relu && v > 0.0)\n                v = 0.0;"),
 }
 # Not listed: removing the amax == 0 special case.  On x86-64 the resulting
 # NaN converts to 0 anyway, so that mutant is equivalent and uncatchable; the
