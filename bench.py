@@ -55,6 +55,9 @@ DECODE_MS = (4, 8, 16, 32)
 PREFILL_MS = (256, 1024, 4096)
 L2_FLUSH_BYTES = 256 << 20   # > 2 x the 126 MB L2
 PREFILL_DISTINCT_ROWS = 256  # distinct generated token rows per projection (tiled up to M)
+# I8_S encoder layer shapes (tokens M, channels K -> N = 4K): activations
+# outweigh weights 16 : 1 (M*K = 16 * N*K)
+I8_SHAPES = ((16384, 256, 1024), (32768, 512, 2048))
 
 
 def parse(argv=None):
@@ -69,7 +72,7 @@ def parse(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="headline only (no configs object)")
-    ap.add_argument("--configs", default="1,2,4,5,chain",
+    ap.add_argument("--configs", default="1,2,4,5,i8,chain",
                     help="comma list of the extra workloads to measure")
     ap.add_argument("--chain", action="store_true",
                     help="time the dependent decoder-layer chain instead of the sweep")
@@ -714,6 +717,49 @@ def measure_configs(args, api, torch, dev, rank, shapes, weights, descs_m1, want
                                              layers=args.layers)
             out[f"5_prefill_sweep_196x_M{M}"] = e
             del table, descs
+            torch.cuda.empty_cache()
+
+    if "i8" in want:
+        for (M, K, N) in I8_SHAPES:
+            W = synth.weights(7000 + K, 0, N, K, 0.05)
+            wq, amax_w = api.i8_quantize_weights(torch.from_numpy(W).to(dev))
+            bias = torch.from_numpy((np.random.default_rng(K).standard_normal(N) * 0.1)
+                                    .astype(np.float32)).to(dev)
+            xr = torch.from_numpy(synth.activations(7000 + K, 1, min(M, 1024), K)).to(dev)
+            x = xr.repeat((M + xr.shape[0] - 1) // xr.shape[0], 1)[:M].contiguous()
+            xq, amax_x, _ = api.quantize_act(x)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            ws = torch.empty(api.tw_i8_workspace_bytes(M, K), dtype=torch.uint8, device=dev)
+            api.check()
+
+            def gemm():
+                api.i8_linear_q(xq, amax_x, wq, amax_w, bias, relu=True, y=y)
+
+            def layer():
+                api.i8_linear(x, wq, amax_w, bias, relu=True, y=y, ws=ws)
+            res = {}
+            for name, fn in (("gemm", gemm), ("layer", layer)):
+                for _ in range(cwarm):
+                    fn()
+                api.check()
+                ms, per = timed_steps(torch, stream, fn, csteps, barrier)
+                api.check()
+                step_s = ms / csteps / 1e3
+                ops = 2 * M * N * K
+                nbytes = M * K + N * K + 4 * M * N + 4 * M + (4 * M * K + M * K if name == "layer" else 0)
+                res[name] = {"us_per_call": step_s * 1e6, "step_times": dist_summary(per),
+                             "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / step_s / 1e9,
+                             "frac_hbm": nbytes / step_s / 1e9 / hbm,
+                             "achieved_tops": ops / step_s / 1e12,
+                             "frac_int8": ops / step_s / 1e12 / int8_peak,
+                             "bound": "hbm" if nbytes / hbm / 1e9 > ops / int8_peak / 1e12 else "tensor",
+                             "launches_per_call": 1 if name == "gemm" else 2}
+            out[f"i8_linear_bias_relu_M{M}_K{K}_N{N}"] = {
+                **res, "inputs": f"{min(M, 1024)} distinct seeded token rows tiled to {M}; "
+                                 "W ~ N(0, 0.05^2); bias ~ N(0, 0.1^2)",
+                "note": "gemm: int8 activations quantised beforehand; layer: fp32 activations "
+                        "quantised in the call (two launches)"}
+            del W, wq, xq, x, xr, y, ws
             torch.cuda.empty_cache()
 
     if "chain" in want:

@@ -316,6 +316,105 @@ TW_API int tw_decoder_chain(const tw_chain_layer *layers, int n_layers,
  * missing or malformed). */
 TW_API int tw_chain_launches(const tw_chain_layer *layers, int n_layers);
 
+/*
+ * I8_S linear layer with fused bias and ReLU
+ * ------------------------------------------
+ * The int8 side of the model: the audio encoder keeps int8 weights and int8
+ * activations and replaces GELU by ReLU ("VibeVoice-ASR-BitNet-ONNX" model
+ * page, "Quantization" table, row "VAE encoders": I8_S), and its fused int8
+ * routines join matmul, bias and ReLU in one pass (aitrends summary,
+ * technical features).  The weights carry one absmax scale per tensor (the
+ * "_S" format, like the ternary one):
+ *   amax_w = max|W|,  wq = clamp(rint(W * (127.0f / amax_w)), -128, 127)
+ * (fp32 multiply, IEEE division, half to even; W == 0 gives wq == 0).
+ * Activations are quantised per token exactly as tw_quantize_act does.
+ *   acc[m, n] = sum_k xq[m, k] * wq[n, k]            (exact int32)
+ *   y[m, n]   = ((float)acc * (amax_x[m] / 127.0f)) * (amax_w / 127.0f) + bias[n]
+ *               then max(0, y) when relu != 0        (fp32, rounded per step)
+ * K must be a positive multiple of 16 (the operands are read as 16-byte
+ * rows; k past K reads as zero), N and M any size >= 1.  All pointers are
+ * device pointers, 16-byte aligned.
+ */
+
+/* HOST-ONLY.  Scratch of tw_i8_linear: the int8 rows and scales of x. */
+TW_API size_t tw_i8_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * Quantise the weights of one I8_S layer: W [N x K] fp32 -> wq [N x K] int8
+ * (row-major) and amax_w (one float).  A non-finite W sets TW_ERR_NONFINITE
+ * in the device error word (tw_check); wq is then unspecified.
+ */
+TW_API int tw_i8_quantize_weights(const float *W, int64_t N, int64_t K, int8_t *wq,
+                                  float *amax_w, tw_stream_t stream);
+
+/*
+ * y [M x N] fp32 from int8 activations xq [M x K] with their per-token
+ * amax_x [M] (as tw_quantize_act writes them), wq [N x K] and amax_w from
+ * tw_i8_quantize_weights, bias [N] fp32 (NULL: no bias), relu 0 or 1.
+ * acc_out [M x N] int32 receives the exact accumulators (NULL: not written).
+ * One launch on the tensor cores.
+ */
+TW_API int tw_i8_linear_q(const int8_t *xq, const float *amax_x, int64_t M, int64_t N, int64_t K,
+                          const int8_t *wq, const float *amax_w, const float *bias, int relu,
+                          float *y, int32_t *acc_out, tw_stream_t stream);
+
+/*
+ * The same layer from fp32 activations x [M x K]: quantises x into ws
+ * (ws_bytes >= tw_i8_workspace_bytes(M, K)), then runs tw_i8_linear_q.
+ */
+TW_API int tw_i8_linear(const float *x, int64_t M, int64_t N, int64_t K, const int8_t *wq,
+                        const float *amax_w, const float *bias, int relu, float *y,
+                        int32_t *acc_out, void *ws, size_t ws_bytes, tw_stream_t stream);
+
+/*
+ * Tensor-parallel split of the projections
+ * ----------------------------------------
+ * Pieces of a Megatron-style split across ranks (one GPU each).  The pages
+ * describe single-process inference; the split is this library's own and
+ * its result is, by construction, the single-device result bit for bit.
+ *  - column-parallel (q, k, v, gate, up): a rank holds rows [n0, n0 + rows)
+ *    of W (tw_pack_slice of the whole matrix's codes, with the whole
+ *    matrix's wscale) and the whole input; its output is its slice of y.
+ *  - row-parallel (o, down): a rank holds input columns [k0, k0 + cols) and
+ *    the matching columns of W (tw_pack_slice).  Per token: tw_row_absmax of
+ *    its slice, a max all-reduce of those M floats over the ranks,
+ *    tw_quantize_act_given with that maximum, tw_ternary_linear_q into its
+ *    int32 acc_out, an int32 sum all-reduce of the M x N partial sums, and
+ *    tw_rescale_acc.  The collectives are the caller's (NCCL).
+ */
+
+/*
+ * Copy the codes of the sub-matrix rows [n0, n0 + rows) x columns
+ * [k0, k0 + cols) of a packed [N x K] matrix into `out` in the packed layout
+ * of a [rows x cols] matrix (out_bytes >= tw_packed_bytes(rows, cols)).
+ * n0 a multiple of 16, k0 and cols multiples of 128; rows past the slice in
+ * its last 16-row block are written as code 0.  Exact (a byte gather).
+ */
+TW_API int tw_pack_slice(const void *packed, int64_t N, int64_t K, int64_t n0, int64_t rows,
+                         int64_t k0, int64_t cols, void *out, size_t out_bytes,
+                         tw_stream_t stream);
+
+/* amax[m] = max_k |x[m, k]| of x [M x K] fp32 (K a multiple of 4); exact. */
+TW_API int tw_row_absmax(const float *x, int64_t M, int64_t K, float *amax, tw_stream_t stream);
+
+/*
+ * Per-token int8 quantisation with a given per-token absmax (as
+ * tw_quantize_act, but amax[m] is an input, e.g. the maximum over the
+ * ranks' slices of the row): xq = clamp(rint(x * (127.0f / amax[m])),
+ * -128, 127); amax[m] == 0 gives xq == 0; qsum[m] = sum_k xq[m, k] (may be
+ * NULL).  K a multiple of 4.
+ */
+TW_API int tw_quantize_act_given(const float *x, int64_t M, int64_t K, const float *amax,
+                                 int8_t *xq, int32_t *qsum, tw_stream_t stream);
+
+/*
+ * y [M x N] = ((float)acc * (amax[m] / 127.0f)) * wscale[0]: the rescale
+ * every projection epilogue of this library applies, for accumulators
+ * summed outside (acc [M x N] int32, amax [M], wscale one float).
+ */
+TW_API int tw_rescale_acc(const int32_t *acc, int64_t M, int64_t N, const float *amax,
+                          const float *wscale, float *y, tw_stream_t stream);
+
 /* Wait for `stream`, then return and clear the device error word of the
  * current device (TW_OK if no kernel reported an error). */
 TW_API int tw_check(tw_stream_t stream);

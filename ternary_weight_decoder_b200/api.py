@@ -71,6 +71,12 @@ tw_debug_wait_timeout = _sig("tw_debug_wait_timeout", _int, [ctypes.c_uint64, _p
 tw_chain_workspace_bytes = _sig("tw_chain_workspace_bytes", _sz, [_p, _int])
 tw_decoder_chain = _sig("tw_decoder_chain", _int, [_p, _int, _p, _p, _sz, _p])
 tw_chain_launches = _sig("tw_chain_launches", _int, [_p, _int])
+tw_i8_workspace_bytes = _sig("tw_i8_workspace_bytes", _sz, [_i64, _i64])
+tw_i8_quantize_weights = _sig("tw_i8_quantize_weights", _int, [_p, _i64, _i64, _p, _p, _p])
+tw_i8_linear_q = _sig("tw_i8_linear_q", _int,
+                      [_p, _p, _i64, _i64, _i64, _p, _p, _p, _int, _p, _p, _p])
+tw_i8_linear = _sig("tw_i8_linear", _int,
+                    [_p, _i64, _i64, _i64, _p, _p, _p, _int, _p, _p, _p, _sz, _p])
 
 
 class ProjDesc(ctypes.Structure):
@@ -330,3 +336,45 @@ def decoder_chain(chain: DecoderChain, first: int = 0, count=None, stream=None):
                          ctypes.POINTER(ChainLayer))
     _raise(tw_decoder_chain(layers, count, ctypes.byref(chain.c_buf), _ptr(chain.ws),
                             chain.ws_bytes, _stream(stream)))
+
+
+# ------------------------------------------------------ I8_S linear layer
+def i8_quantize_weights(W: torch.Tensor, stream=None):
+    """W [N, K] fp32 (CUDA) -> (wq int8 [N, K], amax_w fp32[1])."""
+    _need(W, torch.float32, "W")
+    N, K = W.shape
+    wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    amax = torch.empty(4, dtype=torch.float32, device=W.device)
+    _raise(tw_i8_quantize_weights(_ptr(W), N, K, _ptr(wq), _ptr(amax), _stream(stream)))
+    return wq, amax[:1]
+
+
+def i8_linear_q(xq, amax_x, wq, amax_w, bias=None, relu: bool = True, y=None, acc_out=None,
+                stream=None):
+    """y [M, N] fp32 from xq [M, K] int8 + amax_x [M] and wq [N, K] + amax_w."""
+    _need(xq, torch.int8, "xq")
+    _need(wq, torch.int8, "wq")
+    M, K = xq.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=xq.device)
+    _raise(tw_i8_linear_q(_ptr(xq), _ptr(amax_x), M, N, K, _ptr(wq), _ptr(amax_w), _ptr(bias),
+                          int(bool(relu)), _ptr(y), _ptr(acc_out), _stream(stream)))
+    return y
+
+
+def i8_linear(x, wq, amax_w, bias=None, relu: bool = True, y=None, acc_out=None, ws=None,
+              stream=None):
+    """y [M, N] fp32 = relu?(I8_S layer) from fp32 x [M, K]."""
+    _need(x, torch.float32, "x")
+    _need(wq, torch.int8, "wq")
+    M, K = x.shape
+    N = wq.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    wsb = int(tw_i8_workspace_bytes(M, K))
+    if ws is None:
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=x.device)
+    _raise(tw_i8_linear(_ptr(x), M, N, K, _ptr(wq), _ptr(amax_w), _ptr(bias), int(bool(relu)),
+                        _ptr(y), _ptr(acc_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
