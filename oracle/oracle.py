@@ -56,6 +56,8 @@ def _bind(lib):
     lib.orc_i8_quantize_weights.argtypes = [p, i64, i64, p, p]
     lib.orc_i8_epilogue.restype = None
     lib.orc_i8_epilogue.argtypes = [p, i64, i64, p, ctypes.c_float, p, ctypes.c_int, p]
+    lib.orc_quantize_act_given.restype = None
+    lib.orc_quantize_act_given.argtypes = [p, i64, i64, p, p]
     return lib
 
 
@@ -240,3 +242,15 @@ def i8_linear(x, wq, amax_w, bias=None, relu=True):
     acc = ternary_acc(wq, q)       # an exact int8 dot product for any int8 weights
     y = i8_epilogue(acc, amax, amax_w, bias, relu)
     return {"q": q, "amax": amax, "acc": acc, "y": y}
+
+
+# ------------------------------------------------ tensor-parallel split (R20)
+def quantize_act_given(x, amax):
+    """R20: q int8 [M,K] of x [M,K] with the given per-token amax [M]."""
+    x, px = _c(x, np.float32)
+    amax, pa = _c(amax, np.float32)
+    M, K = x.shape
+    assert amax.shape == (M,)
+    q = np.empty((M, K), np.int8)
+    _load().orc_quantize_act_given(px, M, K, pa, q.ctypes.data)
+    return q

@@ -255,3 +255,33 @@ void orc_i8_epilogue(const int32_t *acc, int64_t M, int64_t N,
         }
     }
 }
+
+/* ------------------------------------------------------------------------
+ * Tensor-parallel split (this library's own; the pages describe one CPU
+ * process).  A row-parallel projection quantises each rank's slice of a
+ * token row with the absmax of the whole row, which the ranks share:
+ *   R20 q = clamp(rint(x * (127 / amax_row)), -128, 127), the R4 rule with
+ *       the given amax (a row maximum over all slices), amax == 0 -> q = 0.
+ * The partial sums of the slices add up to orc_ternary_acc of the whole row.
+ * ---------------------------------------------------------------------- */
+void orc_quantize_act_given(const float *x, int64_t M, int64_t K,
+                            const float *amax, int8_t *q)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        const float a = amax[m];
+        if (a == 0.0f) {
+            for (int64_t k = 0; k < K; ++k)
+                q[m * K + k] = 0;
+            continue;
+        }
+        const float scale = 127.0f / a;
+        for (int64_t k = 0; k < K; ++k) {
+            float r = rintf(x[m * K + k] * scale);
+            if (r > 127.0f)
+                r = 127.0f;
+            if (r < -128.0f)
+                r = -128.0f;
+            q[m * K + k] = (int8_t)r;
+        }
+    }
+}

@@ -71,6 +71,10 @@ tw_debug_wait_timeout = _sig("tw_debug_wait_timeout", _int, [ctypes.c_uint64, _p
 tw_chain_workspace_bytes = _sig("tw_chain_workspace_bytes", _sz, [_p, _int])
 tw_decoder_chain = _sig("tw_decoder_chain", _int, [_p, _int, _p, _p, _sz, _p])
 tw_chain_launches = _sig("tw_chain_launches", _int, [_p, _int])
+tw_pack_slice = _sig("tw_pack_slice", _int, [_p, _i64, _i64, _i64, _i64, _i64, _i64, _p, _sz, _p])
+tw_row_absmax = _sig("tw_row_absmax", _int, [_p, _i64, _i64, _p, _p])
+tw_quantize_act_given = _sig("tw_quantize_act_given", _int, [_p, _i64, _i64, _p, _p, _p, _p])
+tw_rescale_acc = _sig("tw_rescale_acc", _int, [_p, _i64, _i64, _p, _p, _p, _p])
 tw_i8_workspace_bytes = _sig("tw_i8_workspace_bytes", _sz, [_i64, _i64])
 tw_i8_quantize_weights = _sig("tw_i8_quantize_weights", _int, [_p, _i64, _i64, _p, _p, _p])
 tw_i8_linear_q = _sig("tw_i8_linear_q", _int,
@@ -377,4 +381,45 @@ def i8_linear(x, wq, amax_w, bias=None, relu: bool = True, y=None, acc_out=None,
         ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=x.device)
     _raise(tw_i8_linear(_ptr(x), M, N, K, _ptr(wq), _ptr(amax_w), _ptr(bias), int(bool(relu)),
                         _ptr(y), _ptr(acc_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+# ------------------------------------------------ tensor-parallel pieces
+def pack_slice(packed: torch.Tensor, N: int, K: int, n0: int, rows: int, k0: int, cols: int,
+               stream=None):
+    """Packed codes of rows [n0, n0+rows) x columns [k0, k0+cols) of a packed [N, K]."""
+    _need(packed, torch.uint8, "packed")
+    out = torch.empty(max(packed_bytes(rows, cols), 16), dtype=torch.uint8, device=packed.device)
+    _raise(tw_pack_slice(_ptr(packed), N, K, n0, rows, k0, cols, _ptr(out), out.numel(),
+                         _stream(stream)))
+    return out
+
+
+def row_absmax(x: torch.Tensor, stream=None):
+    """amax [M] = max |x| per row of x [M, K] fp32."""
+    _need(x, torch.float32, "x")
+    M, K = x.shape
+    amax = torch.empty(M, dtype=torch.float32, device=x.device)
+    _raise(tw_row_absmax(_ptr(x), M, K, _ptr(amax), _stream(stream)))
+    return amax
+
+
+def quantize_act_given(x: torch.Tensor, amax: torch.Tensor, stream=None):
+    """(xq int8 [M, K], qsum int32 [M]) of x with the given per-token amax."""
+    _need(x, torch.float32, "x")
+    _need(amax, torch.float32, "amax")
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    qsum = torch.empty(M, dtype=torch.int32, device=x.device)
+    _raise(tw_quantize_act_given(_ptr(x), M, K, _ptr(amax), _ptr(xq), _ptr(qsum), _stream(stream)))
+    return xq, qsum
+
+
+def rescale_acc(acc: torch.Tensor, amax: torch.Tensor, wscale: torch.Tensor, y=None, stream=None):
+    """y [M, N] fp32 from summed accumulators acc [M, N] int32."""
+    _need(acc, torch.int32, "acc")
+    M, N = acc.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=acc.device)
+    _raise(tw_rescale_acc(_ptr(acc), M, N, _ptr(amax), _ptr(wscale), _ptr(y), _stream(stream)))
     return y

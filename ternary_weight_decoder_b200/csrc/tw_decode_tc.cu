@@ -16,7 +16,10 @@
 // projections of larger K first, so that the units left at the end of the
 // sweep are the small ones.  Per 128-column k tile (a stage):
 //   * warp 0 (producer) loads the 8 x 512 B code tiles with one 3-D TMA and
-//     the token block (N rows x 128 B) with one bulk copy;
+//     the token block (N rows x 128 B) with one bulk copy into a ring of L
+//     shared-memory stages (L = 8 to 32, as many as fit: the ring is what
+//     keeps enough code bytes in flight to cover the memory latency; it is
+//     decoupled from the 8 tensor-memory A slots below);
 //   * eight expansion warps (two per TMEM lane quarter, alternating stages)
 //     turn each 16-byte lane slot of the code tile into 16 registers with
 //     one AND each -- (word & (3 << 2s per byte)) holds codes + 1 of four
@@ -24,8 +27,11 @@
 //     tensor memory (tcgen05.st 16x256b): column 8s + 2t + h of lane (row)
 //     g or g + 8 holds slot s of the word with k = 64h + 16t + 4s .. + 3.
 //     Slot 3 (4^3 (c + 1) = 128 does not fit int8) is shifted down instead;
-//   * warp 1 issues four MMAs of K = 32, one per slot s (columns 8s .. 8s+7),
-//     into accumulator D_s (N columns each);
+//   * warp 1 waits only for the expansion of the stage (which itself waited
+//     for the stage's bytes), issues four MMAs of K = 32, one per slot s
+//     (columns 8s .. 8s+7), into accumulator D_s (N columns each), and
+//     commits them to the stage's empty barrier, which frees both the shared-
+//     memory stage and, eight stages later, the A slot;
 //   * four epilogue warps (one per lane quarter) read D_0..D_3 and form
 //     acc = D_0 + D_1/4 + D_2/16 + D_3 - sum(q), exact (D_s is a multiple
 //     of 4^s), then y.
@@ -45,8 +51,9 @@
 namespace tw {
 namespace {
 
-constexpr int kStagesTc = 8;
+constexpr int kASlots = 8;                      // tensor-memory A slots (32 columns each)
 constexpr int kRingTc = 8;                      // unit-info entries
+constexpr int kMaxStagesTc = 32;                // shared-memory load stages, at most
 constexpr int kThreadsTc = 14 * 32;
 constexpr int kCodeStageBytes = 8 * kTileBytes;  // 128 rows x 128 k = 4 KB
 constexpr int kTmemColsTc = 512;
@@ -108,7 +115,7 @@ struct TcLayout {
     static constexpr int kMisc = 2048;
     // + the unit order (16 bytes) and the projection cache (40 bytes) per
     // projection after the misc block
-    static int smem(int count) { return 1024 + kStagesTc * kStage + kMisc + 56 * count; }
+    static int smem(int count, int stages) { return 1024 + stages * kStage + kMisc + 56 * count; }
     uint32_t base;
     __device__ uint32_t codes(int s) const { return base + s * kStage; }
     __device__ uint32_t tok(int s) const { return base + s * kStage + kCodeStageBytes; }
@@ -132,28 +139,32 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&v)[NTOK])
         tmem_ld32_nowait(taddr, v);
 }
 
-template <int NTOK>
+// L shared-memory stages (8 .. kMaxStagesTc).  Stage counters are 32-bit:
+// a block streams at most a few thousand stages per call.
+template <int NTOK, int L>
 __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_constant__ TcParams p)
 {
-    using L = TcLayout<NTOK>;
+    static_assert(L >= kASlots && L <= kMaxStagesTc && L % 2 == 0, "load stages");
+    using Lay = TcLayout<NTOK>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
-    const L lay{base};
-    uint8_t *misc = smem_raw + (base - raw) + kStagesTc * L::kStage;
+    const Lay lay{base};
+    uint8_t *misc = smem_raw + (base - raw) + L * Lay::kStage;
     uint64_t *bars = reinterpret_cast<uint64_t *>(misc);
     const uint32_t bar0 = smem_u32(bars);
-    const uint32_t b_full = bar0, b_empty = b_full + 8 * kStagesTc, b_afull = b_empty + 8 * kStagesTc;
-    const uint32_t b_ufull = b_afull + 8 * kStagesTc, b_uempty = b_ufull + 8 * kRingTc;
+    // full/empty: per load stage; afull: per A slot
+    const uint32_t b_full = bar0, b_empty = b_full + 8 * L, b_afull = b_empty + 8 * L;
+    const uint32_t b_ufull = b_afull + 8 * kASlots, b_uempty = b_ufull + 8 * kRingTc;
     const uint32_t b_dfull = b_uempty + 8 * kRingTc, b_dempty = b_dfull + 16;
     const uint32_t b_drain = b_dempty + 16;
     int *stage_stop = reinterpret_cast<int *>(misc + 1024);
-    UnitInfo *ring = reinterpret_cast<UnitInfo *>(misc + 1024 + 4 * kStagesTc);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 1024 + 4 * kStagesTc + 16 * kRingTc);
+    UnitInfo *ring = reinterpret_cast<UnitInfo *>(misc + 1024 + 4 * kMaxStagesTc);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 1024 + 4 * kMaxStagesTc + 16 * kRingTc);
     int *abort_p = reinterpret_cast<int *>(tmem_slot + 1);
     volatile int *abort_flag = abort_p;
-    UnitOrder *order_s = reinterpret_cast<UnitOrder *>(misc + L::kMisc);
-    ProjS *proj_s = reinterpret_cast<ProjS *>(misc + L::kMisc + 16 * p.count);
+    UnitOrder *order_s = reinterpret_cast<UnitOrder *>(misc + Lay::kMisc);
+    ProjS *proj_s = reinterpret_cast<ProjS *>(misc + Lay::kMisc + 16 * p.count);
     for (int i = threadIdx.x; i < p.count; i += kThreadsTc) {
         order_s[i] = p.order[i];
         const DescRecord &r = p.table[i];
@@ -162,11 +173,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStagesTc; ++s) {
+        for (int s = 0; s < L; ++s) {
             mbar_init(b_full + 8 * s, 1);
-            mbar_init(b_empty + 8 * s, 5);   // 4 expansion warps + the MMA commit
-            mbar_init(b_afull + 8 * s, 4);
+            mbar_init(b_empty + 8 * s, 1);   // the MMA commit of the stage
         }
+        for (int a = 0; a < kASlots; ++a)
+            mbar_init(b_afull + 8 * a, 4);   // the 4 expansion warps of the stage's set
         for (int j = 0; j < kRingTc; ++j) {
             mbar_init(b_ufull + 8 * j, 1);
             mbar_init(b_uempty + 8 * j, 4);
@@ -189,18 +201,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
     if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
-            int64_t it = 0;
+            uint32_t it = 0;
             bool ok = true, tokens_ready = false;
             // Token blocks of the stages issued before launch 1 has finished:
             // the codes of the first stages stream while it still quantises.
-            const uint8_t *pend_src[kStagesTc];
-            int pend_s[kStagesTc];
+            const uint8_t *pend_src[L];
+            int pend_s[L];
             int npend = 0;
             auto flush_tokens = [&]() {
                 pdl_wait_tc();
                 tokens_ready = true;
                 for (int i = 0; i < npend; ++i)
-                    bulk_g2s(lay.tok(pend_s[i]), pend_src[i], (uint32_t)L::kBBytes,
+                    bulk_g2s(lay.tok(pend_s[i]), pend_src[i], (uint32_t)Lay::kBBytes,
                              b_full + 8 * pend_s[i]);
                 npend = 0;
             };
@@ -229,23 +241,22 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                 const void *tmap = p.table[u.d].tmap_codes;   // address only
                 const uint8_t *tok_src = p.ws + proj_s[u.d].ws_xq_off;
                 for (int kt = 0; kt < u.KT; ++kt, ++it) {
-                    const int s = (int)(it % kStagesTc);
-                    if (it >= kStagesTc &&
-                        !mbar_wait(b_empty + 8 * s, (uint32_t)((it / kStagesTc - 1) & 1), p.ctl,
-                                   abort_flag)) {
+                    const int s = (int)(it % L);
+                    if (it >= L &&
+                        !mbar_wait(b_empty + 8 * s, (it / L - 1) & 1u, p.ctl, abort_flag)) {
                         ok = false;
                         break;
                     }
                     stage_stop[s] = 0;
-                    mbar_arrive_expect_tx(b_full + 8 * s, (uint32_t)(kCodeStageBytes + L::kBBytes));
+                    mbar_arrive_expect_tx(b_full + 8 * s, (uint32_t)(kCodeStageBytes + Lay::kBBytes));
                     tma_load_3d(lay.codes(s), tmap, 0, kt, 8 * u.rt, b_full + 8 * s);
-                    const uint8_t *src = tok_src + (int64_t)kt * L::kBBytes;
+                    const uint8_t *src = tok_src + (int64_t)kt * Lay::kBBytes;
                     if (tokens_ready) {
-                        bulk_g2s(lay.tok(s), src, (uint32_t)L::kBBytes, b_full + 8 * s);
+                        bulk_g2s(lay.tok(s), src, (uint32_t)Lay::kBBytes, b_full + 8 * s);
                     } else {
                         pend_src[npend] = src;
                         pend_s[npend] = s;
-                        if (++npend == kStagesTc)
+                        if (++npend == L)
                             flush_tokens();   // before any stage is waited on again
                     }
                 }
@@ -254,9 +265,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                 flush_tokens();
             // One stop stage for each expansion set.
             for (int e = 0; e < 2 && ok; ++e, ++it) {
-                const int s = (int)(it % kStagesTc);
-                if (it >= kStagesTc &&
-                    !mbar_wait(b_empty + 8 * s, (uint32_t)((it / kStagesTc - 1) & 1), p.ctl, abort_flag)) {
+                const int s = (int)(it % L);
+                if (it >= L && !mbar_wait(b_empty + 8 * s, (it / L - 1) & 1u, p.ctl, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -266,16 +276,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
             // Drain: every copy this thread issued lands before the block exits.
             WaitCtl drain = p.ctl;
             drain.timeout_ns = kDrainNsTc;
-            for (int64_t j = it - kStagesTc; j < it; ++j)
-                if (j >= 0)
-                    mbar_wait(b_full + 8 * (int)(j % kStagesTc), (uint32_t)((j / kStagesTc) & 1), drain,
-                              nullptr);
+            for (uint32_t j = it > (uint32_t)L ? it - L : 0; j < it; ++j)
+                mbar_wait(b_full + 8 * (int)(j % L), (j / L) & 1u, drain, nullptr);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int64_t it = 0;
+            uint32_t it = 0;
             bool ok = true;
             for (int j = 0; ok; ++j) {
                 const int ju = j % kRingTc;
@@ -291,20 +299,21 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                 tc_fence_after();
                 const uint32_t d0 = tmem + kDCol0 + (uint32_t)(buf * 4 * NTOK);
                 for (int kt = 0; kt < u.KT; ++kt, ++it) {
-                    const int s = (int)(it % kStagesTc);
-                    const uint32_t ph = (uint32_t)((it / kStagesTc) & 1);
-                    if (!mbar_wait(b_full + 8 * s, ph, p.ctl, abort_flag) ||
-                        !mbar_wait(b_afull + 8 * s, ph, p.ctl, abort_flag)) {
+                    // The expansion of this stage waited for its bytes (codes and
+                    // token block) before it arrived here.
+                    const int a = (int)(it % kASlots);
+                    if (!mbar_wait(b_afull + 8 * a, (it / kASlots) & 1u, p.ctl, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
+                    const int s = (int)(it % L);
                     const uint64_t bd = sdesc_k_sw128(lay.tok(s));
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // +32 bytes of K = +2 in the address field
-                        mma_i8_ts(d0 + (uint32_t)(kk * NTOK), tmem + (uint32_t)(32 * s + 8 * kk),
+                        mma_i8_ts(d0 + (uint32_t)(kk * NTOK), tmem + (uint32_t)(32 * a + 8 * kk),
                                   bd + 2 * kk, idesc_tc<NTOK>(), kt > 0 ? 1u : 0u);
-                    mma_commit(b_empty + 8 * s);
+                    mma_commit(b_empty + 8 * s);   // frees stage s, and A slot a for stage it + 8
                 }
                 if (!ok)
                     break;
@@ -390,12 +399,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
         // ------------------------------------------------------ expansion
         const int quarter = warp & 3, set = (warp - 6) >> 2;
         const uint32_t m = 0x03030303u;
-        for (int64_t it = set;; it += 2) {
-            const int s = (int)(it % kStagesTc);
-            if (!mbar_wait(b_full + 8 * s, (uint32_t)((it / kStagesTc) & 1), p.ctl, abort_flag))
+        for (uint32_t it = set;; it += 2) {
+            const int s = (int)(it % L);
+            if (!mbar_wait(b_full + 8 * s, (it / L) & 1u, p.ctl, abort_flag))
                 break;
             if (stage_stop[s])
                 break;
+            // A slot it % 8 is free once the MMAs of stage it - 8 have completed.
+            if (it >= (uint32_t)kASlots &&
+                !mbar_wait(b_empty + 8 * (int)((it - kASlots) % L), ((it - kASlots) / L) & 1u, p.ctl,
+                           abort_flag))
+                break;
+            const uint32_t aslot = it % kASlots;
             tc_fence_after();
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -415,15 +430,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                 r[13] = (w.z >> 6) & m;
                 r[14] = (w.y >> 6) & m;
                 r[15] = (w.w >> 6) & m;
-                tmem_st16x256b_x4(tmem + (uint32_t)(32 * s) + ((uint32_t)(32 * quarter + 16 * h) << 16), r);
+                tmem_st16x256b_x4(tmem + 32 * aslot + ((uint32_t)(32 * quarter + 16 * h) << 16), r);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(b_afull + 8 * s);
-                mbar_arrive(b_empty + 8 * s);
-            }
+            if (lane == 0)
+                mbar_arrive(b_afull + 8 * aslot);
         }
     }
 
@@ -443,11 +456,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
     }
 }
 
-template <int NTOK>
-cudaError_t launch_tc(const TcParams &p, int grid, cudaStream_t stream)
+template <int NTOK, int L>
+cudaError_t launch_tc_l(const TcParams &p, int grid, cudaStream_t stream)
 {
-    const int smem = TcLayout<NTOK>::smem(p.count);
-    cudaError_t e = cudaFuncSetAttribute(k_decode_tc<NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = TcLayout<NTOK>::smem(p.count, L);
+    cudaError_t e = cudaFuncSetAttribute(k_decode_tc<NTOK, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return e;
     // Programmatic dependent launch: the codes stream while launch 1 runs.
@@ -461,7 +474,30 @@ cudaError_t launch_tc(const TcParams &p, int grid, cudaStream_t stream)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_decode_tc<NTOK>, p);
+    return cudaLaunchKernelEx(&cfg, k_decode_tc<NTOK, L>, p);
+}
+
+// The deepest ring of load stages that fits in shared memory beside the
+// per-projection caches (more stages keep more code bytes in flight).
+template <int NTOK>
+cudaError_t launch_tc(const TcParams &p, int grid, cudaStream_t stream)
+{
+    constexpr int kLimit = 227 * 1024;
+#ifdef TW_TC_STAGES
+    if (TW_TC_STAGES == 32 && TcLayout<NTOK>::smem(p.count, 32) <= kLimit) return launch_tc_l<NTOK, 32>(p, grid, stream);
+    if (TW_TC_STAGES == 24 && TcLayout<NTOK>::smem(p.count, 24) <= kLimit) return launch_tc_l<NTOK, 24>(p, grid, stream);
+    if (TW_TC_STAGES == 16 && TcLayout<NTOK>::smem(p.count, 16) <= kLimit) return launch_tc_l<NTOK, 16>(p, grid, stream);
+    if (TW_TC_STAGES == 8) return launch_tc_l<NTOK, 8>(p, grid, stream);
+#endif
+    if (TcLayout<NTOK>::smem(p.count, 32) <= kLimit)
+        return launch_tc_l<NTOK, 32>(p, grid, stream);
+    if (TcLayout<NTOK>::smem(p.count, 24) <= kLimit)
+        return launch_tc_l<NTOK, 24>(p, grid, stream);
+    if (TcLayout<NTOK>::smem(p.count, 16) <= kLimit)
+        return launch_tc_l<NTOK, 16>(p, grid, stream);
+    if (TcLayout<NTOK>::smem(p.count, 8) <= kLimit)
+        return launch_tc_l<NTOK, 8>(p, grid, stream);
+    return cudaErrorInvalidValue;   // too many projections for the caches
 }
 
 }  // namespace

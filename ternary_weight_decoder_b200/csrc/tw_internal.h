@@ -113,7 +113,10 @@ inline int tc_tokens(int64_t M) { return M <= 8 ? 8 : M <= 16 ? 16 : 32; }
 // Which decode kernel runs a sweep of M tokens (measured on B200: the
 // tensor-core sweep wins once the int8 MMAs of the register path, 4 per
 // 8 tokens per tile, and their operand loads no longer keep up with HBM).
-inline bool decode_sweep_on_tensor_cores(int64_t M) { return M > 16; }
+#ifndef TW_TC_DECODE_MIN_M
+#define TW_TC_DECODE_MIN_M 17
+#endif
+inline bool decode_sweep_on_tensor_cores(int64_t M) { return M >= TW_TC_DECODE_MIN_M; }
 // Projections in the order their units are handed out (K descending); the
 // units of entry i are [unit_begin, unit_begin + units), one per 128 rows.
 struct UnitOrder {

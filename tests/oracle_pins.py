@@ -494,5 +494,44 @@ def pin_i8_scale_invariance():
         assert (y2 == y * 2.0 ** j).all()
 
 
+# ------------------------------------------------ tensor-parallel split (R20)
+def pin_quantize_given_own_amax_is_r4():
+    """With each row's own absmax the given-scale rule is the R4 quantiser;
+    a larger given amax follows the fp32 rule (numpy float32 division,
+    product and rint) and never clips."""
+    rng = np.random.default_rng(30)
+    x = rng.standard_normal((5, 96)).astype(np.float32)
+    x[2] = 0.0
+    q, amax = orc.quantize_act(x)
+    assert (orc.quantize_act_given(x, amax) == q).all()
+    big = (amax * np.float32(3.0)).astype(np.float32)
+    got = orc.quantize_act_given(x, big)
+    for m in range(5):
+        if big[m] == 0:
+            assert not got[m].any()
+            continue
+        scale = np.float32(127.0) / big[m]
+        assert (got[m] == np.rint(x[m] * scale).astype(np.int8)).all()
+    assert np.abs(got.astype(np.int32)).max() <= 43   # 127 / 3, rounded
+
+
+def pin_row_parallel_slices_sum_to_the_row():
+    """Slices of a token row quantised with the whole row's absmax, summed
+    over their partial accumulators, give the unsplit layer exactly."""
+    rng = np.random.default_rng(31)
+    N, K, M = 24, 512, 3
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    codes, mean = orc.ternarize(W)
+    full = orc.ternary_linear(x, codes, mean)
+    bounds = [0, 128, 384, 512]
+    amax = np.max([np.abs(x[:, a:b]).max(axis=1) for a, b in zip(bounds, bounds[1:])], axis=0)
+    assert (amax == full["amax"]).all()
+    acc = sum(orc.ternary_acc(codes[:, a:b], orc.quantize_act_given(x[:, a:b], amax))
+              for a, b in zip(bounds, bounds[1:]))
+    assert (acc == full["acc"]).all()
+    assert (orc.rescale(acc, amax, mean) == full["y"]).all()
+
+
 ALL_PINS = {name: fn for name, fn in sorted(globals().items())
             if name.startswith("pin_") and callable(fn)}

@@ -20,7 +20,8 @@ MUTANTS = {
     "no_clip": ("if (r > 1.0)\n            r = 1.0;",
                 "if (r > 2.0)\n            r = 2.0;"),
     "s_not_reciprocal": ("double s = 1.0 / mean;", "double s = mean;"),
-    "scale_128": ("float scale = 127.0f / a;", "float scale = 128.0f / a;"),
+    "scale_128": ("float scale = 127.0f / a;\n        for (int64_t k = 0; k < K; ++k) {\n            float v",
+                  "float scale = 128.0f / a;\n        for (int64_t k = 0; k < K; ++k) {\n            float v"),
     "drop_last_term": ("for (int64_t k = 0; k < K; ++k)\n                sum +=",
                        "for (int64_t k = 0; k < K - 1; ++k)\n                sum +="),
     "sign_flip": ("sum += (int64_t)codes", "sum -= (int64_t)codes"),
@@ -49,12 +50,14 @@ MUTANTS = {
                                "const double w = (double)amax_w;"),
     "i8_token_scale_no_127": ("const double a = (double)amax_x[m] / 127.0;",
                               "const double a = (double)amax_x[m] / 128.0;"),
+    "given_scale_128": ("const float scale = 127.0f / a;", "const float scale = 128.0f / a;"),
     "i8_relu_clamps_above": ("if (relu && v < 0.0)\n                v = 0.0;",
                              "if (relu && v > 0.0)\n                v = 0.0;"),
 }
-# Not listed: removing the amax == 0 special case.  On x86-64 the resulting
-# NaN converts to 0 anyway, so that mutant is equivalent and uncatchable; the
-# special case stays because the conversion of NaN is undefined in C.
+# Not listed: removing the amax == 0 special cases (of orc_quantize_act and
+# orc_quantize_act_given).  On x86-64 the resulting NaN converts to 0 anyway,
+# so those mutants are equivalent and uncatchable; the special cases stay
+# because the conversion of NaN is undefined in C.
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
