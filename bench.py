@@ -439,7 +439,7 @@ def run_chain(args, api, torch, dev, rank, world, dist, local):
 
     def step():
         chain.h.copy_(h0, non_blocking=True)   # every step starts from the same token state
-        api.decoder_chain(chain)
+        api.decoder_chain_fused(chain)
 
     for _ in range(args.warmup):
         step()
@@ -468,7 +468,7 @@ def run_chain(args, api, torch, dev, rank, world, dist, local):
         f0.record(stream)
         for _ in range(k2):
             chain.h.copy_(h0_host, non_blocking=True)
-            api.decoder_chain(chain)
+            api.decoder_chain_fused(chain)
             out.copy_(chain.h.view(-1), non_blocking=True)
             stream.synchronize()
         f1.record(stream)
@@ -493,10 +493,11 @@ def run_chain(args, api, torch, dev, rank, world, dist, local):
                    "l2": f"codes {codes / 1e6:.0f} MB > 126 MB L2; no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": None, "peak_source": peak_source(src),
-                     "algorithmic_bytes_per_step": algo, "weight_bytes_per_step": codes},
+                     "algorithmic_bytes_per_step": algo, "weight_bytes_per_step": codes,
+                     "note": "the fused chain: one persistent launch per 8 tokens"},
         "step_times": dist_summary(per),
         "cpu_baseline": None, "e2e": e2e,
-        "gpu_launches": chain.launches * args.steps, "clocks": clk.summary(),
+        "gpu_launches": chain.fused_launches * args.steps, "clocks": clk.summary(),
     }))
 
 
@@ -768,21 +769,27 @@ def measure_configs(args, api, torch, dev, rank, shapes, weights, descs_m1, want
         h0 = torch.from_numpy(synth.activations(rank_layer_seed(0, rank), 0, M,
                                                 CHAIN_DIMS[0])).to(dev)
 
-        def cstep():
-            chain.h.copy_(h0, non_blocking=True)
-            api.decoder_chain(chain)
-        for _ in range(cwarm):
-            cstep()
-        api.check()
-        ms, per = timed_steps(torch, stream, cstep, csteps, barrier)
-        api.check()
-        algo, codes = chain_bytes(shapes, M)
-        step_s = ms / csteps / 1e3
+        res = {}
+        for name, run, launches in (("fused", api.decoder_chain_fused, chain.fused_launches),
+                                    ("unfused", api.decoder_chain, chain.launches)):
+            def cstep():
+                chain.h.copy_(h0, non_blocking=True)
+                run(chain)
+            for _ in range(cwarm):
+                cstep()
+            api.check()
+            ms, per = timed_steps(torch, stream, cstep, csteps, barrier)
+            api.check()
+            algo, codes = chain_bytes(shapes, M)
+            step_s = ms / csteps / 1e3
+            res[name] = {"tokens_per_s": M / step_s, "us_per_step": step_s * 1e6,
+                         "step_times": dist_summary(per), "frac_hbm": algo / step_s / 1e9 / hbm,
+                         "launches_per_step": launches + 1}
         out["chain_28L_M1"] = {
-            "M": M, "tokens_per_s": M / step_s, "us_per_step": step_s * 1e6,
-            "step_times": dist_summary(per), "algorithmic_bytes": algo,
-            "frac_hbm": algo / step_s / 1e9 / hbm, "launches_per_step": chain.launches + 1,
-            "note": "28 dependent layers from one token state (the +1 launch copies it in)"}
+            "M": M, **res, "algorithmic_bytes": algo,
+            "note": "28 dependent layers from one token state (the +1 launch copies it in); "
+                    "fused: one persistent launch, 112 grid-wide barriers; unfused: per layer "
+                    "4 sweeps and 4 element-wise launches"}
         del chain
     return out
 

@@ -317,6 +317,48 @@ TW_API int tw_decoder_chain(const tw_chain_layer *layers, int n_layers,
 TW_API int tw_chain_launches(const tw_chain_layer *layers, int n_layers);
 
 /*
+ * The same chain fused into one persistent kernel per group of up to 8
+ * tokens: all layers' stages run in one launch with grid-wide barriers
+ * between the dependent stages, and the steps between the projections (the
+ * activation quantisation, the rescale, the attention stand-in, the
+ * residual adds and SiLU * up) are done inside it.  Each stage's work is
+ * split over every SM along rows and k (partial sums are added with integer
+ * atomics, exact in any order); the code stream of later stages is fetched
+ * while the grid waits at a barrier.  Results are byte-identical to
+ * tw_decoder_chain (the same fp32 operations in the same order).
+ *
+ * tw_chain_plan_encode (HOST-ONLY) checks the layers' tables against `buf`
+ * exactly as tw_decoder_chain does and writes a plan of
+ * tw_chain_plan_bytes(n_layers) bytes into host memory, for the SM count of
+ * the current device; the caller copies it to device memory (64-byte
+ * aligned) and keeps both, the tables' buffers and `buf` alive while it is
+ * used.  head_dim must be a multiple of 4.
+ */
+TW_API size_t tw_chain_plan_bytes(int n_layers);
+TW_API int tw_chain_plan_encode(const tw_chain_layer *layers, int n_layers,
+                                const tw_chain_buffers *buf, void *plan, size_t plan_bytes);
+
+/* HOST-ONLY.  Scratch of tw_decoder_chain_fused for a host plan: 256 bytes
+ * of barrier counters, then three int32 sum buffers of 8 rows of the widest
+ * stage's outputs.  It must be zero-filled before its first use; every call
+ * leaves the counters zero again (after TW_ERR_TIMEOUT, zero it again). */
+TW_API size_t tw_chain_fused_workspace_bytes(const void *plan_host);
+
+/* HOST-ONLY.  Kernel launches of one tw_decoder_chain_fused call:
+ * ceil(M / 8). */
+TW_API int tw_chain_fused_launches(const void *plan_host);
+
+/*
+ * Run every layer of an encoded plan (host and device copies) on `stream`:
+ * ceil(M / 8) cooperative launches of one CTA per SM, each running all the
+ * layers for its tokens.  TW_ERR_UNSUPPORTED if the device has fewer SMs
+ * than the plan was encoded for.  Every barrier and copy wait is bounded:
+ * a wait that expires is reported by tw_check as TW_ERR_TIMEOUT.
+ */
+TW_API int tw_decoder_chain_fused(const void *plan_host, const void *plan_dev, void *ws,
+                                  size_t ws_bytes, tw_stream_t stream);
+
+/*
  * I8_S linear layer with fused bias and ReLU
  * ------------------------------------------
  * The int8 side of the model: the audio encoder keeps int8 weights and int8

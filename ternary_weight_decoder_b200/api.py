@@ -71,6 +71,11 @@ tw_debug_wait_timeout = _sig("tw_debug_wait_timeout", _int, [ctypes.c_uint64, _p
 tw_chain_workspace_bytes = _sig("tw_chain_workspace_bytes", _sz, [_p, _int])
 tw_decoder_chain = _sig("tw_decoder_chain", _int, [_p, _int, _p, _p, _sz, _p])
 tw_chain_launches = _sig("tw_chain_launches", _int, [_p, _int])
+tw_chain_plan_bytes = _sig("tw_chain_plan_bytes", _sz, [_int])
+tw_chain_plan_encode = _sig("tw_chain_plan_encode", _int, [_p, _int, _p, _p, _sz])
+tw_chain_fused_workspace_bytes = _sig("tw_chain_fused_workspace_bytes", _sz, [_p])
+tw_chain_fused_launches = _sig("tw_chain_fused_launches", _int, [_p])
+tw_decoder_chain_fused = _sig("tw_decoder_chain_fused", _int, [_p, _p, _p, _sz, _p])
 tw_pack_slice = _sig("tw_pack_slice", _int, [_p, _i64, _i64, _i64, _i64, _i64, _i64, _p, _sz, _p])
 tw_row_absmax = _sig("tw_row_absmax", _int, [_p, _i64, _i64, _p, _p])
 tw_quantize_act_given = _sig("tw_quantize_act_given", _int, [_p, _i64, _i64, _p, _p, _p, _p])
@@ -329,10 +334,27 @@ class DecoderChain:
         self.ws_bytes = int(tw_chain_workspace_bytes(c_layers, self.n_layers))
         self.ws = torch.zeros(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
         self.launches = int(tw_chain_launches(c_layers, self.n_layers))
+        # the fused plan (one persistent launch per 8 tokens)
+        pb = int(tw_chain_plan_bytes(self.n_layers))
+        self.plan_host = torch.empty(pb, dtype=torch.uint8).pin_memory() \
+            if torch.cuda.is_available() else torch.empty(pb, dtype=torch.uint8)
+        _raise(tw_chain_plan_encode(c_layers, self.n_layers, ctypes.byref(self.c_buf),
+                                    _ptr(self.plan_host), pb))
+        self.plan_dev = self.plan_host.to(device) if torch.cuda.is_available() else self.plan_host
+        self.fused_ws_bytes = int(tw_chain_fused_workspace_bytes(_ptr(self.plan_host)))
+        self.fused_ws = torch.zeros(max(self.fused_ws_bytes, 16), dtype=torch.uint8, device=device)
+        self.fused_launches = int(tw_chain_fused_launches(_ptr(self.plan_host)))
+
+
+def decoder_chain_fused(chain: DecoderChain, stream=None):
+    """Run every layer of ``chain`` in the fused persistent kernel."""
+    _raise(tw_decoder_chain_fused(_ptr(chain.plan_host), _ptr(chain.plan_dev), _ptr(chain.fused_ws),
+                                  chain.fused_ws_bytes, _stream(stream)))
 
 
 def decoder_chain(chain: DecoderChain, first: int = 0, count=None, stream=None):
-    """Run layers first .. first+count-1 of ``chain`` (all by default)."""
+    """Run layers first .. first+count-1 of ``chain`` (all by default), one
+    sweep per stage and the steps between them as their own launches."""
     count = chain.n_layers - first if count is None else count
     if not (0 <= first and count >= 1 and first + count <= chain.n_layers):
         raise ValueError("layer range outside the chain")

@@ -750,6 +750,156 @@ int tw_chain_launches(const tw_chain_layer *layers, int n_layers)
     return n;
 }
 
+size_t tw_chain_plan_bytes(int n_layers)
+{
+    if (n_layers < 1)
+        return 0;
+    return sizeof(tw::ChainPlanHeader) + (size_t)4 * n_layers * sizeof(tw::ChainStagePlan);
+}
+
+int tw_chain_plan_encode(const tw_chain_layer *layers, int n_layers, const tw_chain_buffers *buf,
+                         void *plan, size_t plan_bytes)
+{
+    t_last_error[0] = 0;
+    if (!layers || n_layers < 1 || !plan)
+        return fail(TW_ERR_NULL, "tw_chain_plan_encode: layers and plan are required");
+    if (plan_bytes < tw_chain_plan_bytes(n_layers))
+        return fail(TW_ERR_BUFSIZE, "tw_chain_plan_encode: plan buffer %zu < %zu bytes", plan_bytes,
+                    tw_chain_plan_bytes(n_layers));
+    if (int rc = check_chain_buffers(buf))
+        return rc;
+    const tw_chain_buffers &b = *buf;
+    if (b.head_dim % 4)
+        return fail(TW_ERR_SHAPE, "tw_chain_plan_encode: head_dim must be a multiple of 4");
+    ChainStage st[4];
+    chain_stages(b, st);
+    ChainRange ranges[9];
+    chain_ranges(b, ranges);
+    for (int l = 0; l < n_layers; ++l) {
+        const void *host[4], *dev[4];
+        layer_tables(layers[l], host, dev);
+        for (int k = 0; k < 4; ++k)
+            if (int rc = check_chain_stage(host[k], dev[k], st[k], b.M, l, ranges))
+                return rc;
+    }
+    // The grid: one CTA per SM of the current device (148 on a B200 when no
+    // device can be queried).
+    int dev_id = 0, sms = 148;
+    if (cudaGetDevice(&dev_id) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id) != cudaSuccess)
+        sms = 148;
+    cudaGetLastError();
+    memset(plan, 0, tw_chain_plan_bytes(n_layers));
+    auto *hdr = static_cast<tw::ChainPlanHeader *>(plan);
+    auto *stages = reinterpret_cast<tw::ChainStagePlan *>(hdr + 1);
+    int64_t max_ntot = 0, max_K = 0;
+    for (int l = 0; l < n_layers; ++l) {
+        const void *host[4], *dev[4];
+        layer_tables(layers[l], host, dev);
+        for (int k = 0; k < 4; ++k) {
+            const auto *th = static_cast<const tw::TableHeader *>(host[k]);
+            const auto *r = reinterpret_cast<const tw::DescRecord *>(th + 1);
+            tw::ChainStagePlan &sp = stages[4 * l + k];
+            sp.kind = k;
+            sp.nproj = th->count;
+            sp.K = (int32_t)r[0].K;
+            sp.nch = (int32_t)tw::ceil_div(r[0].K / tw::kTileK, tw::kChainChunk);
+            int64_t rb = 0, ntot = 0;
+            for (int i = 0; i < th->count; ++i) {
+                tw::ChainProj &pr = sp.proj[i];
+                pr.packed = r[i].packed;
+                pr.wscale = r[i].wscale;
+                pr.y = r[i].y;
+                pr.acc_out = r[i].acc_out;
+                pr.N = r[i].N;
+                pr.noff = ntot;
+                pr.rb_off = rb;
+                ntot += r[i].N;
+                rb += tw::ceil_div(r[i].N, tw::kTileRows);
+            }
+            sp.rb_total = rb;
+            sp.units = rb * sp.nch;
+            sp.ntot = ntot;
+            if (sp.units > INT32_MAX / 2)
+                return fail(TW_ERR_SHAPE, "tw_chain_plan_encode: stage too large");
+            max_ntot = std::max(max_ntot, ntot);
+            max_K = std::max(max_K, (int64_t)sp.K);
+        }
+    }
+    hdr->magic = tw::kChainPlanMagic;
+    hdr->n_stages = 4 * n_layers;
+    hdr->grid = sms;
+    hdr->n_layers = n_layers;
+    hdr->M = b.M;
+    hdr->hidden = b.hidden;
+    hdr->kv_dim = b.kv_dim;
+    hdr->head_dim = b.head_dim;
+    hdr->inter = b.inter;
+    hdr->h = b.h;
+    hdr->v = b.v;
+    hdr->a = b.a;
+    hdr->o = b.o;
+    hdr->h1 = b.h1;
+    hdr->g = b.g;
+    hdr->u = b.u;
+    hdr->act = b.act;
+    hdr->d = b.d;
+    hdr->max_ntot = max_ntot;
+    hdr->max_K = max_K;
+    hdr->chunk = tw::kChainChunk;
+    return TW_OK;
+}
+
+size_t tw_chain_fused_workspace_bytes(const void *plan_host)
+{
+    const auto *h = static_cast<const tw::ChainPlanHeader *>(plan_host);
+    if (!h || h->magic != tw::kChainPlanMagic)
+        return 0;
+    return (size_t)tw::chain_fused_ws_bytes(*h);
+}
+
+int tw_chain_fused_launches(const void *plan_host)
+{
+    const auto *h = static_cast<const tw::ChainPlanHeader *>(plan_host);
+    if (!h || h->magic != tw::kChainPlanMagic)
+        return 0;
+    return (int)tw::ceil_div(h->M, tw::kChainGroup);
+}
+
+int tw_decoder_chain_fused(const void *plan_host, const void *plan_dev, void *ws, size_t ws_bytes,
+                           tw_stream_t stream)
+{
+    t_last_error[0] = 0;
+    if (!plan_host || !plan_dev || !ws)
+        return fail(TW_ERR_NULL, "tw_decoder_chain_fused: host plan, device plan and ws required");
+    const auto *h = static_cast<const tw::ChainPlanHeader *>(plan_host);
+    if (h->magic != tw::kChainPlanMagic || h->n_stages < 4 || h->chunk != tw::kChainChunk)
+        return fail(TW_ERR_CORRUPT, "tw_decoder_chain_fused: plan was not produced by "
+                    "tw_chain_plan_encode");
+    if ((reinterpret_cast<uintptr_t>(plan_dev) & 63u) || !aligned16(ws))
+        return fail(TW_ERR_ALIGN, "tw_decoder_chain_fused: device plan 64-byte and ws 16-byte "
+                    "alignment required");
+    if (ws_bytes < tw_chain_fused_workspace_bytes(plan_host))
+        return fail(TW_ERR_BUFSIZE, "tw_decoder_chain_fused: workspace %zu < %zu bytes", ws_bytes,
+                    tw_chain_fused_workspace_bytes(plan_host));
+    uint32_t *err = nullptr;
+    if (int rc = err_word(&err))
+        return rc;
+    int dev_id = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev_id);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "device query");
+    if (sms < h->grid)
+        return fail(TW_ERR_UNSUPPORTED, "tw_decoder_chain_fused: plan encoded for %d SMs, device "
+                    "has %d", h->grid, sms);
+    tw::ChainLaunch L{static_cast<const tw::ChainPlanHeader *>(plan_dev), h,
+                      static_cast<uint8_t *>(ws)};
+    e = tw::launch_chain_fused(L, err, kWaitNs, stream);
+    return e == cudaSuccess ? TW_OK : cuda_fail(e, "fused chain launch");
+}
+
 int tw_decoder_chain(const tw_chain_layer *layers, int n_layers, const tw_chain_buffers *buf,
                      void *ws, size_t ws_bytes, tw_stream_t stream)
 {

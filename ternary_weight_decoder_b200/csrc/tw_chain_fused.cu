@@ -1,0 +1,583 @@
+// tw_chain_fused.cu — the decoder-layer chain as one persistent kernel per
+// group of up to 8 tokens: every layer's four dependent stages (q/k/v, o,
+// gate/up, down) with grid-wide barriers between them, the activation
+// quantisation, the rescale, the attention stand-in, both residual adds and
+// SiLU(gate) * up fused into the stages.  (The decoder layer of the
+// Qwen2.5-1.5B LM: "VibeVoice-ASR-BitNet-ONNX" model page, "Layout"; every
+// weight is read once per token: "The Paper Says ARM Support" post, "What
+// the model is trying to do".)
+//
+// Launch: cooperative, one CTA per SM (all co-resident, so the barriers
+// cannot deadlock), NW warps each.
+//
+// A stage's work is split into units of one 16-row block x up to 6 code
+// tiles (768 k) of one projection -- split-K, so that the down projection's
+// 96 long row blocks spread over every warp of the grid.  The CTAs take
+// equal ranges of units, their warps every NW-th unit.  Each warp keeps a
+// ring of S slots that it fills with 1-D bulk copies of its next units'
+// codes, across stage boundaries: the weights do not depend on the
+// activations, so the code stream runs ahead while the grid waits.  A unit's
+// partial sums D = sum_k (c + 1) q are added into an int32 buffer of the
+// stage with integer atomics (exact in any order).
+//
+// Stage s's prologue (every CTA, every thread, after the barrier): read the
+// previous stage's sums, rescale them exactly as the single-projection
+// epilogue does, y = ((float)(D - sum q) * (amax/127)) * wscale, apply the
+// step between the stages -- q/k/v -> a = v repeated per query-head group;
+// o -> h1 = h + o; gate/up -> SiLU(g) * u; down -> h' = h1 + d -- and
+// quantise the result per token (amax, 127/amax, rint) into shared memory
+// for the stage's MMAs.  Each CTA computes the whole input rows (they are a
+// few KB at decode sizes) but writes only its slice of the materialised
+// buffers (q, k, v, a, o, h1, g, u, act, d, h and any acc_out).  The sums
+// live in three rotating buffers: stage s adds into buffer s mod 3, the
+// prologue of s + 1 reads it, and the prologue of s - 1 cleared the buffer
+// of s + 1 -- so every buffer is zero before the first atomic reaches it.
+//
+// Every value is computed with the same fp32 operations as the unfused
+// chain (the same rounding), so the two give the same bytes.  Every wait is
+// bounded: a barrier or ring wait that expires sets the timeout bit, stops
+// the block and drains its copies.
+#include <cstring>
+
+#include "tw_device.cuh"
+#include "tw_gemv.cuh"
+#include "tw_internal.h"
+
+namespace tw {
+namespace {
+
+constexpr int kNW = 16;                    // warps per CTA (all consume and quantise)
+constexpr int kCT = kChainChunk;           // code tiles per unit (one ring slot)
+constexpr int kS = 3;                      // ring slots per warp
+constexpr int kThreadsCh = kNW * 32;
+constexpr int kSlotBytes = kCT * kTileBytes;
+constexpr uint64_t kDrainNsCh = 1000000000ull;
+
+struct ChainParams {
+    const ChainPlanHeader *plan;
+    uint8_t *ws;
+    int m0, mg;                 // token group [m0, m0 + mg)
+    int xstride;                // bytes per activation row in shared memory (max_K + 64)
+    WaitCtl ctl;
+};
+
+__device__ __forceinline__ const ChainStagePlan *stage_of(const ChainPlanHeader *h, int s)
+{
+    return reinterpret_cast<const ChainStagePlan *>(h + 1) + s;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Grid-wide barrier number `k` (1, 2, ...): every CTA's writes before it are
+// visible to every CTA after it.  False when the wait timed out (the block
+// must stop).
+__device__ bool grid_barrier(uint32_t *ctr, uint32_t k, const ChainParams &p, volatile int *abort_flag)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ctr, 1u);
+        const uint32_t target = k * gridDim.x;
+        if (!*abort_flag && ld_acquire_u32(ctr) < target) {
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_u32(ctr) < target) {
+                if (*abort_flag)
+                    break;
+                if (globaltimer_ns() - t0 > p.ctl.timeout_ns) {
+                    atomicOr(p.ctl.err, EFLAG_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    return !*abort_flag;
+}
+
+// A warp's walk over its work units, stage after stage.
+struct UnitIter {
+    int s, n_stages;
+    int u, hi;                  // current unit, end of this CTA's range in stage s
+    int nch, KT, nproj;
+    int rb_off[4];
+    const uint8_t *packed[3];
+    bool valid;
+
+    __device__ void enter(const ChainPlanHeader *h, int stage, int w)
+    {
+        valid = false;
+        for (s = stage; s < n_stages; ++s) {
+            const ChainStagePlan *st = stage_of(h, s);
+            const int units = (int)st->units;
+            const int c = blockIdx.x, G = gridDim.x;
+            const int lo = (int)((int64_t)units * c / G);
+            hi = (int)((int64_t)units * (c + 1) / G);
+            u = lo + w;
+            if (u < hi) {
+                nch = st->nch;
+                KT = st->K / kTileK;
+                nproj = st->nproj;
+                for (int q = 0; q < 3; ++q) {
+                    rb_off[q] = (int)st->proj[q].rb_off;
+                    packed[q] = st->proj[q].packed;
+                }
+                rb_off[3] = (int)st->rb_total;
+                for (int q = nproj; q < 3; ++q)
+                    rb_off[q + 1] = rb_off[3];
+                valid = true;
+                return;
+            }
+        }
+    }
+    __device__ void next(const ChainPlanHeader *h, int w)
+    {
+        u += kNW;
+        if (u >= hi)
+            enter(h, s + 1, w);
+    }
+    // (projection, row block in it, first tile, tiles) of the current unit
+    __device__ void where(int &q, int &rbl, int &kt0, int &n) const
+    {
+        const int rbg = u / nch, kc = u - rbg * nch;
+        q = rbg >= rb_off[1] ? (rbg >= rb_off[2] ? 2 : 1) : 0;
+        rbl = rbg - rb_off[q];
+        kt0 = kc * kCT;
+        n = min(kCT, KT - kt0);
+    }
+    __device__ void issue(uint32_t dst, uint32_t bar) const
+    {
+        int q, rbl, kt0, n;
+        where(q, rbl, kt0, n);
+        const uint8_t *src = packed[q] + ((int64_t)rbl * KT + kt0) * (int64_t)kTileBytes;
+        mbar_arrive_expect_tx(bar, (uint32_t)(n * kTileBytes));
+        bulk_g2s(dst, src, (uint32_t)(n * kTileBytes), bar);
+    }
+};
+
+__device__ __forceinline__ float rescale1(int D, int qs, float sa, float ws)
+{
+    return __fmul_rn(__fmul_rn((float)(D - qs), sa), ws);
+}
+
+__device__ __forceinline__ float silu_mul1(float z, float u)
+{
+    return __fmul_rn(__fdiv_rn(z, __fadd_rn(1.0f, expf(-z))), u);
+}
+
+// The stage input x(m, 4i .. 4i+3) of the prologue of stage kind `kind`
+// (layer's first stage when first_layer), from the previous stage's sums
+// `sum` (row stride prev->ntot) with the previous input's scales.  The
+// helpers below also return the materialised values the slice writers need.
+struct Prev {
+    const int32_t *sum;         // previous stage's sums (token-major, ntot per row)
+    int64_t ntot;
+    const ChainStagePlan *st;   // previous stage
+    const float *sa;            // its input's amax/127 per token (shared memory)
+    const int *qs;              // its input's sum(q) per token (shared memory)
+    const float *ws;            // its projections' wscale (shared memory)
+};
+
+__device__ __forceinline__ int4 ldcg4i(const int32_t *p) { return __ldcg(reinterpret_cast<const int4 *>(p)); }
+__device__ __forceinline__ float4 ldcg4f(const float *p) { return __ldcg(reinterpret_cast<const float4 *>(p)); }
+
+// y (fp32) of column j .. j+3 of projection q of the previous stage, token m.
+__device__ __forceinline__ float4 prev_y4(const Prev &P, int q, int m, int64_t j)
+{
+    const float ws = P.ws[q];
+    const int4 D = ldcg4i(P.sum + (int64_t)m * P.ntot + P.st->proj[q].noff + j);
+    return make_float4(rescale1(D.x, P.qs[m], P.sa[m], ws), rescale1(D.y, P.qs[m], P.sa[m], ws),
+                       rescale1(D.z, P.qs[m], P.sa[m], ws), rescale1(D.w, P.qs[m], P.sa[m], ws));
+}
+
+__device__ __forceinline__ float4 add4(float4 a, float4 b)
+{
+    return make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z), __fadd_rn(a.w, b.w));
+}
+
+// x of stage `kind` at token m (chain row m0 + m), columns 4i .. 4i + 3.
+__device__ __forceinline__ float4 stage_x4(const ChainPlanHeader *h, int kind, bool first_layer,
+                                           const Prev &P, int m, int mrow, int64_t i)
+{
+    const int64_t k = 4 * i;
+    switch (kind) {
+    case kStageQKV:
+        if (first_layer)
+            return ldcg4f(h->h + mrow * h->hidden + k);
+        // h' = h1 + d of the previous layer
+        return add4(ldcg4f(h->h1 + mrow * h->hidden + k), prev_y4(P, 0, m, k));
+    case kStageO: {
+        // a = v, each KV head repeated for the query heads of its group
+        const int64_t group = (h->hidden / h->head_dim) / (h->kv_dim / h->head_dim);
+        const int64_t head = k / h->head_dim, c = k - head * h->head_dim;
+        return prev_y4(P, 2, m, (head / group) * h->head_dim + c);
+    }
+    case kStageGU:
+        return add4(ldcg4f(h->h + mrow * h->hidden + k), prev_y4(P, 0, m, k));
+    default: {   // kStageDown: SiLU(g) * u
+        const float4 g = prev_y4(P, 0, m, k);
+        const float4 u = prev_y4(P, 1, m, k);
+        return make_float4(silu_mul1(g.x, u.x), silu_mul1(g.y, u.y), silu_mul1(g.z, u.z),
+                           silu_mul1(g.w, u.w));
+    }
+    }
+}
+
+__device__ __forceinline__ uint32_t quant4c(float4 v, float scale, bool zero, int &sum)
+{
+    int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+    if (!zero) {
+        q0 = min(max(__float2int_rn(__fmul_rn(v.x, scale)), -128), 127);
+        q1 = min(max(__float2int_rn(__fmul_rn(v.y, scale)), -128), 127);
+        q2 = min(max(__float2int_rn(__fmul_rn(v.z, scale)), -128), 127);
+        q3 = min(max(__float2int_rn(__fmul_rn(v.w, scale)), -128), 127);
+    }
+    sum += q0 + q1 + q2 + q3;
+    return (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) | ((uint32_t)(q2 & 0xff) << 16) |
+           ((uint32_t)(q3 & 0xff) << 24);
+}
+
+// Write this CTA's slice of an [mg x width] materialised buffer: element e
+// of the slice has value fn(m, j) for m = e / width, j = e % width (width a
+// multiple of 4; written 4 at a time).
+template <class F>
+__device__ __forceinline__ void write_slice(float *dst, int64_t width, int mg, int m0, F fn)
+{
+    const int64_t n4 = (int64_t)mg * width / 4;
+    const int64_t lo = n4 * blockIdx.x / gridDim.x, hi = n4 * (blockIdx.x + 1) / gridDim.x;
+    for (int64_t e = lo + threadIdx.x; e < hi; e += kThreadsCh) {
+        const int m = (int)(e / (width / 4));
+        const int64_t j = 4 * (e - (int64_t)m * (width / 4));
+        *reinterpret_cast<float4 *>(dst + (int64_t)(m0 + m) * width + j) = fn(m, j);
+    }
+}
+
+// This CTA's slice of the previous stage's integer outputs into acc_out.
+__device__ __forceinline__ void write_acc_slice(const Prev &P, int q, int mg, int m0)
+{
+    const ChainProj &pr = P.st->proj[q];
+    if (!pr.acc_out)
+        return;
+    const int64_t width = pr.N;
+    const int64_t n = (int64_t)mg * width;
+    const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
+    for (int64_t e = lo + threadIdx.x; e < hi; e += kThreadsCh) {
+        const int m = (int)(e / width);
+        const int64_t j = e - (int64_t)m * width;
+        pr.acc_out[(int64_t)(m0 + m) * width + j] =
+            __ldcg(P.sum + (int64_t)m * P.ntot + pr.noff + j) - P.qs[m];
+    }
+}
+
+// Materialise the outputs of the previous stage (every projection's y and
+// acc_out) and the step values of this prologue, each CTA its slice.
+__device__ void materialise(const ChainPlanHeader *h, int kind, bool first_layer, bool final_phase,
+                            const Prev &P, int mg, int m0)
+{
+    if (P.st) {
+        for (int q = 0; q < P.st->nproj; ++q) {
+            write_slice(P.st->proj[q].y, P.st->proj[q].N, mg, m0,
+                        [&](int m, int64_t j) { return prev_y4(P, q, m, j); });
+            write_acc_slice(P, q, mg, m0);
+        }
+    }
+    if (final_phase || (kind == kStageQKV && !first_layer)) {
+        // h' = h1 + d
+        write_slice(h->h, h->hidden, mg, m0, [&](int m, int64_t j) {
+            return add4(ldcg4f(h->h1 + (int64_t)(m0 + m) * h->hidden + j), prev_y4(P, 0, m, j));
+        });
+    } else if (kind == kStageO) {
+        write_slice(h->a, h->hidden, mg, m0, [&](int m, int64_t j) {
+            return stage_x4(h, kStageO, false, P, m, m0 + m, j / 4);
+        });
+    } else if (kind == kStageGU) {
+        write_slice(h->h1, h->hidden, mg, m0, [&](int m, int64_t j) {
+            return stage_x4(h, kStageGU, false, P, m, m0 + m, j / 4);
+        });
+    } else if (kind == kStageDown) {
+        write_slice(h->act, h->inter, mg, m0, [&](int m, int64_t j) {
+            return stage_x4(h, kStageDown, false, P, m, m0 + m, j / 4);
+        });
+    }
+}
+
+__global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__ ChainParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const ChainPlanHeader *h = p.plan;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int mg = p.mg, m0 = p.m0;
+
+    // Layout: rings | activation rows (kChainGroup x xstride) | scales | reductions | barriers
+    const int ring_bytes = kNW * kS * kSlotBytes;
+    uint8_t *xbuf = smem + ring_bytes;
+    float *sa_s = reinterpret_cast<float *>(xbuf + kChainGroup * p.xstride);   // [8] this stage
+    int *qs_s = reinterpret_cast<int *>(sa_s + kChainGroup);                   // [8]
+    float *scale_s = reinterpret_cast<float *>(qs_s + kChainGroup);            // [8] 127/amax
+    float *psa_s = scale_s + kChainGroup;                                      // [8] previous stage
+    int *pqs_s = reinterpret_cast<int *>(psa_s + kChainGroup);                 // [8]
+    float *pws_s = reinterpret_cast<float *>(pqs_s + kChainGroup);             // [4] its wscales
+    float *red_f = pws_s + 4 + 4;                                              // [kNW][8]
+    int *red_i = reinterpret_cast<int *>(red_f + kNW * kChainGroup);           // [kNW][8]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(
+        (reinterpret_cast<uintptr_t>(red_i + kNW * kChainGroup) + 15) & ~uintptr_t(15));
+    int *abort_p = reinterpret_cast<int *>(bars + kNW * kS);
+    volatile int *abort_flag = abort_p;
+    const uint32_t bar_ring = smem_u32(bars);
+
+    uint32_t *ctr = reinterpret_cast<uint32_t *>(p.ws);
+    const int64_t buf_ints = (kChainGroup * h->max_ntot * 4 + 255) / 256 * 64;
+    int32_t *sums = reinterpret_cast<int32_t *>(p.ws + 256);
+    auto sum_buf = [&](int s) { return sums + (int64_t)(s % 3) * buf_ints; };
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNW * kS; ++i)
+            mbar_init(bar_ring + 8 * i, 1);
+        *abort_p = 0;
+        fence_barrier_init();
+    }
+    // token rows at or past mg stay zero for the whole launch
+    for (int i = threadIdx.x; i < kChainGroup * p.xstride / 16; i += kThreadsCh)
+        reinterpret_cast<uint4 *>(xbuf)[i] = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+
+    // ---- the code ring of this warp (lane 0 issues), primed across stages
+    const uint32_t ring_w0 = smem_u32(smem) + warp * kS * kSlotBytes;
+    const uint32_t ring_w = ring_w0 + lane * 16;
+    const uint32_t bar_w = bar_ring + 8 * warp * kS;
+    UnitIter prod, cons;
+    prod.n_stages = h->n_stages;
+    prod.enter(h, 0, warp);
+    cons = prod;
+    int issued = 0, consumed = 0;
+    for (int s = 0; s < kS && prod.valid; ++s) {
+        if (lane == 0)
+            prod.issue(ring_w0 + s * kSlotBytes, bar_w + 8 * s);
+        prod.next(h, warp);
+        ++issued;
+    }
+    int cslot = 0;
+    uint32_t cphase = 0;
+
+    // ---- clear the first stage's sums, then the first barrier
+    {
+        const int64_t n = (int64_t)kChainGroup * h->max_ntot;
+        const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
+        for (int64_t e = lo + threadIdx.x; e < hi; e += kThreadsCh)
+            sum_buf(0)[e] = 0;
+    }
+    uint32_t nbar = 1;
+    bool ok = grid_barrier(ctr, nbar++, p, abort_flag);
+
+    Prev P;
+    P.st = nullptr;
+    P.sum = nullptr;
+    P.ntot = 0;
+    P.sa = psa_s;
+    P.qs = pqs_s;
+    P.ws = pws_s;
+
+    for (int s = 0; s <= h->n_stages && ok; ++s) {
+        const bool final_phase = s == h->n_stages;
+        const ChainStagePlan *st = final_phase ? nullptr : stage_of(h, s);
+        const int kind = final_phase ? -1 : st->kind;
+        const bool first_layer = s < 4;
+        if (s > 0) {
+            P.st = stage_of(h, s - 1);
+            P.sum = sum_buf(s - 1);
+            P.ntot = P.st->ntot;
+            if (threadIdx.x < P.st->nproj)
+                pws_s[threadIdx.x] = __ldg(P.st->proj[threadIdx.x].wscale);
+            __syncthreads();
+        }
+
+        // ---- prologue 1: materialise slices; clear the sums of stage s + 1
+        materialise(h, kind, first_layer, final_phase, P, mg, m0);
+        if (final_phase)
+            break;
+        if (s + 1 < h->n_stages) {
+            const int64_t n = (int64_t)kChainGroup * stage_of(h, s + 1)->ntot;
+            const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
+            int32_t *b = sum_buf(s + 1);
+            for (int64_t e = lo + threadIdx.x; e < hi; e += kThreadsCh)
+                b[e] = 0;
+        }
+
+        // ---- prologue 2: this stage's input rows, quantised into shared memory
+        const int64_t K = st->K, K4 = K / 4;
+        {
+            // per token: amax over the row, then 127/amax (one token at a time
+            // keeps a single running value per thread)
+            for (int m = 0; m < mg; ++m) {
+                float a = 0.f;
+                for (int64_t i = threadIdx.x; i < K4; i += kThreadsCh) {
+                    const float4 v = stage_x4(h, kind, first_layer, P, m, m0 + m, i);
+                    a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+                }
+#pragma unroll
+                for (int o = 16; o; o >>= 1)
+                    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+                if (lane == 0)
+                    red_f[warp * kChainGroup + m] = a;
+            }
+            __syncthreads();
+            if (threadIdx.x < mg) {
+                float a = 0.f;
+                for (int w = 0; w < kNW; ++w)
+                    a = fmaxf(a, red_f[w * kChainGroup + threadIdx.x]);
+                sa_s[threadIdx.x] = __fdiv_rn(a, 127.f);
+                scale_s[threadIdx.x] = a == 0.f ? 0.f : __fdiv_rn(127.f, a);
+            }
+            __syncthreads();
+            // quantise the rows into shared memory, with sum(q) per token
+            for (int m = 0; m < mg; ++m) {
+                const float sc = scale_s[m];
+                const bool zero = sc == 0.f;
+                uint32_t *row = reinterpret_cast<uint32_t *>(xbuf + m * p.xstride);
+                int sq = 0;
+                for (int64_t i = threadIdx.x; i < K4; i += kThreadsCh)
+                    row[i] = quant4c(stage_x4(h, kind, first_layer, P, m, m0 + m, i), sc, zero, sq);
+#pragma unroll
+                for (int o = 16; o; o >>= 1)
+                    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                if (lane == 0)
+                    red_i[warp * kChainGroup + m] = sq;
+            }
+            __syncthreads();
+            if (threadIdx.x < mg) {
+                int q = 0;
+                for (int w = 0; w < kNW; ++w)
+                    q += red_i[w * kChainGroup + threadIdx.x];
+                qs_s[threadIdx.x] = q;
+            }
+            __syncthreads();
+            // this stage's scales serve the next prologue's rescale
+            if (threadIdx.x < mg) {
+                psa_s[threadIdx.x] = sa_s[threadIdx.x];
+                pqs_s[threadIdx.x] = qs_s[threadIdx.x];
+            }
+        }
+
+        // ---- this warp's units of stage s
+        const int g = lane >> 2, t = lane & 3;
+        const uint32_t xrow = smem_u32(xbuf) + g * p.xstride + 16 * t;
+        const uint32_t xr[1] = {xrow};
+        int32_t *sb = sum_buf(s);
+        const int64_t ntot = st->ntot;
+        while (cons.valid && cons.s == s) {
+            if (!mbar_wait(bar_w + 8 * cslot, cphase, p.ctl, abort_flag)) {
+                ok = false;
+                break;
+            }
+            int q, rbl, kt0, n;
+            cons.where(q, rbl, kt0, n);
+            int acc[1][4][4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    acc[0][a][i] = 0;
+            chunk_mma<1, kCT>(acc, ring_w + cslot * kSlotBytes, xr, (uint32_t)(kt0 * kTileK), n);
+            __syncwarp();
+            if (prod.valid) {
+                if (lane == 0) {
+                    fence_proxy_async_smem();
+                    prod.issue(ring_w0 + cslot * kSlotBytes, bar_w + 8 * cslot);
+                }
+                prod.next(h, warp);
+                ++issued;
+            }
+            ++consumed;
+            if (++cslot == kS) {
+                cslot = 0;
+                cphase ^= 1u;
+            }
+            // partial sums of rows 16 rbl + g (+8), tokens 2t (+1)
+            const int64_t N = st->proj[q].N, noff = st->proj[q].noff;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int tok = 2 * t + (i & 1);
+                const int64_t row = (int64_t)rbl * kTileRows + g + 8 * (i >> 1);
+                if (tok < mg && row < N) {
+                    const int D = acc[0][0][i] + (acc[0][1][i] >> 2) + (acc[0][2][i] >> 4) +
+                                  (acc[0][3][i] >> 6);
+                    atomicAdd(sb + tok * ntot + noff + row, D);
+                }
+            }
+            cons.next(h, warp);
+        }
+        if (!ok)
+            *abort_flag = 1;
+        ok = grid_barrier(ctr, nbar++, p, abort_flag) && ok;
+    }
+
+    if (!ok) {
+        // Drain: every copy this warp still has in flight lands before exit.
+        WaitCtl drain = p.ctl;
+        drain.timeout_ns = kDrainNsCh;
+        for (int i = consumed; i < issued; ++i)
+            mbar_wait(bar_w + 8 * (i % kS), (uint32_t)((i / kS) & 1), drain, nullptr);
+    }
+    __syncthreads();
+    // The last block to finish clears the counters for the next call.
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(ctr + 1, 1u) == gridDim.x - 1) {
+            ctr[0] = 0u;
+            ctr[1] = 0u;
+            __threadfence();
+        }
+    }
+}
+
+}  // namespace
+
+int chain_fused_smem(int64_t max_K)
+{
+    const int xstride = (int)(max_K + 64);
+    return kNW * kS * kSlotBytes + kChainGroup * xstride + 4 * 5 * kChainGroup + 32 +
+           8 * kNW * kChainGroup + 16 + 8 * kNW * kS + 64;
+}
+
+cudaError_t launch_chain_fused(const ChainLaunch &L, uint32_t *err, uint64_t timeout_ns,
+                               cudaStream_t stream)
+{
+    const ChainPlanHeader &hh = *L.host;
+    const int smem = chain_fused_smem(hh.max_K);
+    cudaError_t e = cudaFuncSetAttribute(k_chain, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+        return e;
+    ChainParams p;
+    memset(&p, 0, sizeof(p));
+    p.plan = L.plan;
+    p.ws = L.ws;
+    p.xstride = (int)(hh.max_K + 64);
+    p.ctl.err = err;
+    p.ctl.timeout_ns = timeout_ns;
+    for (int64_t m0 = 0; m0 < hh.M; m0 += kChainGroup) {
+        p.m0 = (int)m0;
+        p.mg = (int)(hh.M - m0 < kChainGroup ? hh.M - m0 : kChainGroup);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)hh.grid);
+        cfg.blockDim = dim3(kThreadsCh);
+        cfg.dynamicSmemBytes = (size_t)smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: the barriers need it
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, k_chain, p);
+        if (e != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace tw

@@ -56,6 +56,58 @@ static_assert(sizeof(TableHeader) == 64, "header size");
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// ------------------------------------------------- fused decoder-layer chain
+// The plan of tw_decoder_chain_fused (host-encoded by tw_chain_plan_encode,
+// copied to the device by the caller): a header, then one stage per
+// (layer, {qkv, o, gate/up, down}).
+constexpr uint32_t kChainPlanMagic = 0x54574332u;  // "TWC2"
+constexpr int kChainGroup = 8;                     // tokens per fused launch
+constexpr int kChainChunk = 6;                     // code tiles per work unit
+enum ChainKind : int32_t { kStageQKV = 0, kStageO = 1, kStageGU = 2, kStageDown = 3 };
+
+struct alignas(64) ChainProj {
+    const uint8_t *packed;
+    const float *wscale;
+    float *y;              // [M x N] output
+    int32_t *acc_out;      // [M x N] int32 output, or null
+    int64_t N;
+    int64_t noff;          // first column of this projection in the stage's sums
+    int64_t rb_off;        // first 16-row block of this projection in the stage
+    int64_t pad;
+};
+static_assert(sizeof(ChainProj) == 64, "chain projection");
+
+struct alignas(64) ChainStagePlan {
+    int32_t kind, nproj, K, nch;   // nch: work units (chunks) per row block
+    int64_t rb_total, units, ntot; // row blocks, units (row block x chunk), sum of N
+    int64_t pad[3];
+    ChainProj proj[3];
+};
+static_assert(sizeof(ChainStagePlan) == 256, "chain stage");
+
+struct alignas(64) ChainPlanHeader {
+    uint32_t magic;
+    int32_t n_stages, grid, n_layers;
+    int64_t M, hidden, kv_dim, head_dim, inter;
+    float *h, *v, *a, *o, *h1, *g, *u, *act, *d;
+    int64_t max_ntot, max_K, chunk;
+};
+static_assert(sizeof(ChainPlanHeader) % 64 == 0, "chain header");
+
+struct ChainLaunch {
+    const ChainPlanHeader *plan;   // device copy
+    const ChainPlanHeader *host;   // host copy (sizes)
+    uint8_t *ws;
+};
+// Scratch of the fused chain: 256 bytes of counters (zero between calls),
+// then three int32 sum buffers of kChainGroup x max_ntot.
+inline int64_t chain_fused_ws_bytes(const ChainPlanHeader &h)
+{
+    return 256 + 3 * ((kChainGroup * h.max_ntot * 4 + 255) / 256 * 256);
+}
+cudaError_t launch_chain_fused(const ChainLaunch &L, uint32_t *err, uint64_t timeout_ns,
+                               cudaStream_t stream);
+
 // Element-wise steps of the decoder-layer chain (tw_chain.cu).
 cudaError_t launch_gqa_expand(const float *v, float *a, int64_t M, int64_t kv_dim,
                               int64_t hidden, int64_t head_dim, cudaStream_t stream);

@@ -333,3 +333,29 @@ def test_chain_binding_owns_the_tensors_it_points_at(lib):
     del x
     gc.collect()
     assert r() is not None and t.count == 1
+
+
+def test_chain_fused_plan_host_checks(lib):
+    """The fused chain's plan passes the same table checks, sizes its
+    scratch from the widest stage and launches once per 8 tokens."""
+    from ternary_weight_decoder_b200 import api
+    import ctypes
+    for M, launches in ((1, 1), (8, 1), (9, 2), (20, 3)):
+        layers, cbuf, keep = _fake_chain(M=M, n_layers=2)
+        nb = api.tw_chain_plan_bytes(2)
+        assert nb >= 4 * 2 * 256
+        plan = np.zeros(nb, np.uint8)
+        assert api.tw_chain_plan_encode(layers, 2, ctypes.byref(cbuf), plan.ctypes.data, nb) == 0, \
+            api.tw_last_error()
+        assert api.tw_chain_fused_launches(plan.ctypes.data) == launches
+        # counters + three sum buffers of 8 rows of the widest stage (gate/up: 2 x 512)
+        assert api.tw_chain_fused_workspace_bytes(plan.ctypes.data) == 256 + 3 * 8 * 1024 * 4
+        assert api.tw_chain_plan_encode(layers, 2, ctypes.byref(cbuf), plan.ctypes.data, nb - 1) == 4
+    # a table that does not match the buffers is refused here too
+    layers, cbuf, keep = _fake_chain(tweak=lambda l, st, a: st == "o" and _tw(a, 0, x=a[0].x + 0x100000))
+    plan = np.zeros(api.tw_chain_plan_bytes(2), np.uint8)
+    assert api.tw_chain_plan_encode(layers, 2, ctypes.byref(cbuf), plan.ctypes.data, plan.size) == 2
+    # a plan that was not encoded is refused before any launch
+    assert api.tw_decoder_chain_fused(np.zeros(512, np.uint8).ctypes.data, 0x7e0000000000,
+                                      0x7c0000000000, 1 << 20, None) == 8
+    assert api.tw_chain_fused_workspace_bytes(np.zeros(512, np.uint8).ctypes.data) == 0

@@ -144,3 +144,57 @@ def test_chain_zero_weights_return_input(dev, api):
     api.check()
     assert np.array_equal(_np(chain.h), h0)
     assert not torch.any(chain.act) and not torch.any(chain.d)
+
+
+def _snapshot(chain, acc):
+    names = ("h", "q", "k", "v", "a", "o", "h1", "g", "u", "act", "d")
+    return ({n: getattr(chain, n).clone() for n in names},
+            {k: t.clone() for k, t in acc.items()})
+
+
+@pytest.mark.parametrize("M,dims", [(1, SMALL), (5, SMALL), (16, SMALL), (3, SMALL_G1),
+                                    (1, QWEN), (9, QWEN), (20, QWEN)])
+def test_chain_fused_matches_unfused(dev, api, M, dims):
+    """The fused persistent chain gives the bytes of the unfused chain (which
+    the stagewise test pins to the oracle): every buffer and every
+    projection's integer outputs of the last layer, twice in a row (the
+    barrier counters and sum buffers are reset by each call)."""
+    import torch
+    n_layers = 3
+    chain, _, acc = _build(api, dev, M, dims, n_layers, seed=500 + M)
+    h0 = G.to_dev(synth.activations(510 + M, 0, M, dims[0]), dev)
+    chain.h.copy_(h0)
+    _poison(chain, acc)
+    api.decoder_chain(chain)
+    api.check()
+    want, want_acc = _snapshot(chain, acc)
+    for _ in range(2):
+        chain.h.copy_(h0)
+        _poison(chain, acc)
+        api.decoder_chain_fused(chain)
+        api.check()
+        got, got_acc = _snapshot(chain, acc)
+        for n in want:
+            assert torch.equal(got[n], want[n]), f"fused chain M={M}: buffer {n} differs"
+        for k in want_acc:
+            if k[0] == n_layers - 1:
+                assert torch.equal(got_acc[k], want_acc[k]), f"fused chain M={M}: acc {k} differs"
+
+
+def test_chain_fused_zero_weights_return_input(dev, api):
+    hidden, kv, hd, inter = SMALL
+    shapes = _shapes(hidden, kv, inter)
+    layers = []
+    for _ in range(2):
+        layer = {}
+        for name in PROJ:
+            N, K = shapes[name]
+            packed, _, wscale = G.ternarize_gpu(np.zeros((N, K), np.float32), dev)
+            layer[name] = (packed, wscale)
+        layers.append(layer)
+    chain = api.DecoderChain(layers, 2, hidden, kv, hd, inter, dev)
+    h0 = synth.activations(8, 0, 2, hidden)
+    chain.h.copy_(G.to_dev(h0, dev))
+    api.decoder_chain_fused(chain)
+    api.check()
+    assert np.array_equal(_np(chain.h), h0)
