@@ -214,13 +214,13 @@ TW_API size_t tw_sweep_table_bytes(int count);
 TW_API int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M,
                           void *table, size_t table_bytes);
 
-/* Scratch needed by tw_decoder_projection_sweep for an encoded HOST table;
- * 0 for prefill, whose callers pass the quantised rows in the descriptors.
+/* Scratch needed by tw_decoder_projection_sweep for an encoded HOST table.
  * For decode (M <= 32) it holds 256 bytes of work counters, then the
  * quantised rows of every projection (room for 8, 16 or 32 token rows of K
- * bytes) and their scales.  It must be zero-filled before its first use
- * with a table; every call leaves the counters zero again (after
- * TW_ERR_TIMEOUT, zero it again). */
+ * bytes) and their scales; for more tokens (whose callers pass the
+ * quantised rows in the descriptors) only the 256 bytes of work counters.
+ * It must be zero-filled before its first use with a table; every call
+ * leaves the counters zero again (after TW_ERR_TIMEOUT, zero it again). */
 TW_API size_t tw_sweep_workspace_bytes(const void *table_host);
 
 /*
@@ -229,7 +229,8 @@ TW_API size_t tw_sweep_workspace_bytes(const void *table_host);
  * launch of the register (mma.sync) kernel -- more only when M*K of the
  * widest projection does not fit shared memory and the tokens are split
  * into groups -- and for 16 < M <= 32 one launch of the tensor-core decode
- * kernel.  Prefill (M > 32): one grouped tensor-core launch.
+ * kernel.  More tokens: one persistent tensor-core launch with the weights
+ * in tensor memory (units of 128 weight rows x 128 tokens).
  *   table_host  the host table written by tw_sweep_table_encode (read for the
  *               launch configuration: count, M, sizes);
  *   table_dev   the caller's device copy of the same bytes (64-byte aligned),

@@ -530,9 +530,12 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
             // 128-row code boxes of the tensor-core sweep.  Without a CUDA
             // driver (-1) a decode table is still encoded for its sizes; the
             // sweep refuses it.
+            // (code boxes of 128 rows for the decode and weights-in-TMEM
+            // kernels, 256 rows for the expanded-weights GEMM)
             int rc = decode ? 0 : tw::encode_xq_tmap(s.xq, M, s.K, r.tmap_xq);
             if (!rc)
-                rc = tw::encode_codes_tmap(r.packed, s.N, s.K, decode ? 8 : 16, r.tmap_codes);
+                rc = tw::encode_codes_tmap(r.packed, s.N, s.K, decode || TW_SWEEP_MID ? 8 : 16,
+                                           r.tmap_codes);
             if (rc && !(decode && rc == -1))
                 return fail(TW_ERR_CUDA, "descriptor %d: cuTensorMapEncodeTiled failed (%d)", d,
                             rc);
@@ -562,7 +565,8 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
     });
     int64_t units = 0;
     for (int i = 0; i < count; ++i) {
-        order[i].units = (int32_t)tw::ceil_div(recs[order[i].d].N, 128);
+        const int64_t n = recs[order[i].d].N;
+        order[i].units = (int32_t)(decode ? tw::ceil_div(n, 128) : tw::mid_units(M, n));
         order[i].unit_begin = units;
         units += order[i].units;
     }
@@ -574,7 +578,9 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
     hdr->total_rb = rb;
     hdr->total_units = units;
     hdr->total_ptiles = ptiles;
-    hdr->ws_bytes = decode ? ws_off + 256 * (int64_t)count : 0;
+    // decode: counters, rows and scales; more tokens: the unit counters of the
+    // weights-in-TMEM kernel
+    hdr->ws_bytes = decode ? ws_off + 256 * (int64_t)count : (TW_SWEEP_MID ? tw::kWsCtrBytes : 0);
     hdr->max_K = max_K;
     hdr->total_cost = cost;
     return TW_OK;
@@ -612,6 +618,24 @@ int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, v
     uint32_t *err = nullptr;
     if (int rc = err_word(&err))
         return rc;
+    if (hdr->M > tw::kDecodeMaxM && TW_SWEEP_MID) {
+        if (ws_bytes < (size_t)hdr->ws_bytes || !ws)
+            return fail(TW_ERR_BUFSIZE, "sweep workspace %zu < %lld bytes", ws_bytes,
+                        (long long)hdr->ws_bytes);
+        if (!aligned16(ws))
+            return fail(TW_ERR_ALIGN, "sweep workspace must be 16-byte aligned");
+        const auto *recs_dev = reinterpret_cast<const tw::DescRecord *>(
+            static_cast<const tw::TableHeader *>(table_dev) + 1);
+        tw::MidLaunch P{};
+        P.table = recs_dev;
+        P.order = reinterpret_cast<const tw::UnitOrder *>(recs_dev + hdr->count);
+        P.count = hdr->count;
+        P.M = hdr->M;
+        P.total_units = hdr->total_units;
+        P.ctr = reinterpret_cast<uint32_t *>(ws);
+        cudaError_t e = tw::launch_mid(P, err, kWaitNs, stream);
+        return e == cudaSuccess ? TW_OK : cuda_fail(e, "prefill sweep launch");
+    }
     if (hdr->M > tw::kDecodeMaxM) {
         tw::PrefillLaunch P{};
         P.table = reinterpret_cast<const tw::DescRecord *>(

@@ -196,6 +196,25 @@ inline int64_t round128(int64_t b) { return (b + 127) / 128 * 128; }
 cudaError_t launch_decode(const DecodeLaunch &L, uint32_t *err, uint64_t timeout_ns,
                           cudaStream_t stream);
 
+// Weights-in-tensor-memory GEMM for more than 32 tokens (tw_mid.cu): units
+// of 128 weight rows x 128 tokens, claimed from counters in 256 bytes of
+// scratch (zero between calls).  Its tables carry 128-row code boxes.
+struct MidLaunch {
+    const DescRecord *table;  // device records
+    const UnitOrder *order;   // device copy of the order (units: row tiles x token tiles)
+    int count;
+    int64_t M, total_units;
+    uint32_t *ctr;
+};
+cudaError_t launch_mid(const MidLaunch &L, uint32_t *err, uint64_t timeout_ns, cudaStream_t stream);
+// Work units of one projection on that path: ceil(N / 128) x ceil(M / 128).
+int64_t mid_units(int64_t M, int64_t N);
+// Which kernel runs a sweep of more than 32 tokens: the weights-in-TMEM
+// GEMM (1) or the expanded-weights GEMM of tw_prefill.cu (0).
+#ifndef TW_SWEEP_MID
+#define TW_SWEEP_MID 1
+#endif
+
 struct PrefillLaunch {
     const DescRecord *table;  // device records (or null: use `single`)
     int count;

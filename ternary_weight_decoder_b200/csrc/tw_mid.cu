@@ -1,0 +1,444 @@
+// tw_mid.cu — ternary GEMM for more than 32 tokens with the weights held
+// in tensor memory: the 128-row side of tcgen05.mma kind::i8 is a tile of
+// ternary codes expanded to int8 {0, 1, 2} (= code + 1) straight into TMEM,
+// and the N side is up to 128 int8 token rows loaded by TMA from xq.
+//
+// What it computes, per projection (per-tensor ternary weights, s =
+// 1/mean|W|: "VibeVoice-ASR-BitNet-ONNX" model page, Quantization table; the
+// prefill length is the audio frame count plus the prompt, one frame per
+// 3200 samples of 24 kHz audio: same page, "Layout"):
+//   D[n, m] = sum_k (code[n, k] + 1) * xq[m, k]           (int32, in TMEM)
+//   acc     = D - qsum[m],   y[m, n] = ((float)acc * (amax[m] / 127)) * mean|W|
+//
+// Why weights on the TMEM side: the expanded weights never pass through
+// shared memory, which carries only the 2-bit codes and the token tile.  Per
+// 128-k stage that is 4 KB of codes and 16 KB of tokens written by TMA and
+// read once by the expansion or the MMAs, against 48 KB of operand reads
+// plus a 32 KB expanded tile when the weights are the shared-memory operand.
+//
+// Work unit: one 128-row tile of one projection times one 128-token tile,
+// over all of K; units are claimed from a counter, projections of larger K
+// first.  Per 128-column k tile (a stage):
+//   * warp 0 loads the 8 x 512 B code tiles (one 3-D TMA box) and the
+//     128 x 128 B token tile (one 2-D TMA box of xq, 128-byte swizzled,
+//     tokens past M read as zero) into a ring of L shared-memory stages;
+//   * eight expansion warps (two sets of four, one warp per TMEM lane
+//     quarter, alternating stages) turn each 16-byte lane slot of the code
+//     tile into 16 registers holding code + 1 for 4 consecutive k each, in
+//     the natural k order of the MMA's K (each register's 16 source bits
+//     come from the word of lane 2(u & 1) + t/2 of the row's quad, fetched
+//     with a shuffle), and store them to one of 8 TMEM A slots
+//     (tcgen05.st 16x256b: column c of a slot holds k = 4c .. 4c + 3);
+//   * warp 1 issues four MMAs of K = 32 into the unit's accumulator (N =
+//     128 columns, one of two) and commits them to the stage's empty
+//     barrier, which frees the stage and, eight stages later, the A slot;
+//   * four epilogue warps (one per lane quarter: 32 weight rows each) read
+//     the accumulator 32 tokens at a time and store y, each store 32
+//     consecutive rows of one token.
+// Every wait is bounded; on a timeout the block stops, drains its copies and
+// MMAs, frees its tensor memory and returns.
+#include <cstring>
+
+#include "tw_device.cuh"
+#include "tw_internal.h"
+#include "tw_tc.cuh"
+
+namespace tw {
+namespace {
+
+constexpr int kNTok = 128;                       // tokens per unit (MMA N)
+constexpr int kASlotsM = 8;
+constexpr int kRingM = 8;                        // unit-info entries
+constexpr int kThreadsM = 14 * 32;
+constexpr int kCodeBytesM = 8 * kTileBytes;       // 128 rows x 128 k = 4 KB
+constexpr int kTokBytesM = kNTok * 128;           // 16 KB
+constexpr int kStageM = kCodeBytesM + kTokBytesM;
+constexpr int kTmemColsM = 512;
+constexpr int kDCol0M = 256;                     // two accumulators after 8 A slots
+constexpr int kMiscM = 2048;
+constexpr uint64_t kDrainNsM = 1000000000ull;
+
+struct UnitM {
+    int d, rt, tk, live;
+};
+
+struct ProjM {
+    int64_t N;
+    float *y;
+    int32_t *acc_out;
+    const float *amax;
+    const int32_t *qsum;
+    float wscale;
+    int KT;
+};
+static_assert(sizeof(ProjM) == 48, "projection cache entry");
+
+struct MidParams {
+    const DescRecord *table;
+    const UnitOrder *order;   // projections by K, descending, with their first unit
+    int count;
+    int M;
+    int tiles_m;              // token tiles of 128
+    int64_t total_units;
+    uint32_t *ctr;            // [0] claim counter, [1] finished blocks
+    WaitCtl ctl;
+};
+
+template <int L>
+constexpr int smem_mid(int count) { return 1024 + L * kStageM + kMiscM + (16 + (int)sizeof(ProjM)) * count; }
+
+// int8 x int8 -> int32, K-major, M = 128, N = 128.
+constexpr uint32_t kIdescMid = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kNTok >> 3) << 17) |
+                               ((128u >> 4) << 24);
+
+__device__ UnitM locate_unit_m(const MidParams &p, const UnitOrder *order, int64_t uid)
+{
+    int lo = 0, hi = p.count - 1;  // last entry with unit_begin <= uid
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (order[mid].unit_begin <= uid)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    const int local = (int)(uid - order[lo].unit_begin);
+    return UnitM{order[lo].d, local / p.tiles_m, local % p.tiles_m, 1};
+}
+
+template <int L>
+__global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ MidParams p)
+{
+    static_assert(L >= kASlotsM && L % 2 == 0, "load stages");
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    auto codes_s = [&](int s) { return base + (uint32_t)(s * kStageM); };
+    auto tok_s = [&](int s) { return base + (uint32_t)(s * kStageM + kCodeBytesM); };
+    uint8_t *misc = smem_raw + (base - raw) + L * kStageM;
+    const uint32_t bar0 = smem_u32(misc);
+    const uint32_t b_full = bar0, b_empty = b_full + 8 * L, b_afull = b_empty + 8 * L;
+    const uint32_t b_ufull = b_afull + 8 * kASlotsM, b_uempty = b_ufull + 8 * kRingM;
+    const uint32_t b_dfull = b_uempty + 8 * kRingM, b_dempty = b_dfull + 16;
+    const uint32_t b_drain = b_dempty + 16;
+    int *stage_stop = reinterpret_cast<int *>(misc + 1024);
+    UnitM *ring = reinterpret_cast<UnitM *>(misc + 1024 + 4 * 32);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 1024 + 4 * 32 + 16 * kRingM);
+    int *abort_p = reinterpret_cast<int *>(tmem_slot + 1);
+    volatile int *abort_flag = abort_p;
+    UnitOrder *order_s = reinterpret_cast<UnitOrder *>(misc + kMiscM);
+    ProjM *proj_s = reinterpret_cast<ProjM *>(misc + kMiscM + 16 * p.count);
+    for (int i = threadIdx.x; i < p.count; i += kThreadsM) {
+        order_s[i] = p.order[i];
+        const DescRecord &r = p.table[i];
+        proj_s[i] = ProjM{r.N, r.y, r.acc_out, r.amax, r.qsum, __ldg(r.wscale), (int)(r.K / kTileK)};
+    }
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < L; ++s) {
+            mbar_init(b_full + 8 * s, 1);
+            mbar_init(b_empty + 8 * s, 1);   // the MMA commit of the stage
+        }
+        for (int a = 0; a < kASlotsM; ++a)
+            mbar_init(b_afull + 8 * a, 4);   // the 4 expansion warps of the stage's set
+        for (int j = 0; j < kRingM; ++j) {
+            mbar_init(b_ufull + 8 * j, 1);
+            mbar_init(b_uempty + 8 * j, 4);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(b_dfull + 8 * b, 1);
+            mbar_init(b_dempty + 8 * b, 4);
+        }
+        mbar_init(b_drain, 1);
+        *abort_p = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1)
+        tmem_alloc(smem_u32(tmem_slot), kTmemColsM);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            auto resolve = [&](uint32_t uid) {
+                return uid < p.total_units ? locate_unit_m(p, order_s, uid) : UnitM{0, 0, 0, 0};
+            };
+            // claims run two units ahead (the counter's round trip is hidden)
+            uint32_t claim1 = atomicAdd(p.ctr, 1u);
+            uint32_t claim2 = atomicAdd(p.ctr, 1u);
+            for (int j = 0; ok; ++j) {
+                const UnitM u = resolve(claim1);
+                claim1 = claim2;
+                const int ju = j % kRingM;
+                if (j >= kRingM &&
+                    !mbar_wait(b_uempty + 8 * ju, (uint32_t)((j / kRingM - 1) & 1), p.ctl, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                ring[ju] = u;
+                mbar_arrive(b_ufull + 8 * ju);
+                if (!u.live)
+                    break;
+                claim2 = atomicAdd(p.ctr, 1u);
+                const void *tmap_c = p.table[u.d].tmap_codes;   // addresses only
+                const void *tmap_x = p.table[u.d].tmap_xq;
+                const int KT = proj_s[u.d].KT;
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = (int)(it % L);
+                    if (it >= L && !mbar_wait(b_empty + 8 * s, (it / L - 1) & 1u, p.ctl, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    stage_stop[s] = 0;
+                    mbar_arrive_expect_tx(b_full + 8 * s, (uint32_t)kStageM);
+                    tma_load_3d(codes_s(s), tmap_c, 0, kt, 8 * u.rt, b_full + 8 * s);
+                    tma_load_2d(tok_s(s), tmap_x, kt * 128, u.tk * kNTok, b_full + 8 * s);
+                }
+            }
+            // One stop stage for each expansion set.
+            for (int e = 0; e < 2 && ok; ++e, ++it) {
+                const int s = (int)(it % L);
+                if (it >= L && !mbar_wait(b_empty + 8 * s, (it / L - 1) & 1u, p.ctl, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                stage_stop[s] = 1;
+                mbar_arrive(b_full + 8 * s);
+            }
+            // Drain: every copy this thread issued lands before the block exits.
+            WaitCtl drain = p.ctl;
+            drain.timeout_ns = kDrainNsM;
+            for (uint32_t j = it > (uint32_t)L ? it - L : 0; j < it; ++j)
+                mbar_wait(b_full + 8 * (int)(j % L), (j / L) & 1u, drain, nullptr);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int j = 0; ok; ++j) {
+                const int ju = j % kRingM;
+                if (!mbar_wait(b_ufull + 8 * ju, (uint32_t)((j / kRingM) & 1), p.ctl, abort_flag))
+                    break;
+                const UnitM u = ring[ju];
+                if (!u.live)
+                    break;
+                const int buf = j & 1;
+                if (j >= 2 &&
+                    !mbar_wait(b_dempty + 8 * buf, (uint32_t)((j / 2 - 1) & 1), p.ctl, abort_flag))
+                    break;
+                tc_fence_after();
+                const uint32_t d0 = tmem + kDCol0M + (uint32_t)(buf * kNTok);
+                const int KT = proj_s[u.d].KT;
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    // The expansion of this stage waited for its bytes (codes and
+                    // tokens) before it arrived here.
+                    const int a = (int)(it % kASlotsM);
+                    if (!mbar_wait(b_afull + 8 * a, (it / kASlotsM) & 1u, p.ctl, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int s = (int)(it % L);
+                    const uint64_t bd = sdesc_k_sw128(tok_s(s));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)  // +32 bytes of K = +2 in the address field
+                        mma_i8_ts(d0, tmem + (uint32_t)(32 * a + 8 * kk), bd + 2 * kk, kIdescMid,
+                                  (kt > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(b_empty + 8 * s);   // frees stage s, and A slot a for stage it + 8
+                }
+                if (!ok)
+                    break;
+                mma_commit(b_dfull + 8 * buf);
+            }
+            // All MMAs issued by this thread complete before TMEM is freed.
+            mma_commit(b_drain);
+            WaitCtl drain = p.ctl;
+            drain.timeout_ns = kDrainNsM;
+            mbar_wait(b_drain, 0, drain, nullptr);
+        }
+        __syncwarp();
+    } else if (warp < 6) {
+        // ------------------------------------------------------ epilogue
+        const int quarter = warp & 3;
+        for (int j = 0;; ++j) {
+            const int ju = j % kRingM;
+            if (!mbar_wait(b_ufull + 8 * ju, (uint32_t)((j / kRingM) & 1), p.ctl, abort_flag))
+                break;
+            const UnitM u = ring[ju];
+            if (!u.live)
+                break;
+            const ProjM pr = proj_s[u.d];
+            const int buf = j & 1;
+            const int64_t row = (int64_t)u.rt * 128 + 32 * quarter + lane;
+            const int m_base = u.tk * kNTok;
+            // this lane's token of each group of 32: scale and sum(q), loaded
+            // before the accumulator is ready
+            float sa_l[kNTok / 32];
+            int qs_l[kNTok / 32];
+#pragma unroll
+            for (int c = 0; c < kNTok / 32; ++c) {
+                const int m = m_base + 32 * c + lane;
+                sa_l[c] = m < p.M ? __fdiv_rn(__ldg(pr.amax + m), 127.f) : 0.f;
+                qs_l[c] = m < p.M ? __ldg(pr.qsum + m) : 0;
+            }
+            if (!mbar_wait(b_dfull + 8 * buf, (uint32_t)((j / 2) & 1), p.ctl, abort_flag))
+                break;
+            tc_fence_after();
+            const uint32_t dq = tmem + kDCol0M + (uint32_t)(buf * kNTok) + ((uint32_t)(32 * quarter) << 16);
+            int nvalid = p.M - m_base;
+            nvalid = nvalid > kNTok ? kNTok : nvalid;
+            const bool row_ok = row < pr.N;
+#pragma unroll 1
+            for (int c = 0; c < kNTok / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(dq + 32 * c, v);   // waits for the load
+                if (c == kNTok / 32 - 1) {
+                    // the accumulator has been read: it may be reused
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(b_dempty + 8 * buf);
+                }
+                if (32 * c >= nvalid)
+                    continue;   // (uniform across the warp)
+#pragma unroll
+                for (int n = 0; n < 32; ++n) {
+                    const float sa = __shfl_sync(0xffffffffu, sa_l[c], n);
+                    const int qs = __shfl_sync(0xffffffffu, qs_l[c], n);
+                    const int m = 32 * c + n;
+                    if (row_ok && m < nvalid) {
+                        const int a = (int)v[n] - qs;
+                        const int64_t o = (int64_t)(m_base + m) * pr.N + row;
+                        pr.y[o] = __fmul_rn(__fmul_rn((float)a, sa), pr.wscale);
+                        if (pr.acc_out)
+                            pr.acc_out[o] = a;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(b_uempty + 8 * ju);
+        }
+    } else {
+        // ------------------------------------------------------ expansion
+        // Lane (g, t) holds the 16-byte lane slot of rows g, g + 8: word j is
+        // row g + 8 (j & 1), k = 64 (j >> 1) + 16 t + 0..15, the code of
+        // k0 + 4s + b at bit 8b + 2s.  The 16x256b store gives this lane
+        // columns 8u + 2t + (i & 1) of rows g + 8 (i >> 1) (register 4u + i);
+        // column c is k = 4c .. 4c + 3, i.e. k0 = 32u + 8t + 4(i & 1), which
+        // lives in word 2(u >> 1) + (i >> 1) of lane 4g + 2(u & 1) + (t >> 1),
+        // slot s = 2(t & 1) + (i & 1).
+        const int quarter = warp & 3, set = (warp - 6) >> 2;
+        const int g = lane >> 2, t = lane & 3;
+        const uint32_t m3 = 0x03030303u;
+        const int sh0 = 4 * (t & 1);   // 2 s for i & 1 == 0
+        for (uint32_t it = set;; it += 2) {
+            const int s = (int)(it % L);
+            if (!mbar_wait(b_full + 8 * s, (it / L) & 1u, p.ctl, abort_flag))
+                break;
+            if (stage_stop[s])
+                break;
+            // A slot it % 8 is free once the MMAs of stage it - 8 have completed.
+            if (it >= (uint32_t)kASlotsM &&
+                !mbar_wait(b_empty + 8 * (int)((it - kASlotsM) % L), ((it - kASlotsM) / L) & 1u, p.ctl,
+                           abort_flag))
+                break;
+            const uint32_t aslot = it % kASlotsM;
+            tc_fence_after();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 w = lds128(codes_s(s) + (2 * quarter + h) * kTileBytes + lane * 16);
+                uint32_t r[16];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int src = 4 * g + 2 * (u & 1) + (t >> 1);
+#pragma unroll
+                    for (int rh = 0; rh < 2; ++rh) {
+                        const int jw = 2 * (u >> 1) + rh;   // uniform across the warp
+                        const uint32_t mine = jw == 0 ? w.x : jw == 1 ? w.y : jw == 2 ? w.z : w.w;
+                        const uint32_t word = __shfl_sync(0xffffffffu, mine, src);
+                        r[4 * u + 2 * rh + 0] = (word >> sh0) & m3;
+                        r[4 * u + 2 * rh + 1] = (word >> (sh0 + 2)) & m3;
+                    }
+                }
+                tmem_st16x256b_x4(tmem + 32 * aslot + ((uint32_t)(32 * quarter + 16 * h) << 16), r);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(b_afull + 8 * aslot);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        tmem_dealloc(tmem, kTmemColsM);
+    // The last block to finish clears the counters for the next call.
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.ctr + 1, 1u) == gridDim.x - 1) {
+            p.ctr[0] = 0u;
+            p.ctr[1] = 0u;
+            __threadfence();
+        }
+    }
+}
+
+template <int L>
+cudaError_t launch_mid_l(const MidParams &p, int grid, cudaStream_t stream)
+{
+    const int smem = smem_mid<L>(p.count);
+    cudaError_t e = cudaFuncSetAttribute(k_mid<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+        return e;
+    k_mid<L><<<(unsigned)grid, kThreadsM, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int64_t mid_units(int64_t M, int64_t N)
+{
+    return ((N + 127) / 128) * ((M + kNTok - 1) / kNTok);
+}
+
+cudaError_t launch_mid(const MidLaunch &L, uint32_t *err, uint64_t timeout_ns, cudaStream_t stream)
+{
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess)
+        return e;
+    MidParams p;
+    memset(&p, 0, sizeof(p));
+    p.table = L.table;
+    p.order = L.order;
+    p.count = L.count;
+    p.M = (int)L.M;
+    p.tiles_m = (int)((L.M + kNTok - 1) / kNTok);
+    p.total_units = L.total_units;
+    p.ctr = L.ctr;
+    p.ctl.err = err;
+    p.ctl.timeout_ns = timeout_ns;
+    const int64_t grid64 = L.total_units < sms ? L.total_units : sms;
+    const int grid = (int)(grid64 < 1 ? 1 : grid64);
+    constexpr int kLimit = 227 * 1024;
+    if (smem_mid<10>(p.count) <= kLimit)
+        return launch_mid_l<10>(p, grid, stream);
+    if (smem_mid<8>(p.count) <= kLimit)
+        return launch_mid_l<8>(p, grid, stream);
+    return cudaErrorInvalidValue;   // too many projections for the caches
+}
+
+}  // namespace tw

@@ -352,3 +352,36 @@ def test_argument_errors(dev, api):
     y = api.ternary_linear(x, packed, wscale, 16)
     api.check()
     assert not y.cpu().numpy().any()
+
+
+@pytest.mark.parametrize("M", [33, 64, 127, 128, 129, 200, 255, 300])
+def test_sweep_mid_m(dev, api, M):
+    """More than 32 tokens (the weights-in-tensor-memory kernel): every
+    token-tile tail, projections whose N is not a multiple of 128 (the last
+    128-row unit partial), several K, twice in a row (the unit counters are
+    left zero for the next call)."""
+    import torch
+    shapes = [(200, 256), (128, 1536), (17, 384), (385, 640), (256, 2048), (1, 128)]
+    descs, keep = [], []
+    for i, (N, K) in enumerate(shapes):
+        W = _weights(N, K, 5000 + 10 * M + i)
+        x = _acts(M, K, 6000 + 10 * M + i)
+        packed, _, wscale = G.ternarize_gpu(W, dev)
+        xq, amax, qsum = api.quantize_act(G.to_dev(x, dev))
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+        acc = torch.full((M, N), int(POISON_I32), dtype=torch.int32, device=dev)
+        descs.append(dict(xq=xq, amax=amax, qsum=qsum, packed=packed, wscale=wscale, y=y,
+                          acc_out=acc, N=N, K=K))
+        keep.append((W, x))
+    table = api.SweepTable(descs, M, device=dev)
+    for _ in range(2):
+        api.decoder_projection_sweep(table)
+        api.check()
+        for d, (W, x) in zip(descs, keep):
+            codes, mean = orc.ternarize(W)
+            ref = orc.ternary_linear(x, codes, mean)
+            assert (d["acc_out"].cpu().numpy() == ref["acc"]).all(), (M, d["N"], d["K"])
+            G.assert_y_close(d["y"].cpu().numpy(), ref["y"], f"M={M} N={d['N']} K={d['K']}")
+        for d in descs:
+            d["y"].fill_(float("nan"))
+            d["acc_out"].fill_(int(POISON_I32))
