@@ -124,13 +124,13 @@ struct UnitIter {
                 nch = st->nch;
                 KT = st->K / kTileK;
                 nproj = st->nproj;
+                // rb_off[q] = first row block of projection q; entries past the
+                // stage's projections hold the total, so where() never picks them
                 for (int q = 0; q < 3; ++q) {
-                    rb_off[q] = (int)st->proj[q].rb_off;
+                    rb_off[q] = q < nproj ? (int)st->proj[q].rb_off : (int)st->rb_total;
                     packed[q] = st->proj[q].packed;
                 }
                 rb_off[3] = (int)st->rb_total;
-                for (int q = nproj; q < 3; ++q)
-                    rb_off[q + 1] = rb_off[3];
                 valid = true;
                 return;
             }

@@ -16,10 +16,12 @@
 //              4-stage ring (k past K and rows past M or N read as zero);
 //   warp 1     MMA issuer and TMEM owner: four tcgen05.mma kind::i8 (K = 32
 //              each) per stage into one of two 128-column int32 accumulators;
-//   warps 2-5  epilogue, one TMEM lane quarter (32 tokens) each: per 32
-//              columns, tcgen05.ld, rescale + bias + ReLU, a 128-byte-
-//              swizzled 4 KB staging buffer (four per warp, in turn), and a
-//              TMA store of the 32 x 32 box (clipped at M and N).  When N is
+//   warps 2-9  epilogue, two per TMEM lane quarter (32 tokens), each taking
+//              half of the tile's columns: per 32 columns, tcgen05.ld,
+//              rescale + bias + ReLU (the tile's bias staged in shared
+//              memory), a 128-byte-swizzled 4 KB staging buffer (three per
+//              warp, in turn), and a TMA store of the 32 x 32 box (clipped
+//              at M and N).  When N is
 //              not a multiple of 4 (the output's row pitch is then not a
 //              multiple of 16 bytes), the warp stores the staged box with
 //              coalesced row writes instead.
@@ -42,16 +44,17 @@ namespace {
 constexpr int kBM = 128;                       // tokens per tile (MMA M)
 constexpr int kBN = 128;                       // weight rows per tile (MMA N)
 constexpr int kBK = 128;                       // bytes of k per stage
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kABytes = kBM * kBK;             // 16 KB
 constexpr int kBBytes = kBN * kBK;             // 16 KB
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 8;
 constexpr int kThreads = (2 + kEpiWarps) * 32;
-constexpr int kEpiBufs = 4;                    // staging buffers per epilogue warp
+constexpr int kEpiBufs = 3;                    // staging buffers per epilogue warp
 constexpr int kBoxBytes = 32 * 32 * 4;         // one 32 x 32 fp32 box
 constexpr int kTmemCols = 2 * kBN;
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiWarps * kEpiBufs * kBoxBytes + 1024;
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiWarps * kEpiBufs * kBoxBytes + 1024 +
+                           kEpiWarps * 64 * 4;
 constexpr uint64_t kDrainNs = 1000000000ull;
 
 struct alignas(64) I8Params {
@@ -99,6 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_i8_gemm(const __grid_constant__
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 512);
     int *abort_p = reinterpret_cast<int *>(misc + 520);
     volatile int *abort_flag = abort_p;
+    float *bias_s = reinterpret_cast<float *>(misc + 1024);   // [kEpiWarps][64]: per warp
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -198,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_i8_gemm(const __grid_constant__
         // ------------------------------------------------------ epilogue
         const int quarter = warp & 3;          // TMEM lanes 32q .. 32q + 31
         const int ew = warp - 2;
+        const int half = ew >> 2;              // columns [64 half, 64 half + 64) of the tile
         const uint32_t stg = stg0 + (uint32_t)(ew * kEpiBufs * kBoxBytes);
         float *stg_f = reinterpret_cast<float *>(gen_base + (stg - base));
         const float sw = __fdiv_rn(__ldg(p.amax_w), 127.f);
@@ -210,14 +215,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_i8_gemm(const __grid_constant__
             const int64_t m0 = mi * kBM + 32 * quarter;   // first token row of this warp
             const int64_t m = m0 + lane;
             const float sa = m < p.M ? __fdiv_rn(__ldg(p.amax_x + m), 127.f) : 0.f;
+            // this half's bias columns into the warp's own shared buffer
+            // (before the wait; the warp's previous tile is done with it)
+            float *bias_t = bias_s + 64 * ew;
+            {
+                const int64_t n = nj * kBN + 64 * half + lane;
+                bias_t[lane] = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.f;
+                bias_t[lane + 32] = (p.bias && n + 32 < p.N) ? __ldg(p.bias + n + 32) : 0.f;
+            }
+            __syncwarp();
             if (!mbar_wait(b_tfull + 8 * ab, (uint32_t)((tt / 2) & 1), p.ctl, abort_flag))
                 break;
             tc_fence_after();
-            for (int cc = 0; cc < kBN / 32; ++cc) {
+            for (int hc = 0; hc < 2; ++hc) {
+                const int cc = 2 * half + hc;
                 const int64_t n0 = nj * kBN + 32 * cc;
                 uint32_t v[32];
                 tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(ab * kBN + 32 * cc), v);
-                if (cc == kBN / 32 - 1) {
+                if (hc == 1) {
                     // the accumulator has been read: release it to the MMA warp
                     tc_fence_before();
                     __syncwarp();
@@ -226,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_i8_gemm(const __grid_constant__
                 }
                 if (n0 >= p.N || m0 >= p.M)
                     continue;   // (uniform across the warp)
-                const float bl = (p.bias && n0 + lane < p.N) ? __ldg(p.bias + n0 + lane) : 0.f;
+                const float4 *bias4 = reinterpret_cast<const float4 *>(bias_t + 32 * hc);
                 for (int pass = 0; pass < (p.acc_out ? 2 : 1); ++pass) {
                     const int b = nbox % kEpiBufs;
                     const uint32_t box = stg + (uint32_t)(b * kBoxBytes);
@@ -239,13 +254,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_i8_gemm(const __grid_constant__
                     for (int c = 0; c < 8; ++c) {
                         float4 f;
                         float *fp = reinterpret_cast<float *>(&f);
+                        const float4 b4 = bias4[c];   // (one broadcast read)
+                        const float *bp = reinterpret_cast<const float *>(&b4);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int j = 4 * c + e;
                             const int a = (int)v[j];
                             if (pass == 0) {
-                                float yv = __fadd_rn(__fmul_rn(__fmul_rn((float)a, sa), sw),
-                                                     __shfl_sync(0xffffffffu, bl, j));
+                                float yv = __fadd_rn(__fmul_rn(__fmul_rn((float)a, sa), sw), bp[e]);
                                 if (p.relu && yv < 0.f)
                                     yv = 0.f;
                                 fp[e] = yv;

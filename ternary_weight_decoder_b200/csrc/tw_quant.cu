@@ -1,6 +1,7 @@
 // tw_quant.cu — stand-alone per-token int8 activation quantisation by absmax
-// (the input of the prefill path).  The decode path fuses the same
-// arithmetic into its own kernel.
+// (the input of the prefill path and of the I8_S layer): one warp per row
+// for rows of up to 1024 elements, one block per row above.  The decode path
+// fuses the same arithmetic into its own kernel.
 //
 // amax = max|x| (exact), scale = 127.0f / amax (IEEE fp32 division),
 // q = clamp(rint(x * scale), -128, 127) with one fp32 multiply and
@@ -80,12 +81,63 @@ __global__ void __launch_bounds__(kQThreads) k_quantize(const float *__restrict_
     }
 }
 
+// One warp per token row, the row held in registers (K <= 32 * 4 * kWarpRegs):
+// for short rows a block per row would leave most of its threads idle.
+constexpr int kWarpRegs = 8;   // float4 per lane
+__global__ void __launch_bounds__(kQThreads) k_quantize_warp(const float *__restrict__ x, int64_t M,
+                                                             int64_t K, int8_t *__restrict__ xq,
+                                                             float *__restrict__ amax_out,
+                                                             int32_t *__restrict__ qsum_out)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t m = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
+    if (m >= M)
+        return;   // (whole warps)
+    const float4 *row = reinterpret_cast<const float4 *>(x + m * K);
+    uint32_t *qrow = reinterpret_cast<uint32_t *>(xq + m * K);
+    const int K4 = (int)(K / 4);
+    float4 v[kWarpRegs];
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < kWarpRegs; ++i) {
+        const int idx = lane + 32 * i;
+        v[i] = idx < K4 ? __ldg(row + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+        a = fmaxf(a, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    const bool zero = (a == 0.f);
+    const float scale = zero ? 0.f : __fdiv_rn(127.f, a);
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < kWarpRegs; ++i) {
+        const int idx = lane + 32 * i;
+        if (idx < K4)
+            qrow[idx] = quant4(v[i], scale, zero, sum);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) {
+        amax_out[m] = a;
+        if (qsum_out)
+            qsum_out[m] = sum;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const float *x, int64_t M, int64_t K, int8_t *xq, float *amax,
                             int32_t *qsum, cudaStream_t stream)
 {
-    k_quantize<<<(unsigned)M, kQThreads, 0, stream>>>(x, K, xq, amax, qsum);
+    if (K <= 32 * 4 * kWarpRegs) {
+        const int64_t rows_per_block = kQThreads / 32;
+        k_quantize_warp<<<(unsigned)((M + rows_per_block - 1) / rows_per_block), kQThreads, 0, stream>>>(
+            x, M, K, xq, amax, qsum);
+    } else {
+        k_quantize<<<(unsigned)M, kQThreads, 0, stream>>>(x, K, xq, amax, qsum);
+    }
     return cudaGetLastError();
 }
 
