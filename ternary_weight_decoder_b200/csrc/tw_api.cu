@@ -127,7 +127,7 @@ int run_prefill_single(const int8_t *xq, const float *amax, const int32_t *qsum,
     r.K = K;
     int rc = tw::encode_xq_tmap(xq, M, K, r.tmap_xq);
     if (!rc)
-        rc = tw::encode_codes_tmap(r.packed, N, K, 16, r.tmap_codes);
+        rc = tw::encode_codes_tmap(r.packed, N, K, 16, 1, r.tmap_codes);
     if (rc)
         return fail(TW_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", rc);
     tw::PrefillLaunch L{};
@@ -535,6 +535,7 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
             int rc = decode ? 0 : tw::encode_xq_tmap(s.xq, M, s.K, r.tmap_xq);
             if (!rc)
                 rc = tw::encode_codes_tmap(r.packed, s.N, s.K, decode || TW_SWEEP_MID ? 8 : 16,
+                                           decode ? tw::kTcGroup : TW_SWEEP_MID ? tw::kMidGroup : 1,
                                            r.tmap_codes);
             if (rc && !(decode && rc == -1))
                 return fail(TW_ERR_CUDA, "descriptor %d: cuTensorMapEncodeTiled failed (%d)", d,

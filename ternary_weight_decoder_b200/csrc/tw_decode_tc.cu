@@ -14,24 +14,27 @@
 // Work unit: one 128-row tile of one projection (8 row blocks of the packed
 // layout) over all of K.  Units are claimed from a counter in the scratch,
 // projections of larger K first, so that the units left at the end of the
-// sweep are the small ones.  Per 128-column k tile (a stage):
-//   * warp 0 (producer) loads the 8 x 512 B code tiles with one 3-D TMA and
-//     the token block (N rows x 128 B) with one bulk copy into a ring of L
-//     shared-memory stages (L = 8 to 32, as many as fit: the ring is what
-//     keeps enough code bytes in flight to cover the memory latency; it is
-//     decoupled from the 8 tensor-memory A slots below);
+// sweep are the small ones.  A stage is a group of four 128-column k tiles
+// (one barrier wait and one commit of the MMA thread per 16 MMAs: measured
+// on B200, the per-stage waits and commits of that single thread, not the
+// MMAs, set the pace with one k tile per stage):
+//   * warp 0 (producer) loads the 8 row blocks x 4 k tiles of codes (16 KB)
+//     with one 3-D TMA and the 4 token blocks (N rows x 128 B each) with one
+//     bulk copy into a ring of L shared-memory stages (as many as fit);
+//     k tiles past K read as zero codes, which expand to zero weights;
 //   * eight expansion warps (two per TMEM lane quarter, alternating stages)
 //     turn each 16-byte lane slot of the code tile into 16 registers with
 //     one AND each -- (word & (3 << 2s per byte)) holds codes + 1 of four
 //     consecutive k, times 4^s -- and store them to the stage's A slot in
 //     tensor memory (tcgen05.st 16x256b): column 8s + 2t + h of lane (row)
 //     g or g + 8 holds slot s of the word with k = 64h + 16t + 4s .. + 3.
-//     Slot 3 (4^3 (c + 1) = 128 does not fit int8) is shifted down instead;
+//     Slot 3 (4^3 (c + 1) = 128 does not fit int8) is shifted down instead.
+//     A stage fills one of two A slots of 4 x 32 columns;
 //   * warp 1 waits only for the expansion of the stage (which itself waited
-//     for the stage's bytes), issues four MMAs of K = 32, one per slot s
-//     (columns 8s .. 8s+7), into accumulator D_s (N columns each), and
+//     for the stage's bytes), issues four MMAs of K = 32 per k tile, one per
+//     slot s (columns 8s .. 8s+7), into accumulator D_s (N columns each), and
 //     commits them to the stage's empty barrier, which frees both the shared-
-//     memory stage and, eight stages later, the A slot;
+//     memory stage and, two stages later, the A slot;
 //   * four epilogue warps (one per lane quarter) read D_0..D_3 and form
 //     acc = D_0 + D_1/4 + D_2/16 + D_3 - sum(q), exact (D_s is a multiple
 //     of 4^s), then y.
@@ -51,11 +54,12 @@
 namespace tw {
 namespace {
 
-constexpr int kASlots = 8;                      // tensor-memory A slots (32 columns each)
+constexpr int kGrp = kTcGroup;                  // k tiles per stage
+constexpr int kASlots = 8 / kGrp;               // tensor-memory A slots (kGrp x 32 columns each)
 constexpr int kRingTc = 8;                      // unit-info entries
-constexpr int kMaxStagesTc = 32;                // shared-memory load stages, at most
+constexpr int kMaxStagesTc = 8;                 // shared-memory load stages, at most
 constexpr int kThreadsTc = 14 * 32;
-constexpr int kCodeStageBytes = 8 * kTileBytes;  // 128 rows x 128 k = 4 KB
+constexpr int kCodeStageBytes = 8 * kGrp * kTileBytes;  // 128 rows x 4 x 128 k = 16 KB
 constexpr int kTmemColsTc = 512;
 constexpr int kDCol0 = 256;                     // accumulators after 8 A slots of 32 columns
 constexpr uint64_t kDrainNsTc = 1000000000ull;
@@ -108,17 +112,23 @@ __device__ UnitInfo locate_unit(const TcParams &p, const UnitOrder *order, const
 }
 
 template <int NTOK>
+struct Lay_check {
+    static constexpr bool ok = (NTOK * 128) % 1024 == 0;   // token blocks stay swizzle-aligned
+};
+
+template <int NTOK>
 struct TcLayout {
     static constexpr int kBBytes = NTOK * 128;                           // token block
     static constexpr int kBPad = (kBBytes + 1023) / 1024 * 1024;
-    static constexpr int kStage = kCodeStageBytes + kBPad;
+    static constexpr int kStage = kCodeStageBytes + kGrp * kBPad;
     static constexpr int kMisc = 2048;
     // + the unit order (16 bytes) and the projection cache (40 bytes) per
     // projection after the misc block
     static int smem(int count, int stages) { return 1024 + stages * kStage + kMisc + 56 * count; }
     uint32_t base;
     __device__ uint32_t codes(int s) const { return base + s * kStage; }
-    __device__ uint32_t tok(int s) const { return base + s * kStage + kCodeStageBytes; }
+    // token block of k tile j (0 .. kGrp - 1) of stage s
+    __device__ uint32_t tok(int s, int j = 0) const { return base + s * kStage + kCodeStageBytes + j * kBPad; }
 };
 
 // int8 x int8 -> int32, K-major, M = 128, N = NTOK.
@@ -139,12 +149,13 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&v)[NTOK])
         tmem_ld32_nowait(taddr, v);
 }
 
-// L shared-memory stages (8 .. kMaxStagesTc).  Stage counters are 32-bit:
+// L shared-memory stages (4 .. kMaxStagesTc).  Stage counters are 32-bit:
 // a block streams at most a few thousand stages per call.
 template <int NTOK, int L>
 __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_constant__ TcParams p)
 {
     static_assert(L >= kASlots && L <= kMaxStagesTc && L % 2 == 0, "load stages");
+    static_assert(Lay_check<NTOK>::ok, "token blocks");
     using Lay = TcLayout<NTOK>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -206,13 +217,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
             // Token blocks of the stages issued before launch 1 has finished:
             // the codes of the first stages stream while it still quantises.
             const uint8_t *pend_src[L];
-            int pend_s[L];
+            int pend_s[L], pend_n[L];
             int npend = 0;
             auto flush_tokens = [&]() {
                 pdl_wait_tc();
                 tokens_ready = true;
                 for (int i = 0; i < npend; ++i)
-                    bulk_g2s(lay.tok(pend_s[i]), pend_src[i], (uint32_t)Lay::kBBytes,
+                    bulk_g2s(lay.tok(pend_s[i]), pend_src[i], (uint32_t)(pend_n[i] * Lay::kBBytes),
                              b_full + 8 * pend_s[i]);
                 npend = 0;
             };
@@ -240,7 +251,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                 claim2 = atomicAdd(p.ctr, 1u);
                 const void *tmap = p.table[u.d].tmap_codes;   // address only
                 const uint8_t *tok_src = p.ws + proj_s[u.d].ws_xq_off;
-                for (int kt = 0; kt < u.KT; ++kt, ++it) {
+                for (int kt0 = 0; kt0 < u.KT; kt0 += kGrp, ++it) {
                     const int s = (int)(it % L);
                     if (it >= L &&
                         !mbar_wait(b_empty + 8 * s, (it / L - 1) & 1u, p.ctl, abort_flag)) {
@@ -248,13 +259,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                         break;
                     }
                     stage_stop[s] = 0;
-                    mbar_arrive_expect_tx(b_full + 8 * s, (uint32_t)(kCodeStageBytes + Lay::kBBytes));
-                    tma_load_3d(lay.codes(s), tmap, 0, kt, 8 * u.rt, b_full + 8 * s);
-                    const uint8_t *src = tok_src + (int64_t)kt * Lay::kBBytes;
+                    const int nk = min(kGrp, u.KT - kt0);   // token blocks that exist
+                    mbar_arrive_expect_tx(b_full + 8 * s,
+                                          (uint32_t)(kCodeStageBytes + nk * Lay::kBBytes));
+                    tma_load_3d(lay.codes(s), tmap, 0, kt0, 8 * u.rt, b_full + 8 * s);
+                    const uint8_t *src = tok_src + (int64_t)kt0 * Lay::kBBytes;
                     if (tokens_ready) {
-                        bulk_g2s(lay.tok(s), src, (uint32_t)Lay::kBBytes, b_full + 8 * s);
+                        bulk_g2s(lay.tok(s), src, (uint32_t)(nk * Lay::kBBytes), b_full + 8 * s);
                     } else {
                         pend_src[npend] = src;
+                        pend_n[npend] = nk;
                         pend_s[npend] = s;
                         if (++npend == L)
                             flush_tokens();   // before any stage is waited on again
@@ -298,9 +312,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                     break;
                 tc_fence_after();
                 const uint32_t d0 = tmem + kDCol0 + (uint32_t)(buf * 4 * NTOK);
-                for (int kt = 0; kt < u.KT; ++kt, ++it) {
+                for (int kt0 = 0; kt0 < u.KT; kt0 += kGrp, ++it) {
                     // The expansion of this stage waited for its bytes (codes and
-                    // token block) before it arrived here.
+                    // token blocks) before it arrived here.
                     const int a = (int)(it % kASlots);
                     if (!mbar_wait(b_afull + 8 * a, (it / kASlots) & 1u, p.ctl, abort_flag)) {
                         ok = false;
@@ -308,12 +322,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                     }
                     tc_fence_after();
                     const int s = (int)(it % L);
-                    const uint64_t bd = sdesc_k_sw128(lay.tok(s));
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // +32 bytes of K = +2 in the address field
-                        mma_i8_ts(d0 + (uint32_t)(kk * NTOK), tmem + (uint32_t)(32 * a + 8 * kk),
-                                  bd + 2 * kk, idesc_tc<NTOK>(), kt > 0 ? 1u : 0u);
-                    mma_commit(b_empty + 8 * s);   // frees stage s, and A slot a for stage it + 8
+                    for (int j = 0; j < kGrp; ++j) {
+                        if (kt0 + j >= u.KT)
+                            break;   // k tiles past K (zero codes): nothing to add
+                        const uint64_t bd = sdesc_k_sw128(lay.tok(s, j));
+                        const uint32_t acol = tmem + (uint32_t)(32 * (kGrp * a + j));
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)  // +32 bytes of K = +2 in the address field
+                            mma_i8_ts(d0 + (uint32_t)(kk * NTOK), acol + (uint32_t)(8 * kk), bd + 2 * kk,
+                                      idesc_tc<NTOK>(), (kt0 > 0 || j > 0) ? 1u : 0u);
+                    }
+                    mma_commit(b_empty + 8 * s);   // frees stage s, and A slot a for stage it + 2
                 }
                 if (!ok)
                     break;
@@ -405,7 +425,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                 break;
             if (stage_stop[s])
                 break;
-            // A slot it % 8 is free once the MMAs of stage it - 8 have completed.
+            // A slot it % 2 is free once the MMAs of stage it - 2 have completed.
             if (it >= (uint32_t)kASlots &&
                 !mbar_wait(b_empty + 8 * (int)((it - kASlots) % L), ((it - kASlots) / L) & 1u, p.ctl,
                            abort_flag))
@@ -413,10 +433,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
             const uint32_t aslot = it % kASlots;
             tc_fence_after();
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                // lane slot of row block 2q + h: words (row g, k 16t..), (row
-                // g+8, same k), (row g, k 64+16t..), (row g+8, same k)
-                const uint4 w = lds128(lay.codes(s) + (2 * quarter + h) * kTileBytes + lane * 16);
+            for (int hj = 0; hj < 2 * kGrp; ++hj) {
+                // k tile j, row block 2q + h of the stage's box (laid out row
+                // block by row block, k tiles inside): lane slot words (row g,
+                // k 16t..), (row g+8, same k), (row g, k 64+16t..), (row g+8, same k)
+                const int h = hj & 1, j = hj >> 1;
+                const uint4 w = lds128(lay.codes(s) + ((2 * quarter + h) * kGrp + j) * kTileBytes + lane * 16);
                 uint32_t r[16];
 #pragma unroll
                 for (int u = 0; u < 3; ++u) {
@@ -430,7 +452,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                 r[13] = (w.z >> 6) & m;
                 r[14] = (w.y >> 6) & m;
                 r[15] = (w.w >> 6) & m;
-                tmem_st16x256b_x4(tmem + 32 * aslot + ((uint32_t)(32 * quarter + 16 * h) << 16), r);
+                tmem_st16x256b_x4(tmem + 32 * (kGrp * aslot + j) + ((uint32_t)(32 * quarter + 16 * h) << 16), r);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -483,20 +505,12 @@ template <int NTOK>
 cudaError_t launch_tc(const TcParams &p, int grid, cudaStream_t stream)
 {
     constexpr int kLimit = 227 * 1024;
-#ifdef TW_TC_STAGES
-    if (TW_TC_STAGES == 32 && TcLayout<NTOK>::smem(p.count, 32) <= kLimit) return launch_tc_l<NTOK, 32>(p, grid, stream);
-    if (TW_TC_STAGES == 24 && TcLayout<NTOK>::smem(p.count, 24) <= kLimit) return launch_tc_l<NTOK, 24>(p, grid, stream);
-    if (TW_TC_STAGES == 16 && TcLayout<NTOK>::smem(p.count, 16) <= kLimit) return launch_tc_l<NTOK, 16>(p, grid, stream);
-    if (TW_TC_STAGES == 8) return launch_tc_l<NTOK, 8>(p, grid, stream);
-#endif
-    if (TcLayout<NTOK>::smem(p.count, 32) <= kLimit)
-        return launch_tc_l<NTOK, 32>(p, grid, stream);
-    if (TcLayout<NTOK>::smem(p.count, 24) <= kLimit)
-        return launch_tc_l<NTOK, 24>(p, grid, stream);
-    if (TcLayout<NTOK>::smem(p.count, 16) <= kLimit)
-        return launch_tc_l<NTOK, 16>(p, grid, stream);
     if (TcLayout<NTOK>::smem(p.count, 8) <= kLimit)
         return launch_tc_l<NTOK, 8>(p, grid, stream);
+    if (TcLayout<NTOK>::smem(p.count, 6) <= kLimit)
+        return launch_tc_l<NTOK, 6>(p, grid, stream);
+    if (TcLayout<NTOK>::smem(p.count, 4) <= kLimit)
+        return launch_tc_l<NTOK, 4>(p, grid, stream);
     return cudaErrorInvalidValue;   // too many projections for the caches
 }
 

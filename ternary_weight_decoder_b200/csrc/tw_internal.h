@@ -231,8 +231,15 @@ int64_t prefill_tiles(int64_t M, int64_t N);
 int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, void *out128);
 // Encode the TMA descriptor of the packed codes of an [N x K] matrix, seen as
 // [ceil(N/16)] x [K/128] tiles of 128 32-bit words (one box = box_rb row
-// blocks of one k tile; row blocks past the matrix read as zero).
-int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, int box_rb, void *out128);
+// blocks x box_kt consecutive k tiles; row blocks and k tiles past the
+// matrix read as zero, which is the code -1 + 1 = 0 after expansion).
+int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, int box_rb, int box_kt,
+                      void *out128);
+// k tiles per pipeline stage of the tensor-core decode (tw_decode_tc.cu) and
+// of the weights-in-TMEM GEMM (tw_mid.cu): one barrier wait and one commit
+// of the MMA thread cover that many k tiles.
+constexpr int kTcGroup = 4;
+constexpr int kMidGroup = 2;
 
 cudaError_t launch_wait_probe(uint32_t *err, uint64_t timeout_ns, cudaStream_t stream);
 

@@ -18,20 +18,23 @@
 //
 // Work unit: one 128-row tile of one projection times one 128-token tile,
 // over all of K; units are claimed from a counter, projections of larger K
-// first.  Per 128-column k tile (a stage):
-//   * warp 0 loads the 8 x 512 B code tiles (one 3-D TMA box) and the
-//     128 x 128 B token tile (one 2-D TMA box of xq, 128-byte swizzled,
-//     tokens past M read as zero) into a ring of L shared-memory stages;
+// first.  A stage is a pair of 128-column k tiles (one barrier wait and one
+// commit of the MMA thread per 8 MMAs):
+//   * warp 0 loads the 8 row blocks x 2 k tiles of codes (one 3-D TMA box,
+//     k tiles past K read as zero codes) and the two 128 x 128 B token tiles
+//     (2-D TMA boxes of xq, 128-byte swizzled, tokens past M read as zero)
+//     into a ring of L shared-memory stages;
 //   * eight expansion warps (two sets of four, one warp per TMEM lane
 //     quarter, alternating stages) turn each 16-byte lane slot of the code
 //     tile into 16 registers holding code + 1 for 4 consecutive k each, in
 //     the natural k order of the MMA's K (each register's 16 source bits
 //     come from the word of lane 2(u & 1) + t/2 of the row's quad, fetched
-//     with a shuffle), and store them to one of 8 TMEM A slots
-//     (tcgen05.st 16x256b: column c of a slot holds k = 4c .. 4c + 3);
-//   * warp 1 issues four MMAs of K = 32 into the unit's accumulator (N =
-//     128 columns, one of two) and commits them to the stage's empty
-//     barrier, which frees the stage and, eight stages later, the A slot;
+//     with a shuffle), and store them to one of 4 TMEM A slots of 2 x 32
+//     columns (tcgen05.st 16x256b: column c of a k tile holds k = 4c .. 4c+3);
+//   * warp 1 issues four MMAs of K = 32 per k tile into the unit's
+//     accumulator (N = 128 columns, one of two) and commits them to the
+//     stage's empty barrier, which frees the stage and, four stages later,
+//     the A slot;
 //   * four epilogue warps (one per lane quarter: 32 weight rows each) read
 //     the accumulator 32 tokens at a time and store y, each store 32
 //     consecutive rows of one token.
@@ -47,12 +50,13 @@ namespace tw {
 namespace {
 
 constexpr int kNTok = 128;                       // tokens per unit (MMA N)
-constexpr int kASlotsM = 8;
+constexpr int kGrpM = kMidGroup;                 // k tiles per stage
+constexpr int kASlotsM = 8 / kGrpM;              // A slots of kGrpM x 32 columns
 constexpr int kRingM = 8;                        // unit-info entries
 constexpr int kThreadsM = 14 * 32;
-constexpr int kCodeBytesM = 8 * kTileBytes;       // 128 rows x 128 k = 4 KB
-constexpr int kTokBytesM = kNTok * 128;           // 16 KB
-constexpr int kStageM = kCodeBytesM + kTokBytesM;
+constexpr int kCodeBytesM = 8 * kGrpM * kTileBytes;   // 128 rows x 2 x 128 k = 8 KB
+constexpr int kTokBytesM = kNTok * 128;           // 16 KB per k tile
+constexpr int kStageM = kCodeBytesM + kGrpM * kTokBytesM;
 constexpr int kTmemColsM = 512;
 constexpr int kDCol0M = 256;                     // two accumulators after 8 A slots
 constexpr int kMiscM = 2048;
@@ -108,12 +112,12 @@ __device__ UnitM locate_unit_m(const MidParams &p, const UnitOrder *order, int64
 template <int L>
 __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ MidParams p)
 {
-    static_assert(L >= kASlotsM && L % 2 == 0, "load stages");
+    static_assert(L >= 2, "load stages");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     auto codes_s = [&](int s) { return base + (uint32_t)(s * kStageM); };
-    auto tok_s = [&](int s) { return base + (uint32_t)(s * kStageM + kCodeBytesM); };
+    auto tok_s = [&](int s, int j) { return base + (uint32_t)(s * kStageM + kCodeBytesM + j * kTokBytesM); };
     uint8_t *misc = smem_raw + (base - raw) + L * kStageM;
     const uint32_t bar0 = smem_u32(misc);
     const uint32_t b_full = bar0, b_empty = b_full + 8 * L, b_afull = b_empty + 8 * L;
@@ -188,16 +192,18 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
                 const void *tmap_c = p.table[u.d].tmap_codes;   // addresses only
                 const void *tmap_x = p.table[u.d].tmap_xq;
                 const int KT = proj_s[u.d].KT;
-                for (int kt = 0; kt < KT; ++kt, ++it) {
+                for (int kt0 = 0; kt0 < KT; kt0 += kGrpM, ++it) {
                     const int s = (int)(it % L);
                     if (it >= L && !mbar_wait(b_empty + 8 * s, (it / L - 1) & 1u, p.ctl, abort_flag)) {
                         ok = false;
                         break;
                     }
                     stage_stop[s] = 0;
-                    mbar_arrive_expect_tx(b_full + 8 * s, (uint32_t)kStageM);
-                    tma_load_3d(codes_s(s), tmap_c, 0, kt, 8 * u.rt, b_full + 8 * s);
-                    tma_load_2d(tok_s(s), tmap_x, kt * 128, u.tk * kNTok, b_full + 8 * s);
+                    const int nk = min(kGrpM, KT - kt0);   // token tiles that exist
+                    mbar_arrive_expect_tx(b_full + 8 * s, (uint32_t)(kCodeBytesM + nk * kTokBytesM));
+                    tma_load_3d(codes_s(s), tmap_c, 0, kt0, 8 * u.rt, b_full + 8 * s);
+                    for (int j = 0; j < nk; ++j)
+                        tma_load_2d(tok_s(s, j), tmap_x, (kt0 + j) * 128, u.tk * kNTok, b_full + 8 * s);
                 }
             }
             // One stop stage for each expansion set.
@@ -236,7 +242,7 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
                 tc_fence_after();
                 const uint32_t d0 = tmem + kDCol0M + (uint32_t)(buf * kNTok);
                 const int KT = proj_s[u.d].KT;
-                for (int kt = 0; kt < KT; ++kt, ++it) {
+                for (int kt0 = 0; kt0 < KT; kt0 += kGrpM, ++it) {
                     // The expansion of this stage waited for its bytes (codes and
                     // tokens) before it arrived here.
                     const int a = (int)(it % kASlotsM);
@@ -246,12 +252,18 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
                     }
                     tc_fence_after();
                     const int s = (int)(it % L);
-                    const uint64_t bd = sdesc_k_sw128(tok_s(s));
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // +32 bytes of K = +2 in the address field
-                        mma_i8_ts(d0, tmem + (uint32_t)(32 * a + 8 * kk), bd + 2 * kk, kIdescMid,
-                                  (kt > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(b_empty + 8 * s);   // frees stage s, and A slot a for stage it + 8
+                    for (int j = 0; j < kGrpM; ++j) {
+                        if (kt0 + j >= KT)
+                            break;   // k tile past K: nothing to add
+                        const uint64_t bd = sdesc_k_sw128(tok_s(s, j));
+                        const uint32_t acol = tmem + (uint32_t)(32 * (kGrpM * a + j));
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)  // +32 bytes of K = +2 in the address field
+                            mma_i8_ts(d0, acol + (uint32_t)(8 * kk), bd + 2 * kk, kIdescMid,
+                                      (kt0 > 0 || j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(b_empty + 8 * s);   // frees stage s, and A slot a for stage it + 4
                 }
                 if (!ok)
                     break;
@@ -345,7 +357,7 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
                 break;
             if (stage_stop[s])
                 break;
-            // A slot it % 8 is free once the MMAs of stage it - 8 have completed.
+            // A slot it % 4 is free once the MMAs of stage it - 4 have completed.
             if (it >= (uint32_t)kASlotsM &&
                 !mbar_wait(b_empty + 8 * (int)((it - kASlotsM) % L), ((it - kASlotsM) / L) & 1u, p.ctl,
                            abort_flag))
@@ -353,8 +365,10 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
             const uint32_t aslot = it % kASlotsM;
             tc_fence_after();
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint4 w = lds128(codes_s(s) + (2 * quarter + h) * kTileBytes + lane * 16);
+            for (int hj = 0; hj < 2 * kGrpM; ++hj) {
+                // row block 2q + h, k tile j of the box (row block by row block)
+                const int h = hj & 1, j = hj >> 1;
+                const uint4 w = lds128(codes_s(s) + ((2 * quarter + h) * kGrpM + j) * kTileBytes + lane * 16);
                 uint32_t r[16];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -368,7 +382,7 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
                         r[4 * u + 2 * rh + 1] = (word >> (sh0 + 2)) & m3;
                     }
                 }
-                tmem_st16x256b_x4(tmem + 32 * aslot + ((uint32_t)(32 * quarter + 16 * h) << 16), r);
+                tmem_st16x256b_x4(tmem + 32 * (kGrpM * aslot + j) + ((uint32_t)(32 * quarter + 16 * h) << 16), r);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -434,10 +448,10 @@ cudaError_t launch_mid(const MidLaunch &L, uint32_t *err, uint64_t timeout_ns, c
     const int64_t grid64 = L.total_units < sms ? L.total_units : sms;
     const int grid = (int)(grid64 < 1 ? 1 : grid64);
     constexpr int kLimit = 227 * 1024;
-    if (smem_mid<10>(p.count) <= kLimit)
-        return launch_mid_l<10>(p, grid, stream);
-    if (smem_mid<8>(p.count) <= kLimit)
-        return launch_mid_l<8>(p, grid, stream);
+    if (smem_mid<5>(p.count) <= kLimit)
+        return launch_mid_l<5>(p, grid, stream);
+    if (smem_mid<4>(p.count) <= kLimit)
+        return launch_mid_l<4>(p, grid, stream);
     return cudaErrorInvalidValue;   // too many projections for the caches
 }
 

@@ -424,7 +424,8 @@ int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, void *out128)
     return 0;
 }
 
-int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, int box_rb, void *out128)
+int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, int box_rb, int box_kt,
+                      void *out128)
 {
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
@@ -441,7 +442,7 @@ int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, int box_rb, v
     const int64_t KT = K / kTileK, nrb = (N + kTileRows - 1) / kTileRows;
     const cuuint64_t dims[3] = {(cuuint64_t)(kTileBytes / 4), (cuuint64_t)KT, (cuuint64_t)nrb};
     const cuuint64_t strides[2] = {(cuuint64_t)kTileBytes, (cuuint64_t)(KT * kTileBytes)};
-    const cuuint32_t box[3] = {kTileBytes / 4, 1, (cuuint32_t)box_rb};
+    const cuuint32_t box[3] = {kTileBytes / 4, (cuuint32_t)box_kt, (cuuint32_t)box_rb};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t *>(packed), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
