@@ -74,18 +74,24 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
 }
 
 // Grid-wide barrier number `k` (1, 2, ...): every CTA's writes before it are
-// visible to every CTA after it.  False when the wait timed out (the block
+// visible to every CTA after it.  ctr[0] counts arrivals; the CTA whose
+// arrival completes barrier k publishes k in ctr[2], which the others poll
+// (a line that only one atomic writes per barrier, so the polls do not
+// queue behind the arrivals).  False when the wait timed out (the block
 // must stop).
 __device__ bool grid_barrier(uint32_t *ctr, uint32_t k, const ChainParams &p, volatile int *abort_flag)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        atomicAdd(ctr, 1u);
         const uint32_t target = k * gridDim.x;
-        if (!*abort_flag && ld_acquire_u32(ctr) < target) {
+        if (atomicAdd(ctr, 1u) == target - 1) {
+            __threadfence();          // every arrival it has seen is ordered before the release
+            atomicExch(ctr + 2, k);   // the last arrival releases barrier k
+        }
+        if (!*abort_flag && ld_acquire_u32(ctr + 2) < k) {
             const uint64_t t0 = globaltimer_ns();
-            while (ld_acquire_u32(ctr) < target) {
+            while (ld_acquire_u32(ctr + 2) < k) {
                 if (*abort_flag)
                     break;
                 if (globaltimer_ns() - t0 > p.ctl.timeout_ns) {
@@ -531,6 +537,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
         if (atomicAdd(ctr + 1, 1u) == gridDim.x - 1) {
             ctr[0] = 0u;
             ctr[1] = 0u;
+            ctr[2] = 0u;
             __threadfence();
         }
     }

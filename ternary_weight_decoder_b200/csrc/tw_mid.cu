@@ -36,8 +36,11 @@
 //     stage's empty barrier, which frees the stage and, four stages later,
 //     the A slot;
 //   * four epilogue warps (one per lane quarter: 32 weight rows each) read
-//     the accumulator 32 tokens at a time and store y, each store 32
-//     consecutive rows of one token.
+//     the accumulator 32 tokens at a time (lane = weight row), rescale, and
+//     stage the 32 x 32 box in shared memory token by token, then store it
+//     with float4 writes: one store instruction covers 4 tokens x 128
+//     contiguous bytes of y (measured on B200: one 4-byte store per lane and
+//     token left the epilogue at about a third of the MMA rate).
 // Every wait is bounded; on a timeout the block stops, drains its copies and
 // MMAs, frees its tensor memory and returns.
 #include <cstring>
@@ -88,8 +91,12 @@ struct MidParams {
     WaitCtl ctl;
 };
 
+constexpr int kBoxM = 32 * 32 * 4;               // one epilogue warp's staging box
 template <int L>
-constexpr int smem_mid(int count) { return 1024 + L * kStageM + kMiscM + (16 + (int)sizeof(ProjM)) * count; }
+constexpr int smem_mid(int count)
+{
+    return 1024 + L * kStageM + 4 * kBoxM + kMiscM + (16 + (int)sizeof(ProjM)) * count;
+}
 
 // int8 x int8 -> int32, K-major, M = 128, N = 128.
 constexpr uint32_t kIdescMid = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kNTok >> 3) << 17) |
@@ -118,7 +125,8 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
     const uint32_t base = (raw + 1023u) & ~1023u;
     auto codes_s = [&](int s) { return base + (uint32_t)(s * kStageM); };
     auto tok_s = [&](int s, int j) { return base + (uint32_t)(s * kStageM + kCodeBytesM + j * kTokBytesM); };
-    uint8_t *misc = smem_raw + (base - raw) + L * kStageM;
+    float *boxes = reinterpret_cast<float *>(smem_raw + (base - raw) + L * kStageM);
+    uint8_t *misc = smem_raw + (base - raw) + L * kStageM + 4 * kBoxM;
     const uint32_t bar0 = smem_u32(misc);
     const uint32_t b_full = bar0, b_empty = b_full + 8 * L, b_afull = b_empty + 8 * L;
     const uint32_t b_ufull = b_afull + 8 * kASlotsM, b_uempty = b_ufull + 8 * kRingM;
@@ -279,6 +287,7 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
     } else if (warp < 6) {
         // ------------------------------------------------------ epilogue
         const int quarter = warp & 3;
+        float *box = boxes + (warp - 2) * (kBoxM / 4);   // [32 tokens][32 rows]
         for (int j = 0;; ++j) {
             const int ju = j % kRingM;
             if (!mbar_wait(b_ufull + 8 * ju, (uint32_t)((j / kRingM) & 1), p.ctl, abort_flag))
@@ -288,7 +297,6 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
                 break;
             const ProjM pr = proj_s[u.d];
             const int buf = j & 1;
-            const int64_t row = (int64_t)u.rt * 128 + 32 * quarter + lane;
             const int m_base = u.tk * kNTok;
             // this lane's token of each group of 32: scale and sum(q), loaded
             // before the accumulator is ready
@@ -306,7 +314,9 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
             const uint32_t dq = tmem + kDCol0M + (uint32_t)(buf * kNTok) + ((uint32_t)(32 * quarter) << 16);
             int nvalid = p.M - m_base;
             nvalid = nvalid > kNTok ? kNTok : nvalid;
-            const bool row_ok = row < pr.N;
+            const int64_t row0 = (int64_t)u.rt * 128 + 32 * quarter;   // the warp's first row
+            // float4 stores need 16-byte aligned rows of y: N a multiple of 4
+            const bool vec = (pr.N & 3) == 0 && row0 + 32 <= pr.N;
 #pragma unroll 1
             for (int c = 0; c < kNTok / 32; ++c) {
                 uint32_t v[32];
@@ -320,18 +330,35 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
                 }
                 if (32 * c >= nvalid)
                     continue;   // (uniform across the warp)
+                for (int pass = 0; pass < (pr.acc_out ? 2 : 1); ++pass) {
+                    // box[n][lane] = token 32c + n of this lane's row
 #pragma unroll
-                for (int n = 0; n < 32; ++n) {
-                    const float sa = __shfl_sync(0xffffffffu, sa_l[c], n);
-                    const int qs = __shfl_sync(0xffffffffu, qs_l[c], n);
-                    const int m = 32 * c + n;
-                    if (row_ok && m < nvalid) {
+                    for (int n = 0; n < 32; ++n) {
+                        const float sa = __shfl_sync(0xffffffffu, sa_l[c], n);
+                        const int qs = __shfl_sync(0xffffffffu, qs_l[c], n);
                         const int a = (int)v[n] - qs;
-                        const int64_t o = (int64_t)(m_base + m) * pr.N + row;
-                        pr.y[o] = __fmul_rn(__fmul_rn((float)a, sa), pr.wscale);
-                        if (pr.acc_out)
-                            pr.acc_out[o] = a;
+                        box[n * 32 + lane] = pass == 0 ? __fmul_rn(__fmul_rn((float)a, sa), pr.wscale)
+                                                       : __int_as_float(a);
                     }
+                    __syncwarp();
+                    float *dst = pass == 0 ? pr.y : reinterpret_cast<float *>(pr.acc_out);
+                    const int mmax = nvalid - 32 * c;   // tokens of this box that exist
+                    if (vec) {
+                        // 8 lanes per token row (128 bytes), 4 tokens per instruction
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int n = 4 * i + (lane >> 3), r4 = 4 * (lane & 7);
+                            if (n < mmax)
+                                *reinterpret_cast<float4 *>(dst + (int64_t)(m_base + 32 * c + n) * pr.N +
+                                                            row0 + r4) =
+                                    *reinterpret_cast<const float4 *>(box + n * 32 + r4);
+                        }
+                    } else {
+                        for (int n = 0; n < 32 && n < mmax; ++n)
+                            if (row0 + lane < pr.N)
+                                dst[(int64_t)(m_base + 32 * c + n) * pr.N + row0 + lane] = box[n * 32 + lane];
+                    }
+                    __syncwarp();
                 }
             }
             __syncwarp();
