@@ -526,16 +526,16 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
         r.tile_begin = tiles;
         r.ptile_begin = ptiles;
         {
-            // prefill: xq tiles of 128 tokens and 256-row code boxes; decode:
-            // 128-row code boxes of the tensor-core sweep.  Without a CUDA
-            // driver (-1) a decode table is still encoded for its sizes; the
-            // sweep refuses it.
-            // (code boxes of 128 rows for the decode and weights-in-TMEM
-            // kernels, 256 rows for the expanded-weights GEMM)
+            // M > 32: xq tiles of 128 tokens; code boxes of 128 rows x 4 k
+            // tiles (tensor-core decode), 128 rows x 2 k tiles (weights-in-TMEM
+            // GEMM) or 256 rows x 1 k tile (expanded-weights GEMM).  Without a
+            // CUDA driver (-1) a decode table is still encoded for its sizes;
+            // the sweep refuses it.
+            const bool mid = tw::sweep_on_mid(M);
             int rc = decode ? 0 : tw::encode_xq_tmap(s.xq, M, s.K, r.tmap_xq);
             if (!rc)
-                rc = tw::encode_codes_tmap(r.packed, s.N, s.K, decode || TW_SWEEP_MID ? 8 : 16,
-                                           decode ? tw::kTcGroup : TW_SWEEP_MID ? tw::kMidGroup : 1,
+                rc = tw::encode_codes_tmap(r.packed, s.N, s.K, decode || mid ? 8 : 16,
+                                           decode ? tw::kTcGroup : mid ? tw::kMidGroup : 1,
                                            r.tmap_codes);
             if (rc && !(decode && rc == -1))
                 return fail(TW_ERR_CUDA, "descriptor %d: cuTensorMapEncodeTiled failed (%d)", d,
@@ -581,7 +581,7 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
     hdr->total_ptiles = ptiles;
     // decode: counters, rows and scales; more tokens: the unit counters of the
     // weights-in-TMEM kernel
-    hdr->ws_bytes = decode ? ws_off + 256 * (int64_t)count : (TW_SWEEP_MID ? tw::kWsCtrBytes : 0);
+    hdr->ws_bytes = decode ? ws_off + 256 * (int64_t)count : (tw::sweep_on_mid(M) ? tw::kWsCtrBytes : 0);
     hdr->max_K = max_K;
     hdr->total_cost = cost;
     return TW_OK;
@@ -619,7 +619,7 @@ int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, v
     uint32_t *err = nullptr;
     if (int rc = err_word(&err))
         return rc;
-    if (hdr->M > tw::kDecodeMaxM && TW_SWEEP_MID) {
+    if (tw::sweep_on_mid(hdr->M)) {
         if (ws_bytes < (size_t)hdr->ws_bytes || !ws)
             return fail(TW_ERR_BUFSIZE, "sweep workspace %zu < %lld bytes", ws_bytes,
                         (long long)hdr->ws_bytes);

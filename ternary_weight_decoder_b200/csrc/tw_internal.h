@@ -209,11 +209,16 @@ struct MidLaunch {
 cudaError_t launch_mid(const MidLaunch &L, uint32_t *err, uint64_t timeout_ns, cudaStream_t stream);
 // Work units of one projection on that path: ceil(N / 128) x ceil(M / 128).
 int64_t mid_units(int64_t M, int64_t N);
-// Which kernel runs a sweep of more than 32 tokens: the weights-in-TMEM
-// GEMM (1) or the expanded-weights GEMM of tw_prefill.cu (0).
-#ifndef TW_SWEEP_MID
-#define TW_SWEEP_MID 1
+// Which kernel runs a sweep of M > 32 tokens: the weights-in-TMEM GEMM up
+// to TW_MID_MAX_M tokens, the expanded-weights GEMM of tw_prefill.cu above
+// (measured on B200 over the 196-projection sweep: 195 / 189 / 244 / 365 us
+// against 246 / 248 / 258 / 421 us at 48 / 64 / 128 / 192 tokens, 450 against
+// 426 us at 256; the first streams each code byte once per 128 tokens, the
+// second expands it into shared memory once per 128-row by 256-token tile).
+#ifndef TW_MID_MAX_M
+#define TW_MID_MAX_M 192
 #endif
+inline bool sweep_on_mid(int64_t M) { return M > kDecodeMaxM && M <= TW_MID_MAX_M; }
 
 struct PrefillLaunch {
     const DescRecord *table;  // device records (or null: use `single`)
