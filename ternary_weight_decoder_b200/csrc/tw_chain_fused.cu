@@ -73,25 +73,27 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
     return v;
 }
 
+__device__ __forceinline__ void red_release_add_u32(uint32_t *p, uint32_t v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" : : "l"(p), "r"(v) : "memory");
+}
+
 // Grid-wide barrier number `k` (1, 2, ...): every CTA's writes before it are
-// visible to every CTA after it.  ctr[0] counts arrivals; the CTA whose
-// arrival completes barrier k publishes k in ctr[2], which the others poll
-// (a line that only one atomic writes per barrier, so the polls do not
-// queue behind the arrivals).  False when the wait timed out (the block
-// must stop).
+// visible to every CTA after it.  ctr[0] counts arrivals over the whole call;
+// after __syncthreads thread 0 adds its CTA's arrival with release semantics
+// (which carry the CTA's writes ordered before it by the block barrier) and
+// polls the count with acquire loads until all k * gridDim.x arrivals are in.
+// The release and acquire replace two full fences per CTA.  False when the
+// wait timed out (the block must stop).
 __device__ bool grid_barrier(uint32_t *ctr, uint32_t k, const ChainParams &p, volatile int *abort_flag)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
         const uint32_t target = k * gridDim.x;
-        if (atomicAdd(ctr, 1u) == target - 1) {
-            __threadfence();          // every arrival it has seen is ordered before the release
-            atomicExch(ctr + 2, k);   // the last arrival releases barrier k
-        }
-        if (!*abort_flag && ld_acquire_u32(ctr + 2) < k) {
+        red_release_add_u32(ctr, 1u);
+        if (!*abort_flag && ld_acquire_u32(ctr) < target) {
             const uint64_t t0 = globaltimer_ns();
-            while (ld_acquire_u32(ctr + 2) < k) {
+            while (ld_acquire_u32(ctr) < target) {
                 if (*abort_flag)
                     break;
                 if (globaltimer_ns() - t0 > p.ctl.timeout_ns) {
@@ -101,7 +103,6 @@ __device__ bool grid_barrier(uint32_t *ctr, uint32_t k, const ChainParams &p, vo
                 }
             }
         }
-        __threadfence();
     }
     __syncthreads();
     return !*abort_flag;
