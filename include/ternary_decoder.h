@@ -205,8 +205,8 @@ TW_API size_t tw_sweep_table_bytes(int count);
  * tw_decoder_projection_sweep; the table stays valid for as long as the
  * buffers it names do.  Layout: a 64-byte header, one 384-byte record per
  * projection, then one 16-byte entry per projection giving the order in
- * which the tensor-core decode sweep hands out its 128-row units
- * (projections of larger K first).  The records embed TMA descriptors --
+ * which the tensor-core kernels hand out their units (projections of larger
+ * K first).  The records embed TMA descriptors --
  * of each xq (M > 32) and of the packed codes (every M) -- and therefore
  * need the CUDA driver: a decode table encoded where the driver is missing
  * still answers the size queries, but the sweep refuses it (TW_ERR_CUDA).
@@ -229,8 +229,11 @@ TW_API size_t tw_sweep_workspace_bytes(const void *table_host);
  * launch of the register (mma.sync) kernel -- more only when M*K of the
  * widest projection does not fit shared memory and the tokens are split
  * into groups -- and for 16 < M <= 32 one launch of the tensor-core decode
- * kernel.  More tokens: one persistent tensor-core launch with the weights
- * in tensor memory (units of 128 weight rows x 128 tokens).
+ * kernel.  33..192 tokens: one persistent tensor-core launch with the
+ * weights in tensor memory (units of 128 weight rows x 128 tokens, claimed
+ * from the counters in the workspace); more tokens: one persistent
+ * tensor-core launch with the weights expanded in shared memory (output
+ * tiles of 128 tokens x 256 weight rows dealt out round robin).
  *   table_host  the host table written by tw_sweep_table_encode (read for the
  *               launch configuration: count, M, sizes);
  *   table_dev   the caller's device copy of the same bytes (64-byte aligned),

@@ -13,8 +13,11 @@
 // page, "Layout".)
 //
 // Tile: 128 tokens x 256 weight rows, K in stages of 128 (one swizzle atom),
-// four MMAs of K = 32 per stage; four stages of A + code tiles in flight,
-// three expanded B tiles.  Persistent: one CTA per SM walks the
+// four MMAs of K = 32 per stage; five stages of A + code tiles in flight,
+// two expanded B tiles (measured on B200: the A + code ring, whose stages
+// are held from the TMA issue until their MMAs complete, is the deeper
+// need: 398 against 424 us at 256 tokens and 1.40 against 1.47 ms at 1024
+// over the 196 projections).  Persistent: one CTA per SM walks the
 // output tiles of every projection (all token tiles of a weight tile run
 // back to back across the grid, so the weight codes stream from HBM once
 // and the activations stay in L2).  Two TMEM accumulators let the epilogue
@@ -37,8 +40,8 @@ namespace {
 constexpr int kBM = 128;                 // tokens per tile (MMA M)
 constexpr int kBN = 256;                 // weight rows per tile (MMA N)
 constexpr int kBK = 128;                 // k per stage
-constexpr int kLoadStages = 4;           // A + code tiles in flight
-constexpr int kBStages = 3;              // expanded B tiles
+constexpr int kLoadStages = 5;           // A + code tiles in flight
+constexpr int kBStages = 2;              // expanded B tiles
 constexpr int kABytes = kBM * kBK;       // 16 KB
 constexpr int kBBytes = kBN * kBK;       // 32 KB
 constexpr int kCodeBytes = kBN / kTileRows * kTileBytes;  // 16 tiles = 8 KB
@@ -49,6 +52,7 @@ constexpr int kTmemCols = 512;           // two 256-column accumulators
 constexpr int kStageRowF = 36;           // epilogue staging row (floats), 32 + 4 pad
 constexpr int kStagingBytes = 4 * 32 * kStageRowF * 4;
 constexpr int kSmemBytes = 1024 + kLoadStages * kLoadBytes + kBStages * kBBytes + kStagingBytes + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 constexpr uint64_t kDrainNs = 1000000000ull;
 
 struct PrefillParams {
@@ -136,8 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     SmemLayout L{base};
     uint8_t *misc = gen_base + kLoadStages * kLoadBytes + kBStages * kBBytes + kStagingBytes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(misc);
-    // barriers: ld_full[4], ld_empty[4], b_full[3], b_empty[3], tmem_full[2],
-    // tmem_empty[2], drain
+    // barriers: ld_full[kLoadStages], ld_empty[kLoadStages], b_full[kBStages],
+    // b_empty[kBStages], tmem_full[2], tmem_empty[2], drain
     const uint32_t bar0 = smem_u32(bars);
     const uint32_t b_ldfull = bar0, b_ldempty = bar0 + 8 * kLoadStages;
     const uint32_t b_bfull = bar0 + 16 * kLoadStages, b_bempty = b_bfull + 8 * kBStages;
