@@ -161,7 +161,11 @@ def profiled_traffic(kernel_src, M, layers):
 
 def decode_kernel_src(M):
     """Source file of the dominant kernel of a sweep of M tokens."""
-    return "tw_prefill.cu" if M > 32 else "tw_decode_tc.cu" if M > 16 else "tw_decode.cu"
+    if M > 192:
+        return "tw_prefill.cu"
+    if M > 32:
+        return "tw_mid.cu"
+    return "tw_decode_tc.cu" if M > 8 else "tw_decode.cu"
 
 
 def sweep_bytes(shapes, M):
@@ -540,6 +544,32 @@ def _oracle_sample(M, rows_cap, token_cap, budget_s, layers=28, sample_layers=1)
             "sample": desc, **cpu_info()}
 
 
+def _oracle_call_us(projs, M, budget_s):
+    """Microseconds per call of the oracle on one host core, run back to back
+    for about budget_s over the given (layer, projection) indices at M tokens
+    (the whole matrices)."""
+    from oracle import oracle as orc
+    from ternary_weight_decoder_b200 import synth
+    shapes = {(l, p): (N, K) for (l, p, _, N, K) in synth.sweep_shapes(1)}
+    sample = []
+    for lp in projs:
+        N, K = shapes[lp]
+        if lp not in _ORACLE_CODES:
+            _ORACLE_CODES[lp] = orc.ternarize(synth.weights(lp[0], lp[1], N, K))
+        codes, mean = _ORACLE_CODES[lp]
+        sample.append((synth.activations(lp[0], lp[1], M, K), codes, mean))
+    timed, passes = 0.0, 0
+    while timed < budget_s or passes == 0:
+        t0 = time.perf_counter()
+        for x, codes, mean in sample:
+            orc.ternary_linear(x, codes, mean)
+        timed += time.perf_counter() - t0
+        passes += 1
+    return {"value": timed / passes * 1e6, "unit": "us per call", "cores": 1, "kind": "oracle",
+            "sample": f"{len(sample)} whole projection(s) of layer 0 at {M} token(s), {passes} passes, "
+                      f"{timed:.1f} s timed", **cpu_info()}
+
+
 def cpu_oracle_sample(M, budget_s=10.0, sample_layers=4, layers=28):
     """Headline CPU baseline: the oracle over all rows of the projections
     of the first `sample_layers` layers at M tokens."""
@@ -648,6 +678,8 @@ def measure_configs(args, api, torch, dev, rank, shapes, weights, descs_m1, want
             "frac_hbm_at_median": nbytes / (s["median_us"] * 1e-6) / 1e9 / hbm,
             "launches_per_call": 2, "l2": "flushed (256 MB written) before every call",
             "note": "launch-latency bound: the 0.6 MB of work is 0.09 us of HBM time"}
+        if cpu_ok:
+            out["1_gemv_1536x1536_M1"]["oracle"] = _oracle_call_us([(0, 0)], 1, 2.0)
 
     if "2" in want:
         layer0 = descs_m1[:7]
@@ -665,6 +697,8 @@ def measure_configs(args, api, torch, dev, rank, shapes, weights, descs_m1, want
             "algorithmic_bytes": nbytes,
             "frac_hbm_at_median": nbytes / (s["median_us"] * 1e-6) / 1e9 / hbm,
             "launches_per_call": t1.launches, "l2": "flushed (256 MB written) before every call"}
+        if cpu_ok:
+            out["2_layer_7proj_M1"]["oracle"] = _oracle_call_us([(0, p) for p in range(7)], 1, 3.0)
         del t1
     del flush_buf
 

@@ -225,10 +225,10 @@ TW_API size_t tw_sweep_workspace_bytes(const void *table_host);
 
 /*
  * Run the layer over every projection of an encoded table.  Decode
- * (M <= 32): one quantisation launch, then for M <= 16 one persistent
+ * (M <= 32): one quantisation launch, then for M <= 8 one persistent
  * launch of the register (mma.sync) kernel -- more only when M*K of the
  * widest projection does not fit shared memory and the tokens are split
- * into groups -- and for 16 < M <= 32 one launch of the tensor-core decode
+ * into groups -- and for 8 < M <= 32 one launch of the tensor-core decode
  * kernel.  33..192 tokens: one persistent tensor-core launch with the
  * weights in tensor memory (units of 128 weight rows x 128 tokens, claimed
  * from the counters in the workspace); more tokens: one persistent

@@ -23,21 +23,25 @@
 //     bulk copy into a ring of L shared-memory stages (as many as fit);
 //     k tiles past K read as zero codes, which expand to zero weights;
 //   * eight expansion warps (two per TMEM lane quarter, alternating stages)
-//     turn each 16-byte lane slot of the code tile into 16 registers with
-//     one AND each -- (word & (3 << 2s per byte)) holds codes + 1 of four
-//     consecutive k, times 4^s -- and store them to the stage's A slot in
-//     tensor memory (tcgen05.st 16x256b): column 8s + 2t + h of lane (row)
-//     g or g + 8 holds slot s of the word with k = 64h + 16t + 4s .. + 3.
-//     Slot 3 (4^3 (c + 1) = 128 does not fit int8) is shifted down instead.
-//     A stage fills one of two A slots of 4 x 32 columns;
+//     turn each 16-byte lane slot of the code tile into 16 registers -- the
+//     2-bit slot s of every byte of a word holds codes + 1 of four
+//     consecutive k -- and store them to the stage's A slot in tensor memory
+//     (tcgen05.st 16x256b): column 8s + 2t + h of lane (row) g or g + 8
+//     holds slot s of the word with k = 64h + 16t + 4s .. + 3.  A stage
+//     fills one of kASlots A slots of 4 x 32 columns;
 //   * warp 1 waits only for the expansion of the stage (which itself waited
 //     for the stage's bytes), issues four MMAs of K = 32 per k tile, one per
-//     slot s (columns 8s .. 8s+7), into accumulator D_s (N columns each), and
-//     commits them to the stage's empty barrier, which frees both the shared-
-//     memory stage and, two stages later, the A slot;
-//   * four epilogue warps (one per lane quarter) read D_0..D_3 and form
-//     acc = D_0 + D_1/4 + D_2/16 + D_3 - sum(q), exact (D_s is a multiple
-//     of 4^s), then y.
+//     slot s (columns 8s .. 8s+7), and commits them to the stage's empty
+//     barrier, which frees both the shared-memory stage and, kASlots stages
+//     later, the A slot;
+//   * four epilogue warps (one per lane quarter) read the accumulator, form
+//     acc = D - sum(q), exact, then y.
+// With 32 tokens the slots are expanded unscaled ((word >> 2s) & 0x03 per
+// byte) and every MMA adds into one accumulator D.  With 8 or 16 tokens they
+// are expanded with one AND each ((word & (3 << 2s per byte)) is c + 1 times
+// 4^s; slot 3, whose 4^3 (c + 1) = 128 does not fit int8, is shifted down
+// instead), MMA s adds into accumulator D_s, and the epilogue forms
+// D = D_0 + D_1/4 + D_2/16 + D_3 (exact: D_s is a multiple of 4^s).
 // The token block pairs position 4c + b of each 128-byte row with the k of
 // A column c, so the quantisation launch stores logical k group
 // G = 16h + 4t + s of a tile at column c = 8s + 2t + h, and swizzles the
@@ -55,13 +59,27 @@ namespace tw {
 namespace {
 
 constexpr int kGrp = kTcGroup;                  // k tiles per stage
-constexpr int kASlots = 8 / kGrp;               // tensor-memory A slots (kGrp x 32 columns each)
 constexpr int kRingTc = 8;                      // unit-info entries
 constexpr int kMaxStagesTc = 8;                 // shared-memory load stages, at most
 constexpr int kThreadsTc = 14 * 32;
 constexpr int kCodeStageBytes = 8 * kGrp * kTileBytes;  // 128 rows x 4 x 128 k = 16 KB
 constexpr int kTmemColsTc = 512;
-constexpr int kDCol0 = 256;                     // accumulators after 8 A slots of 32 columns
+
+// Tensor-memory plan per token-block width.  32 tokens: one accumulator per
+// buffer (every slot's codes expanded unscaled, c + 1 in {0, 1, 2}) and
+// three A slots, so that the expansion stays further ahead and the epilogue
+// reads one accumulator; 8 or 16 tokens: one accumulator per 2-bit slot
+// (expanded with one AND, scaled by 4^s) and two A slots.  Measured on B200
+// over the 196 projections: 138.3 against 144.4 us at 32 tokens, 117.8
+// against 119.8 us at 16 for the four-accumulator plan.
+template <int NTOK>
+struct AccPlan {
+    static constexpr bool kOneD = NTOK == 32;
+    static constexpr int kASlots = kOneD ? 3 : 2;           // A slots of kGrp x 32 columns
+    static constexpr int kDCol0 = 32 * kGrp * kASlots;      // the two accumulator buffers
+    static constexpr int kDCols = kOneD ? NTOK : 4 * NTOK;  // columns of one buffer
+    static_assert(kDCol0 + 2 * kDCols <= 512, "tensor memory");
+};
 constexpr uint64_t kDrainNsTc = 1000000000ull;
 
 struct UnitInfo {
@@ -154,6 +172,8 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&v)[NTOK])
 template <int NTOK, int L>
 __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_constant__ TcParams p)
 {
+    using AP = AccPlan<NTOK>;
+    constexpr int kASlots = AP::kASlots, kDCol0 = AP::kDCol0;
     static_assert(L >= kASlots && L <= kMaxStagesTc && L % 2 == 0, "load stages");
     static_assert(Lay_check<NTOK>::ok, "token blocks");
     using Lay = TcLayout<NTOK>;
@@ -311,7 +331,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                     !mbar_wait(b_dempty + 8 * buf, (uint32_t)((j / 2 - 1) & 1), p.ctl, abort_flag))
                     break;
                 tc_fence_after();
-                const uint32_t d0 = tmem + kDCol0 + (uint32_t)(buf * 4 * NTOK);
+                const uint32_t d0 = tmem + kDCol0 + (uint32_t)(buf * AP::kDCols);
                 for (int kt0 = 0; kt0 < u.KT; kt0 += kGrp, ++it) {
                     // The expansion of this stage waited for its bytes (codes and
                     // token blocks) before it arrived here.
@@ -322,16 +342,34 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                     }
                     tc_fence_after();
                     const int s = (int)(it % L);
+                    // Descriptors of the stage: k tile j's token block is kBPad
+                    // bytes after the previous one; +32 bytes of K = +2 in the
+                    // address field.  A full group runs without a test per
+                    // k tile (measured: 130.1 -> 128.0 us at 20 tokens).
+                    const uint64_t bd0 = sdesc_k_sw128(lay.tok(s, 0));
+                    const uint32_t acol0 = tmem + (uint32_t)(32 * kGrp * a);
+                    const uint32_t first = kt0 > 0 ? 1u : 0u;
+                    auto mma_tile = [&](int j) {
 #pragma unroll
-                    for (int j = 0; j < kGrp; ++j) {
-                        if (kt0 + j >= u.KT)
-                            break;   // k tiles past K (zero codes): nothing to add
-                        const uint64_t bd = sdesc_k_sw128(lay.tok(s, j));
-                        const uint32_t acol = tmem + (uint32_t)(32 * (kGrp * a + j));
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t d = AP::kOneD ? d0 : d0 + (uint32_t)(kk * NTOK);
+                            const uint32_t acc_in = j > 0 || (AP::kOneD && kk > 0) ? 1u : first;
+                            mma_i8_ts(d, acol0 + (uint32_t)(32 * j + 8 * kk),
+                                      bd0 + (uint64_t)((Lay::kBPad >> 4) * j + 2 * kk), idesc_tc<NTOK>(),
+                                      acc_in);
+                        }
+                    };
+                    if (kt0 + kGrp <= u.KT) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)  // +32 bytes of K = +2 in the address field
-                            mma_i8_ts(d0 + (uint32_t)(kk * NTOK), acol + (uint32_t)(8 * kk), bd + 2 * kk,
-                                      idesc_tc<NTOK>(), (kt0 > 0 || j > 0) ? 1u : 0u);
+                        for (int j = 0; j < kGrp; ++j)
+                            mma_tile(j);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < kGrp; ++j) {
+                            if (kt0 + j >= u.KT)
+                                break;   // k tiles past K (zero codes): nothing to add
+                            mma_tile(j);
+                        }
                     }
                     mma_commit(b_empty + 8 * s);   // frees stage s, and A slot a for stage it + 2
                 }
@@ -370,7 +408,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
             const uint8_t *info = p.ws + p.ws_sa_off + 256 * (int64_t)u.d;
             const float sa_l = lane < p.M ? reinterpret_cast<const float *>(info)[lane] : 0.f;
             const int qs_l = lane < p.M ? reinterpret_cast<const int *>(info + 128)[lane] : 0;
-            const uint32_t dq = tmem + kDCol0 + (uint32_t)(buf * 4 * NTOK) + ((uint32_t)(32 * quarter) << 16);
+            const uint32_t dq = tmem + kDCol0 + (uint32_t)(buf * AP::kDCols) + ((uint32_t)(32 * quarter) << 16);
             int acc[NTOK];
             {
                 uint32_t v[NTOK];
@@ -379,6 +417,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
 #pragma unroll
                 for (int n = 0; n < NTOK; ++n)
                     acc[n] = (int)v[n];
+            }
+            if constexpr (!AP::kOneD) {
+                uint32_t v[NTOK];
                 tmem_ld_n<NTOK>(dq + NTOK, v);
                 tmem_wait_ld();
 #pragma unroll
@@ -425,7 +466,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                 break;
             if (stage_stop[s])
                 break;
-            // A slot it % 2 is free once the MMAs of stage it - 2 have completed.
+            // A slot it % kASlots is free once the MMAs of stage it - kASlots
+            // have completed.
             if (it >= (uint32_t)kASlots &&
                 !mbar_wait(b_empty + 8 * (int)((it - kASlots) % L), ((it - kASlots) / L) & 1u, p.ctl,
                            abort_flag))
@@ -440,18 +482,28 @@ __global__ void __launch_bounds__(kThreadsTc, 1) k_decode_tc(const __grid_consta
                 const int h = hj & 1, j = hj >> 1;
                 const uint4 w = lds128(lay.codes(s) + ((2 * quarter + h) * kGrp + j) * kTileBytes + lane * 16);
                 uint32_t r[16];
+                if constexpr (AP::kOneD) {
 #pragma unroll
-                for (int u = 0; u < 3; ++u) {
-                    const uint32_t mu = m << (2 * u);
-                    r[4 * u + 0] = w.x & mu;
-                    r[4 * u + 1] = w.z & mu;
-                    r[4 * u + 2] = w.y & mu;
-                    r[4 * u + 3] = w.w & mu;
+                    for (int u = 0; u < 4; ++u) {
+                        r[4 * u + 0] = (w.x >> (2 * u)) & m;
+                        r[4 * u + 1] = (w.z >> (2 * u)) & m;
+                        r[4 * u + 2] = (w.y >> (2 * u)) & m;
+                        r[4 * u + 3] = (w.w >> (2 * u)) & m;
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 3; ++u) {
+                        const uint32_t mu = m << (2 * u);
+                        r[4 * u + 0] = w.x & mu;
+                        r[4 * u + 1] = w.z & mu;
+                        r[4 * u + 2] = w.y & mu;
+                        r[4 * u + 3] = w.w & mu;
+                    }
+                    r[12] = (w.x >> 6) & m;
+                    r[13] = (w.z >> 6) & m;
+                    r[14] = (w.y >> 6) & m;
+                    r[15] = (w.w >> 6) & m;
                 }
-                r[12] = (w.x >> 6) & m;
-                r[13] = (w.z >> 6) & m;
-                r[14] = (w.y >> 6) & m;
-                r[15] = (w.w >> 6) & m;
                 tmem_st16x256b_x4(tmem + 32 * (kGrp * aslot + j) + ((uint32_t)(32 * quarter + 16 * h) << 16), r);
             }
             tmem_wait_st();

@@ -162,11 +162,13 @@ constexpr int64_t kWsCtrBytes = 256;
 // do not fit one warp's registers); the others by as few as fill the GPU.
 constexpr int64_t kQuantSmallK = 1536;
 inline int tc_tokens(int64_t M) { return M <= 8 ? 8 : M <= 16 ? 16 : 32; }
-// Which decode kernel runs a sweep of M tokens (measured on B200: the
-// tensor-core sweep wins once the int8 MMAs of the register path, 4 per
-// 8 tokens per tile, and their operand loads no longer keep up with HBM).
+// Which decode kernel runs a sweep of M tokens (measured on B200 over the
+// 196 projections: the tensor-core sweep wins once the int8 MMAs of the
+// register path, 4 per 8 tokens per tile, and their operand loads no longer
+// keep up with HBM -- 115.7 / 117.8 us against 119.9 / 124.0 us at 12 / 16
+// tokens, 83 us for the register path at 8).
 #ifndef TW_TC_DECODE_MIN_M
-#define TW_TC_DECODE_MIN_M 17
+#define TW_TC_DECODE_MIN_M 9
 #endif
 inline bool decode_sweep_on_tensor_cores(int64_t M) { return M >= TW_TC_DECODE_MIN_M; }
 // Projections in the order their units are handed out (K descending); the

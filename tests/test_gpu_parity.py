@@ -296,9 +296,10 @@ def test_sweep_chunk_tails(dev, api, M):
         G.assert_y_close(d["y"].cpu().numpy(), ref["y"], f"M={M} N={N} K={K}")
 
 
-@pytest.mark.parametrize("M", [17, 20, 24, 31])
+@pytest.mark.parametrize("M", [9, 12, 16, 17, 20, 24, 31, 32])
 def test_sweep_tensor_core_decode_ragged(dev, api, M):
-    """The tensor-core decode kernel (17..32 tokens): every token-block width,
+    """The tensor-core decode kernel (9..32 tokens): every token-block width
+    (16 with four slot accumulators, 32 with one),
     projections whose N is not a multiple of 128 (the last 128-row unit
     partial, row blocks past N read as zero), several K, and the unit order
     (larger K first) different from the record order."""
