@@ -570,6 +570,46 @@ def _oracle_call_us(projs, M, budget_s):
                       f"{timed:.1f} s timed", **cpu_info()}
 
 
+def _oracle_i8_us(W, bias, x, M, budget_s):
+    """Microseconds per call of the oracle's I8_S layer over all M rows, from
+    the rows of x (a sample of the rows) run back to back for about budget_s
+    and extrapolated by row count."""
+    from oracle import oracle as orc
+    wq, amax_w = orc.i8_quantize_weights(W)
+    timed, passes = 0.0, 0
+    while timed < budget_s or passes == 0:
+        t0 = time.perf_counter()
+        orc.i8_linear(x, wq, amax_w, bias, relu=True)
+        timed += time.perf_counter() - t0
+        passes += 1
+    return {"value": timed / passes * 1e6 * M / x.shape[0], "unit": "us per call", "cores": 1,
+            "kind": "oracle", "sample": f"{x.shape[0]} of {M} token rows, {passes} passes, "
+            f"{timed:.1f} s timed; extrapolated by row count", **cpu_info()}
+
+
+def _oracle_chain_us(M, layers, budget_s):
+    """Microseconds per token step of the oracle's decoder-layer chain: one
+    layer (layer 0's projections) run back to back for about budget_s,
+    times the layer count."""
+    from oracle import oracle as orc
+    from ternary_weight_decoder_b200 import synth
+    layer = {}
+    for (l, p, name, N, K) in synth.sweep_shapes(1):
+        if (l, p) not in _ORACLE_CODES:
+            _ORACLE_CODES[(l, p)] = orc.ternarize(synth.weights(l, p, N, K))
+        layer[name] = _ORACLE_CODES[(l, p)]
+    h = synth.activations(0, 0, M, CHAIN_DIMS[0])
+    timed, passes = 0.0, 0
+    while timed < budget_s or passes == 0:
+        t0 = time.perf_counter()
+        orc.decoder_layer(h, layer, head_dim=CHAIN_DIMS[2])
+        timed += time.perf_counter() - t0
+        passes += 1
+    return {"value": timed / passes * 1e6 * layers, "unit": "us per step", "cores": 1,
+            "kind": "oracle", "sample": f"1 of {layers} layers, {M} token(s), {passes} passes, "
+            f"{timed:.1f} s timed; extrapolated by layer count", **cpu_info()}
+
+
 def cpu_oracle_sample(M, budget_s=10.0, sample_layers=4, layers=28):
     """Headline CPU baseline: the oracle over all rows of the projections
     of the first `sample_layers` layers at M tokens."""
@@ -794,6 +834,9 @@ def measure_configs(args, api, torch, dev, rank, shapes, weights, descs_m1, want
                                  "W ~ N(0, 0.05^2); bias ~ N(0, 0.1^2)",
                 "note": "gemm: int8 activations quantised beforehand; layer: fp32 activations "
                         "quantised in the call (two launches)"}
+            if cpu_ok:
+                out[f"i8_linear_bias_relu_M{M}_K{K}_N{N}"]["oracle"] = _oracle_i8_us(
+                    W, bias.cpu().numpy(), xr[:64].cpu().numpy(), M, 2.0)
             del W, wq, xq, x, xr, y, ws
             torch.cuda.empty_cache()
 
@@ -824,6 +867,8 @@ def measure_configs(args, api, torch, dev, rank, shapes, weights, descs_m1, want
             "note": "28 dependent layers from one token state (the +1 launch copies it in); "
                     "fused: one persistent launch, 112 grid-wide barriers; unfused: per layer "
                     "4 sweeps and 4 element-wise launches"}
+        if cpu_ok:
+            out["chain_28L_M1"]["oracle"] = _oracle_chain_us(M, args.layers, 3.0)
         del chain
     return out
 
