@@ -169,7 +169,9 @@ TW_API int tw_ternary_linear(const float *x, int64_t M, int64_t N, int64_t K,
 
 /*
  * Same product on activations already quantised by tw_quantize_act:
- * xq [M x K] int8, amax [M] fp32, qsum [M] int32 (required).
+ * xq [M x K] int8, amax [M] fp32, qsum [M] int32 (required).  ws and
+ * ws_bytes are not used (NULL and 0 are fine); they keep the argument list
+ * of tw_ternary_linear.
  */
 TW_API int tw_ternary_linear_q(const int8_t *xq, const float *amax,
                         const int32_t *qsum, int64_t M, int64_t N, int64_t K,
@@ -179,11 +181,15 @@ TW_API int tw_ternary_linear_q(const int8_t *xq, const float *amax,
 
 /*
  * One projection of a decoder sweep.  All pointers are device pointers.
- * Decode sweeps (M <= 32) read x; prefill sweeps (M > 32) read xq, amax and
- * qsum (from tw_quantize_act) and ignore x.
+ * Decode sweeps (M <= 32) read x.  Sweeps of more than 32 tokens read xq,
+ * amax and qsum: either as given (from tw_quantize_act; x NULL) or, when x
+ * is given too, as written by the sweep itself, which then quantises every
+ * such x into its xq, amax and qsum (R2-R4, the same bits as
+ * tw_quantize_act) in one launch over all projections before the GEMM.
  */
 typedef struct tw_proj_desc {
-    const float *x;        /* [M x K] fp32 activations (decode)            */
+    const float *x;        /* [M x K] fp32 activations (decode; prefill:   */
+                           /* optional, quantised into xq/amax/qsum)       */
     const int8_t *xq;      /* [M x K] int8 activations (prefill)           */
     const float *amax;     /* [M] absmax that goes with xq (prefill)       */
     const int32_t *qsum;   /* [M] row sums of xq (prefill)                 */
@@ -233,7 +239,8 @@ TW_API size_t tw_sweep_workspace_bytes(const void *table_host);
  * weights in tensor memory (units of 128 weight rows x 128 tokens, claimed
  * from the counters in the workspace); more tokens: one persistent
  * tensor-core launch with the weights expanded in shared memory (output
- * tiles of 128 tokens x 256 weight rows dealt out round robin).
+ * tiles of 128 tokens x 256 weight rows dealt out round robin).  Either is
+ * preceded by one quantisation launch when some descriptor gives x.
  *   table_host  the host table written by tw_sweep_table_encode (read for the
  *               launch configuration: count, M, sizes);
  *   table_dev   the caller's device copy of the same bytes (64-byte aligned),

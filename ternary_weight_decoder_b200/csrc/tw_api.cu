@@ -595,6 +595,19 @@ size_t tw_sweep_workspace_bytes(const void *table_host)
     return (size_t)hdr->ws_bytes;
 }
 
+// Whether a sweep of more than 32 tokens quantises some descriptor's fp32 x
+// itself (first launch) before the GEMM.
+static bool sweep_quantises_x(const tw::TableHeader *hdr)
+{
+    if (hdr->M <= tw::kDecodeMaxM)
+        return false;
+    const auto *recs = reinterpret_cast<const tw::DescRecord *>(hdr + 1);
+    for (int d = 0; d < hdr->count; ++d)
+        if (recs[d].x)
+            return true;
+    return false;
+}
+
 // Projections of a host table with K > kQuantSmallK (they lead the unit order).
 static int big_k_projections(const tw::TableHeader *hdr)
 {
@@ -627,6 +640,11 @@ int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, v
             return fail(TW_ERR_ALIGN, "sweep workspace must be 16-byte aligned");
         const auto *recs_dev = reinterpret_cast<const tw::DescRecord *>(
             static_cast<const tw::TableHeader *>(table_dev) + 1);
+        if (sweep_quantises_x(hdr)) {
+            cudaError_t e = tw::launch_quant_own(recs_dev, hdr->count, hdr->M, stream);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "sweep quantisation launch");
+        }
         tw::MidLaunch P{};
         P.table = recs_dev;
         P.order = reinterpret_cast<const tw::UnitOrder *>(recs_dev + hdr->count);
@@ -641,6 +659,11 @@ int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, v
         tw::PrefillLaunch P{};
         P.table = reinterpret_cast<const tw::DescRecord *>(
             static_cast<const tw::TableHeader *>(table_dev) + 1);
+        if (sweep_quantises_x(hdr)) {
+            cudaError_t e = tw::launch_quant_own(P.table, hdr->count, hdr->M, stream);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "sweep quantisation launch");
+        }
         P.single = nullptr;
         P.count = hdr->count;
         P.M = hdr->M;
@@ -695,7 +718,7 @@ int tw_sweep_launches(const void *table_host)
     if (!hdr || hdr->magic != tw::kTableMagic)
         return 0;
     if (hdr->M > tw::kDecodeMaxM)
-        return 1;
+        return sweep_quantises_x(hdr) ? 2 : 1;
     const int n_big = big_k_projections(hdr);
     if (!tw::decode_sweep_on_tensor_cores(hdr->M))
         return tw::decode_launches(hdr->count, hdr->M, hdr->max_K, n_big);

@@ -89,6 +89,9 @@ struct QuantParams {
     const UnitOrder *order;   // null: projection i is record i; else order[i0 + i].d
     int i0;
     int wait_prev;            // wait for the preceding launch before finishing
+    int own;                  // 1: q, amax and sum(q) go to each record's own xq, amax
+                              // and qsum (sweeps of more than 32 tokens given fp32 x);
+                              // records without x are skipped
     uint8_t *ws;
     int64_t ws_sa_off;
 };
@@ -159,13 +162,15 @@ __global__ void __launch_bounds__(kQThreads) k_quant_rows(const __grid_constant_
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wpr = p.wpr, rloc = warp / wpr, wr = warp % wpr;
     const int64_t row_id = (int64_t)blockIdx.x * (kQThreads / 32 / wpr) + rloc;
-    const bool live = row_id < (int64_t)p.count * p.M;
-    const int pi = live ? (int)(row_id / p.M) : 0, m = live ? (int)(row_id % p.M) : 0;
+    const bool in_range = row_id < (int64_t)p.count * p.M;
+    const int pi = in_range ? (int)(row_id / p.M) : 0, m = in_range ? (int)(row_id % p.M) : 0;
     const int d = p.order ? p.order[p.i0 + pi].d : pi;
     const DescRecord &r = rec(p, d);
+    const bool live = in_range && (!p.own || r.x != nullptr);
     const int64_t K4 = live ? r.K / 4 : 0;
     const float4 *row = reinterpret_cast<const float4 *>(r.x + (int64_t)m * r.K);
-    uint32_t *qrow = reinterpret_cast<uint32_t *>(p.ws + r.ws_xq_off + (int64_t)m * r.K);
+    uint32_t *qrow = p.own ? reinterpret_cast<uint32_t *>(const_cast<int8_t *>(r.xq) + (int64_t)m * r.K)
+                           : reinterpret_cast<uint32_t *>(p.ws + r.ws_xq_off + (int64_t)m * r.K);
     const int T = 32 * wpr, ti = 32 * wr + lane;   // threads of the row, index within it
     const bool in_regs = K4 <= (int64_t)kQRegs * T;
 
@@ -253,9 +258,14 @@ __global__ void __launch_bounds__(kQThreads) k_quant_rows(const __grid_constant_
             sum += red_i[rloc * wpr + w];
     }
     if (live && ti == 0) {
-        uint8_t *info = p.ws + p.ws_sa_off + 256 * (int64_t)d;
-        reinterpret_cast<float *>(info)[m] = __fdiv_rn(a, 127.f);
-        reinterpret_cast<int *>(info + 128)[m] = sum;
+        if (p.own) {
+            const_cast<float *>(r.amax)[m] = a;
+            const_cast<int32_t *>(r.qsum)[m] = sum;
+        } else {
+            uint8_t *info = p.ws + p.ws_sa_off + 256 * (int64_t)d;
+            reinterpret_cast<float *>(info)[m] = __fdiv_rn(a, 127.f);
+            reinterpret_cast<int *>(info + 128)[m] = sum;
+        }
     }
     // This launch overlaps the preceding one (programmatic dependent launch);
     // it completes only after that one has, so that waiting for this launch
@@ -812,6 +822,17 @@ cudaError_t launch_plan(const DecodeParams &p, const DecodePlan &g, int grid, in
 int quant_launches(int64_t count, int64_t M, int n_big)
 {
     return quant_launches_impl(count, M, n_big);
+}
+
+cudaError_t launch_quant_own(const DescRecord *table, int count, int64_t M, cudaStream_t stream)
+{
+    QuantParams q;
+    memset(&q, 0, sizeof(q));
+    q.table = table;
+    q.count = count;
+    q.M = (int)M;
+    q.own = 1;
+    return launch_quant_rows(q, 0, stream);
 }
 
 cudaError_t launch_quant_tc(const DescRecord *table, const UnitOrder *order, int n_big, int count,

@@ -192,6 +192,10 @@ struct DecodeTcLaunch {
 cudaError_t launch_decode_tc(const DecodeTcLaunch &L, uint32_t *err, uint64_t timeout_ns,
                              cudaStream_t stream);
 // Quantise every (projection, token) row into the token blocks above.
+// Quantise every record's fp32 x (records without x are skipped) into its
+// own xq, amax and qsum: the first launch of a sweep of more than 32 tokens
+// whose descriptors give x.
+cudaError_t launch_quant_own(const DescRecord *table, int count, int64_t M, cudaStream_t stream);
 cudaError_t launch_quant_tc(const DescRecord *table, const UnitOrder *order, int n_big, int count,
                             int64_t M, int ntok, uint8_t *ws, int64_t ws_sa_off, cudaStream_t stream);
 inline int64_t round128(int64_t b) { return (b + 127) / 128 * 128; }

@@ -6,9 +6,10 @@
 // s = 1/mean|W|; codes are -1, 0 or +1 ("The Paper Says ARM Support" post,
 // "What the model is trying to do").  mean|W| is accumulated in fp64 in a
 // fixed order (each row over k, then the rows over n) so that the codes do
-// not depend on how the sum is scheduled; the sum is offline work done once
-// per matrix, so the first stage is one thread per row and the second one
-// thread in total.
+// not depend on how the sum is scheduled: one thread per row adds its row
+// in k order, one thread adds the row sums in n order.  Both stage their
+// operands through shared memory with coalesced loads, so that only the
+// chains of dependent fp64 additions remain serial.
 #include "tw_device.cuh"
 #include "tw_internal.h"
 
@@ -17,32 +18,72 @@ namespace {
 
 constexpr double kMeanFloor = 1e-5;
 
-__global__ void k_row_abs_sum(const float *__restrict__ W, int64_t N, int64_t K,
-                              double *__restrict__ rowsum, uint32_t *err)
+constexpr int kRowsPerBlock = 128;   // one thread per row; 4 warps
+constexpr int kSumChunk = 32;        // k per staged chunk (K is a multiple of 128)
+
+// Rows n0 .. n0 + 127 of the block: per chunk of 32 k, warp w loads rows
+// 32w .. 32w + 31 with one coalesced 128-byte load each (lane = k), then
+// thread t adds row t's 32 values in k order.
+__global__ void __launch_bounds__(kRowsPerBlock) k_row_abs_sum(const float *__restrict__ W, int64_t N,
+                                                               int64_t K, double *__restrict__ rowsum,
+                                                               uint32_t *err)
 {
-    const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (n >= N)
-        return;
-    const float *row = W + n * K;
+    __shared__ float tile[kRowsPerBlock][kSumChunk + 1];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n0 = (int64_t)blockIdx.x * kRowsPerBlock;
+    const int64_t n = n0 + threadIdx.x;
     double s = 0.0;
     bool finite = true;
-    for (int64_t k = 0; k < K; ++k) {
-        const float v = __ldg(row + k);
-        finite &= isfinite(v);
-        s = __dadd_rn(s, fabs((double)v));
+    for (int64_t k0 = 0; k0 < K; k0 += kSumChunk) {
+        float v[32];
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+            const int64_t row = n0 + 32 * warp + r;
+            v[r] = row < N ? __ldg(W + row * K + k0 + lane) : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+            tile[32 * warp + r][lane] = v[r];
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < kSumChunk; ++j) {
+            const float x = tile[threadIdx.x][j];
+            finite &= isfinite(x);
+            s = __dadd_rn(s, fabs((double)x));
+        }
+        __syncthreads();
     }
-    rowsum[n] = s;
-    if (!finite)
-        atomicOr(err, EFLAG_NONFINITE);
+    if (n < N) {
+        rowsum[n] = s;
+        if (!finite)
+            atomicOr(err, EFLAG_NONFINITE);
+    }
 }
 
 // ws layout: [0] double s = 1/mean; [32..] row sums.
-__global__ void k_total(const double *__restrict__ rowsum, int64_t N, int64_t K, double *s_out,
-                        double *mean_abs, float *wscale)
+constexpr int kTotalThreads = 256;
+constexpr int kTotalChunk = 2048;    // row sums staged per step (16 KB)
+
+// The block stages the row sums through shared memory; thread 0 adds them
+// in n order.
+__global__ void __launch_bounds__(kTotalThreads) k_total(const double *__restrict__ rowsum, int64_t N,
+                                                         int64_t K, double *s_out, double *mean_abs,
+                                                         float *wscale)
 {
+    __shared__ double buf[kTotalChunk];
     double t = 0.0;
-    for (int64_t n = 0; n < N; ++n)
-        t = __dadd_rn(t, rowsum[n]);
+    for (int64_t n0 = 0; n0 < N; n0 += kTotalChunk) {
+        const int cnt = (int)(N - n0 < kTotalChunk ? N - n0 : kTotalChunk);
+        for (int i = threadIdx.x; i < cnt; i += kTotalThreads)
+            buf[i] = rowsum[n0 + i];
+        __syncthreads();
+        if (threadIdx.x == 0)
+            for (int i = 0; i < cnt; ++i)
+                t = __dadd_rn(t, buf[i]);
+        __syncthreads();
+    }
+    if (threadIdx.x != 0)
+        return;
     double mean = __ddiv_rn(t, (double)(N * K));
     if (!(mean >= kMeanFloor))
         mean = kMeanFloor;
@@ -138,9 +179,9 @@ cudaError_t launch_ternarize(const float *W, int64_t N, int64_t K, uint8_t *pack
 {
     double *s_ptr = reinterpret_cast<double *>(ws);
     double *rowsum = reinterpret_cast<double *>(static_cast<char *>(ws) + 256);
-    const int threads = 128;
-    k_row_abs_sum<<<(unsigned)ceil_div(N, threads), threads, 0, stream>>>(W, N, K, rowsum, err);
-    k_total<<<1, 1, 0, stream>>>(rowsum, N, K, s_ptr, mean_abs, wscale);
+    k_row_abs_sum<<<(unsigned)ceil_div(N, kRowsPerBlock), kRowsPerBlock, 0, stream>>>(W, N, K, rowsum,
+                                                                                      err);
+    k_total<<<1, kTotalThreads, 0, stream>>>(rowsum, N, K, s_ptr, mean_abs, wscale);
     const int64_t n_words = ceil_div(N, kTileRows) * kTileRows * K / 16;
     k_pack<<<(unsigned)ceil_div(n_words, 256), 256, 0, stream>>>(
         W, N, K, s_ptr, reinterpret_cast<uint32_t *>(packed), n_words);

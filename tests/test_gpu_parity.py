@@ -329,6 +329,59 @@ def test_sweep_tensor_core_decode_ragged(dev, api, M):
             d["acc_out"].fill_(int(POISON_I32))
 
 
+@pytest.mark.parametrize("M", [33, 200, 300])
+def test_sweep_more_tokens_from_fp32_x(dev, api, M):
+    """Sweeps of more than 32 tokens given fp32 x (weights-in-tensor-memory
+    kernel at 33 and 200 tokens, expanded-weights kernel at 300): the sweep
+    quantises x into each descriptor's xq, amax and qsum (bit-exact against
+    the oracle's R2-R4) before the product; a descriptor given xq without x
+    in the same table is used as given (and left as it was)."""
+    import torch
+    shapes = [(200, 256), (128, 1536), (17, 384), (385, 640), (256, 2048), (1, 128)]
+    descs, keep = [], []
+    for i, (N, K) in enumerate(shapes):
+        W = _weights(N, K, 7000 + 10 * M + i)
+        x = _acts(M, K, 7500 + 10 * M + i)
+        packed, _, wscale = G.ternarize_gpu(W, dev)
+        from_x = i % 3 != 2
+        if from_x:
+            xq = torch.full((M, K), -77, dtype=torch.int8, device=dev)
+            amax = torch.full((M,), float("nan"), dtype=torch.float32, device=dev)
+            qsum = torch.full((M,), int(POISON_I32), dtype=torch.int32, device=dev)
+            xd = G.to_dev(x, dev)
+        else:
+            xq, amax, qsum = api.quantize_act(G.to_dev(x, dev))
+            xd = None
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+        acc = torch.full((M, N), int(POISON_I32), dtype=torch.int32, device=dev)
+        d = dict(xq=xq, amax=amax, qsum=qsum, packed=packed, wscale=wscale, y=y, acc_out=acc,
+                 N=N, K=K)
+        if xd is not None:
+            d["x"] = xd
+        descs.append(d)
+        keep.append((W, x, from_x))
+    table = api.SweepTable(descs, M, device=dev)
+    assert table.launches == 2
+    for _ in range(2):
+        api.decoder_projection_sweep(table)
+        api.check()
+        for d, (W, x, from_x) in zip(descs, keep):
+            q_ref, amax_ref = orc.quantize_act(x)
+            assert np.array_equal(d["xq"].cpu().numpy(), q_ref), (M, d["N"], d["K"], from_x)
+            assert np.array_equal(d["amax"].cpu().numpy(), amax_ref), (M, d["K"], from_x)
+            assert np.array_equal(d["qsum"].cpu().numpy(),
+                                  q_ref.astype(np.int64).sum(axis=1).astype(np.int32))
+            codes, mean = orc.ternarize(W)
+            ref = orc.ternary_linear(x, codes, mean)
+            assert (d["acc_out"].cpu().numpy() == ref["acc"]).all(), (M, d["N"], d["K"])
+            G.assert_y_close(d["y"].cpu().numpy(), ref["y"], f"M={M} N={d['N']} K={d['K']}")
+        for d, (_, _, from_x) in zip(descs, keep):
+            d["y"].fill_(float("nan"))
+            d["acc_out"].fill_(int(POISON_I32))
+            if from_x:
+                d["xq"].fill_(-77)
+
+
 # ------------------------------------------------------------ errors
 def test_wait_timeout_is_reported(dev, api):
     api.debug_wait_timeout(2_000_000)   # 2 ms; nothing ever arrives
