@@ -52,14 +52,59 @@ constexpr int kS = 3;                      // ring slots per warp
 constexpr int kThreadsCh = kNW * 32;
 constexpr int kSlotBytes = kCT * kTileBytes;
 constexpr uint64_t kDrainNsCh = 1000000000ull;
+// A stage input row of up to kXR float4 per thread (K <= 10240) for up to
+// kRegTokens tokens stays in registers between the amax and the
+// quantisation passes; each pass then issues all its loads at once.
+constexpr int kXR = 5;
+constexpr int kRegTokens = 2;
+// The down projection's input as read back by the quantisation: SiLU(g) * u
+// is computed once, by the CTA whose slice of `act` holds it (materialise),
+// and after a grid-wide barrier read by every CTA (measured on B200: every
+// CTA computing the whole row took 7 us per down stage).
+constexpr int kStageDownAct = 4;
 
 struct ChainParams {
     const ChainPlanHeader *plan;
     uint8_t *ws;
     int m0, mg;                 // token group [m0, m0 + mg)
     int xstride;                // bytes per activation row in shared memory (max_K + 64)
+    int unit_cache;             // the stages' unit fields are copied to shared memory
     WaitCtl ctl;
 };
+
+// What a warp's walk over its units needs of each stage -- this CTA's range
+// [lo, hi) of the stage's units among them -- computed once per stage and
+// kept in shared memory when it fits (measured on B200: read from the plan
+// in global memory with two 64-bit divisions per step, a warp's step from
+// its last unit of a stage to its first of the next took 0.6-1 us, on every
+// stage's critical path).
+struct UnitS {
+    int lo, hi, nch, KT;
+    int rb_off[4];              // first row block of each projection; past nproj: the total
+    const uint8_t *packed[3];
+    int nproj, pad;
+};
+static_assert(sizeof(UnitS) == 64, "unit cache entry");
+
+__device__ __forceinline__ UnitS unit_fields(const ChainStagePlan *st)
+{
+    UnitS u;
+    const int64_t units = st->units;
+    u.lo = (int)(units * blockIdx.x / gridDim.x);
+    u.hi = (int)(units * (blockIdx.x + 1) / gridDim.x);
+    u.nch = st->nch;
+    u.KT = st->K / kTileK;
+    u.nproj = st->nproj;
+    // entries past the stage's projections hold the total, so where() never
+    // picks them
+    for (int q = 0; q < 3; ++q) {
+        u.rb_off[q] = q < u.nproj ? (int)st->proj[q].rb_off : (int)st->rb_total;
+        u.packed[q] = st->proj[q].packed;
+    }
+    u.rb_off[3] = (int)st->rb_total;
+    u.pad = 0;
+    return u;
+}
 
 __device__ __forceinline__ const ChainStagePlan *stage_of(const ChainPlanHeader *h, int s)
 {
@@ -116,28 +161,23 @@ struct UnitIter {
     int rb_off[4];
     const uint8_t *packed[3];
     bool valid;
+    const UnitS *cache;         // the stages' unit fields in shared memory, or null
 
     __device__ void enter(const ChainPlanHeader *h, int stage, int w)
     {
         valid = false;
         for (s = stage; s < n_stages; ++s) {
-            const ChainStagePlan *st = stage_of(h, s);
-            const int units = (int)st->units;
-            const int c = blockIdx.x, G = gridDim.x;
-            const int lo = (int)((int64_t)units * c / G);
-            hi = (int)((int64_t)units * (c + 1) / G);
-            u = lo + w;
+            const UnitS f = cache ? cache[s] : unit_fields(stage_of(h, s));
+            hi = f.hi;
+            u = f.lo + w;
             if (u < hi) {
-                nch = st->nch;
-                KT = st->K / kTileK;
-                nproj = st->nproj;
-                // rb_off[q] = first row block of projection q; entries past the
-                // stage's projections hold the total, so where() never picks them
-                for (int q = 0; q < 3; ++q) {
-                    rb_off[q] = q < nproj ? (int)st->proj[q].rb_off : (int)st->rb_total;
-                    packed[q] = st->proj[q].packed;
-                }
-                rb_off[3] = (int)st->rb_total;
+                nch = f.nch;
+                KT = f.KT;
+                nproj = f.nproj;
+                for (int q = 0; q < 4; ++q)
+                    rb_off[q] = f.rb_off[q];
+                for (int q = 0; q < 3; ++q)
+                    packed[q] = f.packed[q];
                 valid = true;
                 return;
             }
@@ -227,9 +267,81 @@ __device__ __forceinline__ float4 stage_x4(const ChainPlanHeader *h, int kind, b
     }
     case kStageGU:
         return add4(ldcg4f(h->h + mrow * h->hidden + k), prev_y4(P, 0, m, k));
+    case kStageDownAct:
+        return ldcg4f(h->act + mrow * h->inter + k);
     default: {   // kStageDown: SiLU(g) * u
         const float4 g = prev_y4(P, 0, m, k);
         const float4 u = prev_y4(P, 1, m, k);
+        return make_float4(silu_mul1(g.x, u.x), silu_mul1(g.y, u.y), silu_mul1(g.z, u.z),
+                           silu_mul1(g.w, u.w));
+    }
+    }
+}
+
+// The same value as stage_x4, in two steps: stage_raw issues the loads
+// (up to two 16-byte words: a = h, h1 or the sums of projection 0; b = the
+// sums of the projection the step reads), stage_val computes from them.  A
+// caller that loads all its elements before computing any has one L2
+// round trip in flight instead of one per element.
+__device__ __forceinline__ void stage_raw(const ChainPlanHeader *h, int kind, bool first_layer,
+                                          const Prev &P, int m, int mrow, int64_t i, int4 &a, int4 &b)
+{
+    const int64_t k = 4 * i;
+    switch (kind) {
+    case kStageQKV:
+        if (first_layer) {
+            a = ldcg4i(reinterpret_cast<const int32_t *>(h->h + mrow * h->hidden + k));
+        } else {
+            a = ldcg4i(reinterpret_cast<const int32_t *>(h->h1 + mrow * h->hidden + k));
+            b = ldcg4i(P.sum + (int64_t)m * P.ntot + P.st->proj[0].noff + k);
+        }
+        break;
+    case kStageO: {
+        const int64_t group = (h->hidden / h->head_dim) / (h->kv_dim / h->head_dim);
+        const int64_t head = k / h->head_dim, c = k - head * h->head_dim;
+        b = ldcg4i(P.sum + (int64_t)m * P.ntot + P.st->proj[2].noff + (head / group) * h->head_dim + c);
+        break;
+    }
+    case kStageGU:
+        a = ldcg4i(reinterpret_cast<const int32_t *>(h->h + mrow * h->hidden + k));
+        b = ldcg4i(P.sum + (int64_t)m * P.ntot + P.st->proj[0].noff + k);
+        break;
+    case kStageDownAct:
+        a = ldcg4i(reinterpret_cast<const int32_t *>(h->act + mrow * h->inter + k));
+        break;
+    default:
+        a = ldcg4i(P.sum + (int64_t)m * P.ntot + P.st->proj[0].noff + k);
+        b = ldcg4i(P.sum + (int64_t)m * P.ntot + P.st->proj[1].noff + k);
+        break;
+    }
+}
+
+__device__ __forceinline__ float4 rescale4(int4 D, const Prev &P, int q, int m)
+{
+    const float ws = P.ws[q];
+    return make_float4(rescale1(D.x, P.qs[m], P.sa[m], ws), rescale1(D.y, P.qs[m], P.sa[m], ws),
+                       rescale1(D.z, P.qs[m], P.sa[m], ws), rescale1(D.w, P.qs[m], P.sa[m], ws));
+}
+
+__device__ __forceinline__ float4 as_f4(int4 a)
+{
+    return make_float4(__int_as_float(a.x), __int_as_float(a.y), __int_as_float(a.z), __int_as_float(a.w));
+}
+
+__device__ __forceinline__ float4 stage_val(int kind, bool first_layer, const Prev &P, int m, int4 a,
+                                            int4 b)
+{
+    switch (kind) {
+    case kStageQKV:
+        return first_layer ? as_f4(a) : add4(as_f4(a), rescale4(b, P, 0, m));
+    case kStageO:
+        return rescale4(b, P, 2, m);
+    case kStageGU:
+        return add4(as_f4(a), rescale4(b, P, 0, m));
+    case kStageDownAct:
+        return as_f4(a);
+    default: {
+        const float4 g = rescale4(a, P, 0, m), u = rescale4(b, P, 1, m);
         return make_float4(silu_mul1(g.x, u.x), silu_mul1(g.y, u.y), silu_mul1(g.z, u.z),
                            silu_mul1(g.w, u.w));
     }
@@ -252,13 +364,15 @@ __device__ __forceinline__ uint32_t quant4c(float4 v, float scale, bool zero, in
 
 // Write this CTA's slice of an [mg x width] materialised buffer: element e
 // of the slice has value fn(m, j) for m = e / width, j = e % width (width a
-// multiple of 4; written 4 at a time).
+// multiple of 4; written 4 at a time) -- by threads tid = 0 .. nt - 1 of a
+// group of the CTA's warps.
 template <class F>
-__device__ __forceinline__ void write_slice(float *dst, int64_t width, int mg, int m0, F fn)
+__device__ __forceinline__ void write_slice(float *dst, int64_t width, int mg, int m0, int tid, int nt,
+                                            F fn)
 {
     const int64_t n4 = (int64_t)mg * width / 4;
     const int64_t lo = n4 * blockIdx.x / gridDim.x, hi = n4 * (blockIdx.x + 1) / gridDim.x;
-    for (int64_t e = lo + threadIdx.x; e < hi; e += kThreadsCh) {
+    for (int64_t e = lo + tid; e < hi; e += nt) {
         const int m = (int)(e / (width / 4));
         const int64_t j = 4 * (e - (int64_t)m * (width / 4));
         *reinterpret_cast<float4 *>(dst + (int64_t)(m0 + m) * width + j) = fn(m, j);
@@ -266,7 +380,7 @@ __device__ __forceinline__ void write_slice(float *dst, int64_t width, int mg, i
 }
 
 // This CTA's slice of the previous stage's integer outputs into acc_out.
-__device__ __forceinline__ void write_acc_slice(const Prev &P, int q, int mg, int m0)
+__device__ __forceinline__ void write_acc_slice(const Prev &P, int q, int mg, int m0, int tid, int nt)
 {
     const ChainProj &pr = P.st->proj[q];
     if (!pr.acc_out)
@@ -274,7 +388,7 @@ __device__ __forceinline__ void write_acc_slice(const Prev &P, int q, int mg, in
     const int64_t width = pr.N;
     const int64_t n = (int64_t)mg * width;
     const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
-    for (int64_t e = lo + threadIdx.x; e < hi; e += kThreadsCh) {
+    for (int64_t e = lo + tid; e < hi; e += nt) {
         const int m = (int)(e / width);
         const int64_t j = e - (int64_t)m * width;
         pr.acc_out[(int64_t)(m0 + m) * width + j] =
@@ -283,32 +397,43 @@ __device__ __forceinline__ void write_acc_slice(const Prev &P, int q, int mg, in
 }
 
 // Materialise the outputs of the previous stage (every projection's y and
-// acc_out) and the step values of this prologue, each CTA its slice.
+// acc_out) and the step values of this prologue, each CTA its slice.  The
+// pieces (one per previous projection, one for the step values) go to
+// disjoint groups of the CTA's warps, so that their L2 round trips overlap
+// (measured on B200: 4.0 us per stage one after another).
 __device__ void materialise(const ChainPlanHeader *h, int kind, bool first_layer, bool final_phase,
                             const Prev &P, int mg, int m0)
 {
-    if (P.st) {
-        for (int q = 0; q < P.st->nproj; ++q) {
-            write_slice(P.st->proj[q].y, P.st->proj[q].N, mg, m0,
-                        [&](int m, int64_t j) { return prev_y4(P, q, m, j); });
-            write_acc_slice(P, q, mg, m0);
-        }
-    }
-    if (final_phase || (kind == kStageQKV && !first_layer)) {
+    const int nprev = P.st ? P.st->nproj : 0;
+    const bool step = final_phase || (kind == kStageQKV && !first_layer) || kind == kStageO ||
+                      kind == kStageGU || kind == kStageDown;
+    const int nc = nprev + (step ? 1 : 0);
+    if (nc == 0)
+        return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = warp % nc;                                  // this warp's piece
+    const int tid = (warp / nc) * 32 + lane;                  // its index in the group
+    const int nt = ((kNW - 1 - c) / nc + 1) * 32;             // threads of the group
+    if (c < nprev) {
+        const int q = c;
+        write_slice(P.st->proj[q].y, P.st->proj[q].N, mg, m0, tid, nt,
+                    [&](int m, int64_t j) { return prev_y4(P, q, m, j); });
+        write_acc_slice(P, q, mg, m0, tid, nt);
+    } else if (final_phase || (kind == kStageQKV && !first_layer)) {
         // h' = h1 + d
-        write_slice(h->h, h->hidden, mg, m0, [&](int m, int64_t j) {
+        write_slice(h->h, h->hidden, mg, m0, tid, nt, [&](int m, int64_t j) {
             return add4(ldcg4f(h->h1 + (int64_t)(m0 + m) * h->hidden + j), prev_y4(P, 0, m, j));
         });
     } else if (kind == kStageO) {
-        write_slice(h->a, h->hidden, mg, m0, [&](int m, int64_t j) {
+        write_slice(h->a, h->hidden, mg, m0, tid, nt, [&](int m, int64_t j) {
             return stage_x4(h, kStageO, false, P, m, m0 + m, j / 4);
         });
     } else if (kind == kStageGU) {
-        write_slice(h->h1, h->hidden, mg, m0, [&](int m, int64_t j) {
+        write_slice(h->h1, h->hidden, mg, m0, tid, nt, [&](int m, int64_t j) {
             return stage_x4(h, kStageGU, false, P, m, m0 + m, j / 4);
         });
-    } else if (kind == kStageDown) {
-        write_slice(h->act, h->inter, mg, m0, [&](int m, int64_t j) {
+    } else {
+        write_slice(h->act, h->inter, mg, m0, tid, nt, [&](int m, int64_t j) {
             return stage_x4(h, kStageDown, false, P, m, m0 + m, j / 4);
         });
     }
@@ -327,9 +452,11 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
     float *sa_s = reinterpret_cast<float *>(xbuf + kChainGroup * p.xstride);   // [8] this stage
     int *qs_s = reinterpret_cast<int *>(sa_s + kChainGroup);                   // [8]
     float *scale_s = reinterpret_cast<float *>(qs_s + kChainGroup);            // [8] 127/amax
-    float *psa_s = scale_s + kChainGroup;                                      // [8] previous stage
-    int *pqs_s = reinterpret_cast<int *>(psa_s + kChainGroup);                 // [8]
-    float *pws_s = reinterpret_cast<float *>(pqs_s + kChainGroup);             // [4] its wscales
+    // amax/127 and sum(q) of stage s's input at [s & 1] (a stage's outputs
+    // are materialised after the next stage's prologue has written its own)
+    float *psa2 = scale_s + kChainGroup;                                       // [2][8]
+    int *pqs2 = reinterpret_cast<int *>(psa2 + 2 * kChainGroup);               // [2][8]
+    float *pws_s = reinterpret_cast<float *>(pqs2 + 2 * kChainGroup);          // [4] wscales
     float *red_f = pws_s + 4 + 4;                                              // [kNW][8]
     int *red_i = reinterpret_cast<int *>(red_f + kNW * kChainGroup);           // [kNW][8]
     uint64_t *bars = reinterpret_cast<uint64_t *>(
@@ -337,6 +464,11 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
     int *abort_p = reinterpret_cast<int *>(bars + kNW * kS);
     volatile int *abort_flag = abort_p;
     const uint32_t bar_ring = smem_u32(bars);
+    UnitS *ucache = reinterpret_cast<UnitS *>(
+        (reinterpret_cast<uintptr_t>(abort_p + 1) + 63) & ~uintptr_t(63));
+    if (p.unit_cache)
+        for (int i = threadIdx.x; i < h->n_stages; i += kThreadsCh)
+            ucache[i] = unit_fields(stage_of(h, i));
 
     uint32_t *ctr = reinterpret_cast<uint32_t *>(p.ws);
     const int64_t buf_ints = (kChainGroup * h->max_ntot * 4 + 255) / 256 * 64;
@@ -360,6 +492,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
     const uint32_t bar_w = bar_ring + 8 * warp * kS;
     UnitIter prod, cons;
     prod.n_stages = h->n_stages;
+    prod.cache = p.unit_cache ? ucache : nullptr;
     prod.enter(h, 0, warp);
     cons = prod;
     int issued = 0, consumed = 0;
@@ -386,8 +519,8 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
     P.st = nullptr;
     P.sum = nullptr;
     P.ntot = 0;
-    P.sa = psa_s;
-    P.qs = pqs_s;
+    P.sa = psa2;
+    P.qs = pqs2;
     P.ws = pws_s;
 
     for (int s = 0; s <= h->n_stages && ok; ++s) {
@@ -395,36 +528,138 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
         const ChainStagePlan *st = final_phase ? nullptr : stage_of(h, s);
         const int kind = final_phase ? -1 : st->kind;
         const bool first_layer = s < 4;
+        // The plan entries of the next stages, into this SM's L1 (the units
+        // of stage s walk into stage s + 1's, the ring's producer further).
+        if (threadIdx.x < 8 && s + 1 + (threadIdx.x >> 1) < h->n_stages)
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const uint8_t *>(
+                             stage_of(h, s + 1 + (threadIdx.x >> 1))) + 128 * (threadIdx.x & 1)));
         if (s > 0) {
+            // (pws_s holds stage s - 1's wscales, loaded before the barrier)
             P.st = stage_of(h, s - 1);
             P.sum = sum_buf(s - 1);
             P.ntot = P.st->ntot;
-            if (threadIdx.x < P.st->nproj)
-                pws_s[threadIdx.x] = __ldg(P.st->proj[threadIdx.x].wscale);
-            __syncthreads();
+            P.sa = psa2 + ((s - 1) & 1) * kChainGroup;
+            P.qs = pqs2 + ((s - 1) & 1) * kChainGroup;
         }
 
-        // ---- prologue 1: materialise slices; clear the sums of stage s + 1
-        materialise(h, kind, first_layer, final_phase, P, mg, m0);
+        // ---- materialise this CTA's slices of the previous stage's outputs
+        // and of the step values; clear its slice of stage s + 1's sums.
+        // Nothing in stage s reads them, except the down stage's input
+        // (`act`): every other stage does this after its units, off the
+        // critical path (measured on B200: about 2 us per stage before them).
+        auto materialise_and_clear = [&]() {
+            materialise(h, kind, first_layer, final_phase, P, mg, m0);
+            if (!final_phase && s + 1 < h->n_stages) {
+                const int64_t n = (int64_t)kChainGroup * stage_of(h, s + 1)->ntot;
+                const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
+                int32_t *b = sum_buf(s + 1);
+                for (int64_t e = lo + threadIdx.x; e < hi; e += kThreadsCh)
+                    b[e] = 0;
+            }
+        };
+        const bool late = !final_phase && kind != kStageDown;
+        if (!late)
+            materialise_and_clear();
         if (final_phase)
             break;
-        if (s + 1 < h->n_stages) {
-            const int64_t n = (int64_t)kChainGroup * stage_of(h, s + 1)->ntot;
-            const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
-            int32_t *b = sum_buf(s + 1);
-            for (int64_t e = lo + threadIdx.x; e < hi; e += kThreadsCh)
-                b[e] = 0;
+        // the down stage reads SiLU(g) * u back from `act`, whole, once
+        // every CTA has written its slice
+        int xkind = kind;
+        if (kind == kStageDown) {
+            if (!grid_barrier(ctr, nbar++, p, abort_flag)) {
+                ok = false;
+                break;
+            }
+            xkind = kStageDownAct;
         }
 
         // ---- prologue 2: this stage's input rows, quantised into shared memory
         const int64_t K = st->K, K4 = K / 4;
-        {
+        if (mg <= kRegTokens && K4 <= (int64_t)kXR * kThreadsCh) {
+            // per token: the thread's elements i = tid + j * kThreadsCh, all
+            // loaded at once and kept; amax over the row; 127/amax
+            float4 v[kRegTokens][kXR];
+            float am[kRegTokens];
+#pragma unroll
+            for (int m = 0; m < kRegTokens; ++m) {
+                am[m] = 0.f;
+                int4 ra[kXR], rb[kXR];
+#pragma unroll
+                for (int j = 0; j < kXR; ++j) {
+                    const int64_t i = threadIdx.x + (int64_t)j * kThreadsCh;
+                    ra[j] = make_int4(0, 0, 0, 0);
+                    rb[j] = make_int4(0, 0, 0, 0);
+                    if (m < mg && i < K4)
+                        stage_raw(h, xkind, first_layer, P, m, m0 + m, i, ra[j], rb[j]);
+                }
+#pragma unroll
+                for (int j = 0; j < kXR; ++j) {
+                    const int64_t i = threadIdx.x + (int64_t)j * kThreadsCh;
+                    v[m][j] = (m < mg && i < K4) ? stage_val(xkind, first_layer, P, m, ra[j], rb[j])
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < kRegTokens; ++m) {
+#pragma unroll
+                for (int j = 0; j < kXR; ++j)
+                    am[m] = fmaxf(am[m], fmaxf(fmaxf(fabsf(v[m][j].x), fabsf(v[m][j].y)),
+                                               fmaxf(fabsf(v[m][j].z), fabsf(v[m][j].w))));
+#pragma unroll
+                for (int o = 16; o; o >>= 1)
+                    am[m] = fmaxf(am[m], __shfl_xor_sync(0xffffffffu, am[m], o));
+                if (lane == 0 && m < mg)
+                    red_f[warp * kChainGroup + m] = am[m];
+            }
+            __syncthreads();
+            if (threadIdx.x < mg) {
+                float a = 0.f;
+                for (int w = 0; w < kNW; ++w)
+                    a = fmaxf(a, red_f[w * kChainGroup + threadIdx.x]);
+                sa_s[threadIdx.x] = __fdiv_rn(a, 127.f);
+                scale_s[threadIdx.x] = a == 0.f ? 0.f : __fdiv_rn(127.f, a);
+            }
+            __syncthreads();
+            // quantise the kept values into shared memory, with sum(q) per token
+#pragma unroll
+            for (int m = 0; m < kRegTokens; ++m) {
+                if (m >= mg)
+                    break;
+                const float sc = scale_s[m];
+                const bool zero = sc == 0.f;
+                uint32_t *row = reinterpret_cast<uint32_t *>(xbuf + m * p.xstride);
+                int sq = 0;
+#pragma unroll
+                for (int j = 0; j < kXR; ++j) {
+                    const int64_t i = threadIdx.x + (int64_t)j * kThreadsCh;
+                    if (i < K4)
+                        row[i] = quant4c(v[m][j], sc, zero, sq);
+                }
+#pragma unroll
+                for (int o = 16; o; o >>= 1)
+                    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                if (lane == 0)
+                    red_i[warp * kChainGroup + m] = sq;
+            }
+            __syncthreads();
+            if (threadIdx.x < mg) {
+                int q = 0;
+                for (int w = 0; w < kNW; ++w)
+                    q += red_i[w * kChainGroup + threadIdx.x];
+                qs_s[threadIdx.x] = q;
+            }
+            __syncthreads();
+            if (threadIdx.x < mg) {
+                psa2[(s & 1) * kChainGroup + threadIdx.x] = sa_s[threadIdx.x];
+                pqs2[(s & 1) * kChainGroup + threadIdx.x] = qs_s[threadIdx.x];
+            }
+        } else {
             // per token: amax over the row, then 127/amax (one token at a time
             // keeps a single running value per thread)
             for (int m = 0; m < mg; ++m) {
                 float a = 0.f;
                 for (int64_t i = threadIdx.x; i < K4; i += kThreadsCh) {
-                    const float4 v = stage_x4(h, kind, first_layer, P, m, m0 + m, i);
+                    const float4 v = stage_x4(h, xkind, first_layer, P, m, m0 + m, i);
                     a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
                 }
 #pragma unroll
@@ -449,7 +684,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
                 uint32_t *row = reinterpret_cast<uint32_t *>(xbuf + m * p.xstride);
                 int sq = 0;
                 for (int64_t i = threadIdx.x; i < K4; i += kThreadsCh)
-                    row[i] = quant4c(stage_x4(h, kind, first_layer, P, m, m0 + m, i), sc, zero, sq);
+                    row[i] = quant4c(stage_x4(h, xkind, first_layer, P, m, m0 + m, i), sc, zero, sq);
 #pragma unroll
                 for (int o = 16; o; o >>= 1)
                     sq += __shfl_xor_sync(0xffffffffu, sq, o);
@@ -466,8 +701,8 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
             __syncthreads();
             // this stage's scales serve the next prologue's rescale
             if (threadIdx.x < mg) {
-                psa_s[threadIdx.x] = sa_s[threadIdx.x];
-                pqs_s[threadIdx.x] = qs_s[threadIdx.x];
+                psa2[(s & 1) * kChainGroup + threadIdx.x] = sa_s[threadIdx.x];
+                pqs2[(s & 1) * kChainGroup + threadIdx.x] = qs_s[threadIdx.x];
             }
         }
 
@@ -521,6 +756,12 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
         }
         if (!ok)
             *abort_flag = 1;
+        else if (late)
+            materialise_and_clear();
+        // this stage's wscales for the next prologue's rescale (the load's
+        // latency hides in the barrier; the barrier orders the store)
+        if (threadIdx.x < st->nproj)
+            pws_s[threadIdx.x] = __ldg(st->proj[threadIdx.x].wscale);
         ok = grid_barrier(ctr, nbar++, p, abort_flag) && ok;
     }
 
@@ -549,7 +790,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
 int chain_fused_smem(int64_t max_K)
 {
     const int xstride = (int)(max_K + 64);
-    return kNW * kS * kSlotBytes + kChainGroup * xstride + 4 * 5 * kChainGroup + 32 +
+    return kNW * kS * kSlotBytes + kChainGroup * xstride + 4 * 7 * kChainGroup + 32 +
            8 * kNW * kChainGroup + 16 + 8 * kNW * kS + 64;
 }
 
@@ -557,7 +798,10 @@ cudaError_t launch_chain_fused(const ChainLaunch &L, uint32_t *err, uint64_t tim
                                cudaStream_t stream)
 {
     const ChainPlanHeader &hh = *L.host;
-    const int smem = chain_fused_smem(hh.max_K);
+    const int base = chain_fused_smem(hh.max_K);
+    const int cache_bytes = 64 + 64 * hh.n_stages;
+    const bool cache = base + cache_bytes <= 227 * 1024;
+    const int smem = base + (cache ? cache_bytes : 0);
     cudaError_t e = cudaFuncSetAttribute(k_chain, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return e;
@@ -566,6 +810,7 @@ cudaError_t launch_chain_fused(const ChainLaunch &L, uint32_t *err, uint64_t tim
     p.plan = L.plan;
     p.ws = L.ws;
     p.xstride = (int)(hh.max_K + 64);
+    p.unit_cache = cache ? 1 : 0;
     p.ctl.err = err;
     p.ctl.timeout_ns = timeout_ns;
     for (int64_t m0 = 0; m0 < hh.M; m0 += kChainGroup) {
