@@ -54,9 +54,10 @@ constexpr int kSlotBytes = kCT * kTileBytes;
 constexpr uint64_t kDrainNsCh = 1000000000ull;
 // A stage input row of up to kXR float4 per thread (K <= 10240) for up to
 // kRegTokens tokens stays in registers between the amax and the
-// quantisation passes; each pass then issues all its loads at once.
+// quantisation passes; each pass then issues all its loads at once.  (Two
+// tokens spill registers of the 512-thread CTA.)
 constexpr int kXR = 5;
-constexpr int kRegTokens = 2;
+constexpr int kRegTokens = 1;
 // The down projection's input as read back by the quantisation: SiLU(g) * u
 // is computed once, by the CTA whose slice of `act` holds it (materialise),
 // and after a grid-wide barrier read by every CTA (measured on B200: every
@@ -153,13 +154,17 @@ __device__ bool grid_barrier(uint32_t *ctr, uint32_t k, const ChainParams &p, vo
     return !*abort_flag;
 }
 
-// A warp's walk over its work units, stage after stage.
+// A warp's walk over its work units, stage after stage.  Its fields are
+// scalars, indexed by selection, so that it stays in registers (measured on
+// B200: with arrays indexed by the projection it lived in local memory,
+// which the large shared-memory carve-out leaves no L1 for, and each step
+// paid L2 round trips).
 struct UnitIter {
     int s, n_stages;
     int u, hi;                  // current unit, end of this CTA's range in stage s
     int nch, KT, nproj;
-    int rb_off[4];
-    const uint8_t *packed[3];
+    int rb1, rb2;               // first row block of projections 1 and 2 (the total past nproj)
+    const uint8_t *packed0, *packed1, *packed2;
     bool valid;
     const UnitS *cache;         // the stages' unit fields in shared memory, or null
 
@@ -174,10 +179,11 @@ struct UnitIter {
                 nch = f.nch;
                 KT = f.KT;
                 nproj = f.nproj;
-                for (int q = 0; q < 4; ++q)
-                    rb_off[q] = f.rb_off[q];
-                for (int q = 0; q < 3; ++q)
-                    packed[q] = f.packed[q];
+                rb1 = f.rb_off[1];
+                rb2 = f.rb_off[2];
+                packed0 = f.packed[0];
+                packed1 = f.packed[1];
+                packed2 = f.packed[2];
                 valid = true;
                 return;
             }
@@ -193,8 +199,8 @@ struct UnitIter {
     __device__ void where(int &q, int &rbl, int &kt0, int &n) const
     {
         const int rbg = u / nch, kc = u - rbg * nch;
-        q = rbg >= rb_off[1] ? (rbg >= rb_off[2] ? 2 : 1) : 0;
-        rbl = rbg - rb_off[q];
+        q = rbg >= rb1 ? (rbg >= rb2 ? 2 : 1) : 0;
+        rbl = rbg - (q == 0 ? 0 : q == 1 ? rb1 : rb2);
         kt0 = kc * kCT;
         n = min(kCT, KT - kt0);
     }
@@ -202,7 +208,8 @@ struct UnitIter {
     {
         int q, rbl, kt0, n;
         where(q, rbl, kt0, n);
-        const uint8_t *src = packed[q] + ((int64_t)rbl * KT + kt0) * (int64_t)kTileBytes;
+        const uint8_t *src = (q == 0 ? packed0 : q == 1 ? packed1 : packed2) +
+                             ((int64_t)rbl * KT + kt0) * (int64_t)kTileBytes;
         mbar_arrive_expect_tx(bar, (uint32_t)(n * kTileBytes));
         bulk_g2s(dst, src, (uint32_t)(n * kTileBytes), bar);
     }
