@@ -350,7 +350,7 @@ TW_API int tw_chain_plan_encode(const tw_chain_layer *layers, int n_layers,
                                 const tw_chain_buffers *buf, void *plan, size_t plan_bytes);
 
 /* HOST-ONLY.  Scratch of tw_decoder_chain_fused for a host plan: 256 bytes
- * of barrier counters, then three int32 sum buffers of 8 rows of the widest
+ * of barrier counters, then four int32 sum buffers of 8 rows of the widest
  * stage's outputs.  It must be zero-filled before its first use; every call
  * leaves the counters zero again (after TW_ERR_TIMEOUT, zero it again). */
 TW_API size_t tw_chain_fused_workspace_bytes(const void *plan_host);

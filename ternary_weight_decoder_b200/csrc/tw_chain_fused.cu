@@ -29,9 +29,12 @@
 // for the stage's MMAs.  Each CTA computes the whole input rows (they are a
 // few KB at decode sizes) but writes only its slice of the materialised
 // buffers (q, k, v, a, o, h1, g, u, act, d, h and any acc_out).  The sums
-// live in three rotating buffers: stage s adds into buffer s mod 3, the
-// prologue of s + 1 reads it, and the prologue of s - 1 cleared the buffer
-// of s + 1 -- so every buffer is zero before the first atomic reaches it.
+// live in kChainSumBufs = 4 rotating buffers: stage s adds into buffer
+// s mod 4; stage s + 1 reads it (its prologue, and its materialisation,
+// which runs after its units, between its arrival at the barrier and its
+// wait); stage s clears the buffer of s + 1 before it arrives at its
+// barrier -- so every buffer is zero before the first atomic reaches it,
+// and none is cleared while a CTA still materialises from it.
 //
 // Every value is computed with the same fp32 operations as the unfused
 // chain (the same rounding), so the two give the same bytes.  Every wait is
@@ -131,12 +134,19 @@ __device__ __forceinline__ void red_release_add_u32(uint32_t *p, uint32_t v)
 // polls the count with acquire loads until all k * gridDim.x arrivals are in.
 // The release and acquire replace two full fences per CTA.  False when the
 // wait timed out (the block must stop).
-__device__ bool grid_barrier(uint32_t *ctr, uint32_t k, const ChainParams &p, volatile int *abort_flag)
+// The barrier in two halves: the arrival, then -- after work that needs no
+// other CTA's -- the wait.
+__device__ __forceinline__ void grid_arrive(uint32_t *ctr)
 {
     __syncthreads();
+    if (threadIdx.x == 0)
+        red_release_add_u32(ctr, 1u);
+}
+
+__device__ bool grid_wait(uint32_t *ctr, uint32_t k, const ChainParams &p, volatile int *abort_flag)
+{
     if (threadIdx.x == 0) {
         const uint32_t target = k * gridDim.x;
-        red_release_add_u32(ctr, 1u);
         if (!*abort_flag && ld_acquire_u32(ctr) < target) {
             const uint64_t t0 = globaltimer_ns();
             while (ld_acquire_u32(ctr) < target) {
@@ -152,6 +162,13 @@ __device__ bool grid_barrier(uint32_t *ctr, uint32_t k, const ChainParams &p, vo
     }
     __syncthreads();
     return !*abort_flag;
+}
+
+__device__ __forceinline__ bool grid_barrier(uint32_t *ctr, uint32_t k, const ChainParams &p,
+                                             volatile int *abort_flag)
+{
+    grid_arrive(ctr);
+    return grid_wait(ctr, k, p, abort_flag);
 }
 
 // A warp's walk over its work units, stage after stage.  Its fields are
@@ -463,7 +480,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
     // are materialised after the next stage's prologue has written its own)
     float *psa2 = scale_s + kChainGroup;                                       // [2][8]
     int *pqs2 = reinterpret_cast<int *>(psa2 + 2 * kChainGroup);               // [2][8]
-    float *pws_s = reinterpret_cast<float *>(pqs2 + 2 * kChainGroup);          // [4] wscales
+    float *pws_s = reinterpret_cast<float *>(pqs2 + 2 * kChainGroup);          // [2][4] wscales
     float *red_f = pws_s + 4 + 4;                                              // [kNW][8]
     int *red_i = reinterpret_cast<int *>(red_f + kNW * kChainGroup);           // [kNW][8]
     uint64_t *bars = reinterpret_cast<uint64_t *>(
@@ -480,7 +497,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
     uint32_t *ctr = reinterpret_cast<uint32_t *>(p.ws);
     const int64_t buf_ints = (kChainGroup * h->max_ntot * 4 + 255) / 256 * 64;
     int32_t *sums = reinterpret_cast<int32_t *>(p.ws + 256);
-    auto sum_buf = [&](int s) { return sums + (int64_t)(s % 3) * buf_ints; };
+    auto sum_buf = [&](int s) { return sums + (int64_t)(s % kChainSumBufs) * buf_ints; };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNW * kS; ++i)
@@ -547,6 +564,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
             P.ntot = P.st->ntot;
             P.sa = psa2 + ((s - 1) & 1) * kChainGroup;
             P.qs = pqs2 + ((s - 1) & 1) * kChainGroup;
+            P.ws = pws_s + ((s - 1) & 1) * 4;
         }
 
         // ---- materialise this CTA's slices of the previous stage's outputs
@@ -554,8 +572,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
         // Nothing in stage s reads them, except the down stage's input
         // (`act`): every other stage does this after its units, off the
         // critical path (measured on B200: about 2 us per stage before them).
-        auto materialise_and_clear = [&]() {
-            materialise(h, kind, first_layer, final_phase, P, mg, m0);
+        auto clear_next = [&]() {
             if (!final_phase && s + 1 < h->n_stages) {
                 const int64_t n = (int64_t)kChainGroup * stage_of(h, s + 1)->ntot;
                 const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
@@ -565,8 +582,10 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
             }
         };
         const bool late = !final_phase && kind != kStageDown;
-        if (!late)
-            materialise_and_clear();
+        if (!late) {
+            materialise(h, kind, first_layer, final_phase, P, mg, m0);
+            clear_next();
+        }
         if (final_phase)
             break;
         // the down stage reads SiLU(g) * u back from `act`, whole, once
@@ -764,12 +783,15 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
         if (!ok)
             *abort_flag = 1;
         else if (late)
-            materialise_and_clear();
-        // this stage's wscales for the next prologue's rescale (the load's
-        // latency hides in the barrier; the barrier orders the store)
+            clear_next();
+        grid_arrive(ctr);
+        if (ok && late)   // off the critical path: while the other CTAs finish
+            materialise(h, kind, first_layer, final_phase, P, mg, m0);
+        // this stage's wscales for the next stage (the load's latency hides
+        // in the barrier; the barrier orders the store)
         if (threadIdx.x < st->nproj)
-            pws_s[threadIdx.x] = __ldg(st->proj[threadIdx.x].wscale);
-        ok = grid_barrier(ctr, nbar++, p, abort_flag) && ok;
+            pws_s[(s & 1) * 4 + threadIdx.x] = __ldg(st->proj[threadIdx.x].wscale);
+        ok = grid_wait(ctr, nbar++, p, abort_flag) && ok;
     }
 
     if (!ok) {

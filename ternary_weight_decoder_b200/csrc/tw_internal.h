@@ -63,6 +63,7 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 constexpr uint32_t kChainPlanMagic = 0x54574332u;  // "TWC2"
 constexpr int kChainGroup = 8;                     // tokens per fused launch
 constexpr int kChainChunk = 6;                     // code tiles per work unit
+constexpr int kChainSumBufs = 4;                   // rotating partial-sum buffers
 enum ChainKind : int32_t { kStageQKV = 0, kStageO = 1, kStageGU = 2, kStageDown = 3 };
 
 struct alignas(64) ChainProj {
@@ -100,10 +101,10 @@ struct ChainLaunch {
     uint8_t *ws;
 };
 // Scratch of the fused chain: 256 bytes of counters (zero between calls),
-// then three int32 sum buffers of kChainGroup x max_ntot.
+// then kChainSumBufs int32 sum buffers of kChainGroup x max_ntot.
 inline int64_t chain_fused_ws_bytes(const ChainPlanHeader &h)
 {
-    return 256 + 3 * ((kChainGroup * h.max_ntot * 4 + 255) / 256 * 256);
+    return 256 + kChainSumBufs * ((kChainGroup * h.max_ntot * 4 + 255) / 256 * 256);
 }
 cudaError_t launch_chain_fused(const ChainLaunch &L, uint32_t *err, uint64_t timeout_ns,
                                cudaStream_t stream);

@@ -349,7 +349,7 @@ def test_chain_fused_plan_host_checks(lib):
             api.tw_last_error()
         assert api.tw_chain_fused_launches(plan.ctypes.data) == launches
         # counters + three sum buffers of 8 rows of the widest stage (gate/up: 2 x 512)
-        assert api.tw_chain_fused_workspace_bytes(plan.ctypes.data) == 256 + 3 * 8 * 1024 * 4
+        assert api.tw_chain_fused_workspace_bytes(plan.ctypes.data) == 256 + 4 * 8 * 1024 * 4
         assert api.tw_chain_plan_encode(layers, 2, ctypes.byref(cbuf), plan.ctypes.data, nb - 1) == 4
     # a table that does not match the buffers is refused here too
     layers, cbuf, keep = _fake_chain(tweak=lambda l, st, a: st == "o" and _tw(a, 0, x=a[0].x + 0x100000))
