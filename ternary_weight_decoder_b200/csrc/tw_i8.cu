@@ -208,22 +208,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_i8_gemm(const __grid_constant__
         const float sw = __fdiv_rn(__ldg(p.amax_w), 127.f);
         int64_t tt = 0;
         int nbox = 0;                           // boxes this warp has staged
+        // The per-token scale and this half's bias columns of a tile are
+        // loaded one tile ahead, so that their L2 round trip overlaps the
+        // previous tile's epilogue instead of preceding this one's.
+        float amax_n = 0.f, bias_n0 = 0.f, bias_n1 = 0.f;
+        auto load_scales = [&](int64_t t) {
+            if (t >= p.tiles)
+                return;
+            int64_t mi, nj;
+            tile_coords(p, t, mi, nj);
+            const int64_t m = mi * kBM + 32 * quarter + lane;
+            const int64_t n = nj * kBN + 64 * half + lane;
+            amax_n = m < p.M ? __ldg(p.amax_x + m) : 0.f;
+            bias_n0 = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.f;
+            bias_n1 = (p.bias && n + 32 < p.N) ? __ldg(p.bias + n + 32) : 0.f;
+        };
+        load_scales(blockIdx.x);
         for (int64_t t = blockIdx.x; t < p.tiles; t += G, ++tt) {
             int64_t mi, nj;
             tile_coords(p, t, mi, nj);
             const int ab = (int)(tt & 1);
             const int64_t m0 = mi * kBM + 32 * quarter;   // first token row of this warp
             const int64_t m = m0 + lane;
-            const float sa = m < p.M ? __fdiv_rn(__ldg(p.amax_x + m), 127.f) : 0.f;
+            const float sa = m < p.M ? __fdiv_rn(amax_n, 127.f) : 0.f;
             // this half's bias columns into the warp's own shared buffer
-            // (before the wait; the warp's previous tile is done with it)
+            // (the warp's previous tile is done with it)
             float *bias_t = bias_s + 64 * ew;
-            {
-                const int64_t n = nj * kBN + 64 * half + lane;
-                bias_t[lane] = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.f;
-                bias_t[lane + 32] = (p.bias && n + 32 < p.N) ? __ldg(p.bias + n + 32) : 0.f;
-            }
+            bias_t[lane] = bias_n0;
+            bias_t[lane + 32] = bias_n1;
             __syncwarp();
+            load_scales(t + G);
             if (!mbar_wait(b_tfull + 8 * ab, (uint32_t)((tt / 2) & 1), p.ctl, abort_flag))
                 break;
             tc_fence_after();
