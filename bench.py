@@ -617,6 +617,25 @@ def cpu_oracle_sample(M, budget_s=10.0, sample_layers=4, layers=28):
                           sample_layers=sample_layers)
 
 
+def headline_config(M, layers, world):
+    """The `config` of the headline line, the same for both arms."""
+    shapes = [(N, K) for (_, _, _, N, K) in _sweep_shapes(layers)]
+    algo = sum(N * K // 4 + M * K * 4 + M * N * 4 for (N, K) in shapes)
+    if M <= 32:
+        workload = (f"decode_sweep_196x_M{M}" if layers == 28
+                    else f"decode_sweep_{7 * layers}x_M{M}")
+    else:
+        workload = f"prefill_sweep_{7 * layers}x_M{M}"
+    return {"workload": workload, "M": M, "projections": len(shapes), "layers": layers,
+            "parallelism": f"dp{world} (independent replicas, no collective)",
+            "l2": f"inputs {algo / 1e6:.0f} MB > 126 MB L2; no flush"}
+
+
+def _sweep_shapes(layers):
+    from ternary_weight_decoder_b200 import synth
+    return synth.sweep_shapes(layers)
+
+
 def run_reference(args):
     """The oracle as it stands, on host cores, on the same metric and config."""
     rank = int(os.environ.get("RANK", "0"))
@@ -661,8 +680,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
-        "config": {"workload": f"decode_sweep_196x_M{M}", "M": M,
-                   "projections": len(shapes)},
+        "config": headline_config(M, args.layers, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": samp, **cpu_info()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -1044,12 +1062,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
-        "config": {"workload": (f"decode_sweep_196x_M{M}" if args.layers == 28
-                                else f"decode_sweep_{7 * args.layers}x_M{M}") if M <= 32
-                   else f"prefill_sweep_{7 * args.layers}x_M{M}",
-                   "M": M, "projections": len(shapes), "layers": args.layers,
-                   "parallelism": f"dp{world} (independent replicas, no collective)",
-                   "l2": f"inputs {algo_bytes / 1e6:.0f} MB > 126 MB L2; no flush"},
+        "config": headline_config(M, args.layers, world),
         "roofline": roofline, "step_times": dist_summary(per), "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
