@@ -510,6 +510,10 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
     Plan *plan = reinterpret_cast<Plan *>(misc + 256 * kXE + 8 * (NC * p.slots + 2 * kXE));
     volatile int *xoff = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(plan) + 64);
     ProjC *pcache = reinterpret_cast<ProjC *>(reinterpret_cast<uint8_t *>(plan) + 128);
+    // the activation ring's entry starts (in shared memory: a local array
+    // indexed by entry lands in local memory, which the shared-memory
+    // carve-out leaves no L1 for)
+    int64_t *xstart = reinterpret_cast<int64_t *>(pcache + kPC);
     const uint32_t bar_ring = smem_u32(bars);
     const uint32_t bar_xfull = bar_ring + 8 * NC * p.slots;
     const uint32_t bar_xempty = bar_xfull + 8 * kXE;
@@ -551,7 +555,8 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
             // Positions are counted monotonically; entry seg lives at
             // start[seg % kXE] mod xcap.  `tail` is the oldest entry not yet
             // known to be free.
-            int64_t head = 0, start[kXE];
+            int64_t head = 0;
+            int64_t *start = xstart;
             int tail = 0;
             bool ok = true;
             for (int d = pl.d_lo; d <= pl.d_hi && ok; ++d) {

@@ -330,12 +330,16 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
                 }
                 if (32 * c >= nvalid)
                     continue;   // (uniform across the warp)
+                // (selected, not indexed: the arrays stay in registers)
+                static_assert(kNTok / 32 == 4, "token groups");
+                const float sa_c = c == 0 ? sa_l[0] : c == 1 ? sa_l[1] : c == 2 ? sa_l[2] : sa_l[3];
+                const int qs_c = c == 0 ? qs_l[0] : c == 1 ? qs_l[1] : c == 2 ? qs_l[2] : qs_l[3];
                 for (int pass = 0; pass < (pr.acc_out ? 2 : 1); ++pass) {
                     // box[n][lane] = token 32c + n of this lane's row
 #pragma unroll
                     for (int n = 0; n < 32; ++n) {
-                        const float sa = __shfl_sync(0xffffffffu, sa_l[c], n);
-                        const int qs = __shfl_sync(0xffffffffu, qs_l[c], n);
+                        const float sa = __shfl_sync(0xffffffffu, sa_c, n);
+                        const int qs = __shfl_sync(0xffffffffu, qs_c, n);
                         const int a = (int)v[n] - qs;
                         box[n * 32 + lane] = pass == 0 ? __fmul_rn(__fmul_rn((float)a, sa), pr.wscale)
                                                        : __int_as_float(a);
