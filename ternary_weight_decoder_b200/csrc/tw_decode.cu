@@ -557,7 +557,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
             // known to be free.
             int64_t head = 0;
             int64_t *start = xstart;
-            int tail = 0;
+            int tail = 0, nissued = 0;
             bool ok = true;
             for (int d = pl.d_lo; d <= pl.d_hi && ok; ++d) {
                 const int seg = d - pl.d_lo, e = seg % kXE;
@@ -588,12 +588,13 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) k_decode(const __grid_consta
                     bulk_g2s(dst + tok * (uint32_t)rs, p.ws + r.ws_xq_off + (int64_t)(p.m0 + tok) * r.K,
                              (uint32_t)r.K, bx);
                 bulk_g2s(smem_u32(info + 256 * e), p.ws + p.ws_sa_off + 256 * (int64_t)d, 256, bx);
+                ++nissued;
             }
-            // Drain: the activation copies of the last entries land before exit.
+            // Drain: the activation copies of the last entries issued land
+            // before exit.
             WaitCtl drain = p.ctl;
             drain.timeout_ns = kDrainNs;
-            const int nseg = pl.d_hi - pl.d_lo + 1;
-            for (int seg = nseg - kXE; seg < nseg; ++seg)
+            for (int seg = nissued - kXE; seg < nissued; ++seg)
                 if (seg >= 0)
                     mbar_wait(bar_xfull + 8 * (seg % kXE), (seg / kXE) & 1, drain, nullptr);
         }
