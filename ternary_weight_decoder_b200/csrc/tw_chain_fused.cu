@@ -463,6 +463,14 @@ __device__ void materialise(const ChainPlanHeader *h, int kind, bool first_layer
     }
 }
 
+// Copy one stage plan (256 bytes) into shared memory: threads 0 .. 15.
+__device__ __forceinline__ void copy_stage(ChainStagePlan *dst, const ChainStagePlan *src)
+{
+    static_assert(sizeof(ChainStagePlan) == 16 * 16, "stage plan copy");
+    if (threadIdx.x < 16)
+        reinterpret_cast<int4 *>(dst)[threadIdx.x] = reinterpret_cast<const int4 *>(src)[threadIdx.x];
+}
+
 __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__ ChainParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -488,11 +496,22 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
     int *abort_p = reinterpret_cast<int *>(bars + kNW * kS);
     volatile int *abort_flag = abort_p;
     const uint32_t bar_ring = smem_u32(bars);
-    UnitS *ucache = reinterpret_cast<UnitS *>(
+    // The plan header and a ring of four stage plans (stages s - 1 .. s + 2
+    // at stage s), so that the stage loop reads no plan field from global
+    // memory (measured on B200: each such read an L2 round trip on the
+    // path of the prologue and of the materialisation).
+    ChainStagePlan *sring = reinterpret_cast<ChainStagePlan *>(
         (reinterpret_cast<uintptr_t>(abort_p + 1) + 63) & ~uintptr_t(63));
+    ChainPlanHeader *hs = reinterpret_cast<ChainPlanHeader *>(sring + 4);
+    UnitS *ucache = reinterpret_cast<UnitS *>(
+        (reinterpret_cast<uintptr_t>(hs + 1) + 63) & ~uintptr_t(63));
     if (p.unit_cache)
         for (int i = threadIdx.x; i < h->n_stages; i += kThreadsCh)
             ucache[i] = unit_fields(stage_of(h, i));
+    for (int i = threadIdx.x; i < (int)(sizeof(ChainPlanHeader) / 16); i += kThreadsCh)
+        reinterpret_cast<int4 *>(hs)[i] = reinterpret_cast<const int4 *>(h)[i];
+    for (int i = 0; i < 2 && i < h->n_stages; ++i)
+        copy_stage(sring + i, stage_of(h, i));
 
     uint32_t *ctr = reinterpret_cast<uint32_t *>(p.ws);
     const int64_t buf_ints = (kChainGroup * h->max_ntot * 4 + 255) / 256 * 64;
@@ -547,19 +566,24 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
     P.qs = pqs2;
     P.ws = pws_s;
 
-    for (int s = 0; s <= h->n_stages && ok; ++s) {
-        const bool final_phase = s == h->n_stages;
-        const ChainStagePlan *st = final_phase ? nullptr : stage_of(h, s);
+    const int n_stages = h->n_stages;
+    for (int s = 0; s <= n_stages && ok; ++s) {
+        const bool final_phase = s == n_stages;
+        const ChainStagePlan *st = final_phase ? nullptr : sring + (s & 3);
+        // (stage s - 2's slot: its last reader, stage s - 1's
+        // materialisation, is behind the barrier)
+        if (s + 2 < n_stages)
+            copy_stage(sring + ((s + 2) & 3), stage_of(h, s + 2));
         const int kind = final_phase ? -1 : st->kind;
         const bool first_layer = s < 4;
         // The plan entries of the next stages, into this SM's L1 (the units
         // of stage s walk into stage s + 1's, the ring's producer further).
-        if (threadIdx.x < 8 && s + 1 + (threadIdx.x >> 1) < h->n_stages)
+        if (threadIdx.x < 8 && s + 1 + (threadIdx.x >> 1) < n_stages)
             asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const uint8_t *>(
                              stage_of(h, s + 1 + (threadIdx.x >> 1))) + 128 * (threadIdx.x & 1)));
         if (s > 0) {
             // (pws_s holds stage s - 1's wscales, loaded before the barrier)
-            P.st = stage_of(h, s - 1);
+            P.st = sring + ((s - 1) & 3);
             P.sum = sum_buf(s - 1);
             P.ntot = P.st->ntot;
             P.sa = psa2 + ((s - 1) & 1) * kChainGroup;
@@ -573,8 +597,8 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
         // (`act`): every other stage does this after its units, off the
         // critical path (measured on B200: about 2 us per stage before them).
         auto clear_next = [&]() {
-            if (!final_phase && s + 1 < h->n_stages) {
-                const int64_t n = (int64_t)kChainGroup * stage_of(h, s + 1)->ntot;
+            if (!final_phase && s + 1 < n_stages) {
+                const int64_t n = (int64_t)kChainGroup * sring[(s + 1) & 3].ntot;
                 const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
                 int32_t *b = sum_buf(s + 1);
                 for (int64_t e = lo + threadIdx.x; e < hi; e += kThreadsCh)
@@ -583,7 +607,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
         };
         const bool late = !final_phase && kind != kStageDown;
         if (!late) {
-            materialise(h, kind, first_layer, final_phase, P, mg, m0);
+            materialise(hs, kind, first_layer, final_phase, P, mg, m0);
             clear_next();
         }
         if (final_phase)
@@ -616,7 +640,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
                     ra[j] = make_int4(0, 0, 0, 0);
                     rb[j] = make_int4(0, 0, 0, 0);
                     if (m < mg && i < K4)
-                        stage_raw(h, xkind, first_layer, P, m, m0 + m, i, ra[j], rb[j]);
+                        stage_raw(hs, xkind, first_layer, P, m, m0 + m, i, ra[j], rb[j]);
                 }
 #pragma unroll
                 for (int j = 0; j < kXR; ++j) {
@@ -685,7 +709,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
             for (int m = 0; m < mg; ++m) {
                 float a = 0.f;
                 for (int64_t i = threadIdx.x; i < K4; i += kThreadsCh) {
-                    const float4 v = stage_x4(h, xkind, first_layer, P, m, m0 + m, i);
+                    const float4 v = stage_x4(hs, xkind, first_layer, P, m, m0 + m, i);
                     a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
                 }
 #pragma unroll
@@ -710,7 +734,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
                 uint32_t *row = reinterpret_cast<uint32_t *>(xbuf + m * p.xstride);
                 int sq = 0;
                 for (int64_t i = threadIdx.x; i < K4; i += kThreadsCh)
-                    row[i] = quant4c(stage_x4(h, xkind, first_layer, P, m, m0 + m, i), sc, zero, sq);
+                    row[i] = quant4c(stage_x4(hs, xkind, first_layer, P, m, m0 + m, i), sc, zero, sq);
 #pragma unroll
                 for (int o = 16; o; o >>= 1)
                     sq += __shfl_xor_sync(0xffffffffu, sq, o);
@@ -786,7 +810,7 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
             clear_next();
         grid_arrive(ctr);
         if (ok && late)   // off the critical path: while the other CTAs finish
-            materialise(h, kind, first_layer, final_phase, P, mg, m0);
+            materialise(hs, kind, first_layer, final_phase, P, mg, m0);
         // this stage's wscales for the next stage (the load's latency hides
         // in the barrier; the barrier orders the store)
         if (threadIdx.x < st->nproj)
@@ -820,7 +844,8 @@ int chain_fused_smem(int64_t max_K)
 {
     const int xstride = (int)(max_K + 64);
     return kNW * kS * kSlotBytes + kChainGroup * xstride + 4 * 7 * kChainGroup + 32 +
-           8 * kNW * kChainGroup + 16 + 8 * kNW * kS + 64;
+           8 * kNW * kChainGroup + 16 + 8 * kNW * kS + 64 + 4 * (int)sizeof(ChainStagePlan) +
+           (int)sizeof(ChainPlanHeader) + 64;
 }
 
 cudaError_t launch_chain_fused(const ChainLaunch &L, uint32_t *err, uint64_t timeout_ns,
