@@ -285,8 +285,8 @@ __device__ __forceinline__ float4 stage_x4(const ChainPlanHeader *h, int kind, b
         return add4(ldcg4f(h->h1 + mrow * h->hidden + k), prev_y4(P, 0, m, k));
     case kStageO: {
         // a = v, each KV head repeated for the query heads of its group
-        const int64_t group = (h->hidden / h->head_dim) / (h->kv_dim / h->head_dim);
-        const int64_t head = k / h->head_dim, c = k - head * h->head_dim;
+        const int hd = (int)h->head_dim, group = (int)(h->hidden / h->kv_dim);
+        const int head = (int)k / hd, c = (int)k - head * hd;
         return prev_y4(P, 2, m, (head / group) * h->head_dim + c);
     }
     case kStageGU:
@@ -321,8 +321,8 @@ __device__ __forceinline__ void stage_raw(const ChainPlanHeader *h, int kind, bo
         }
         break;
     case kStageO: {
-        const int64_t group = (h->hidden / h->head_dim) / (h->kv_dim / h->head_dim);
-        const int64_t head = k / h->head_dim, c = k - head * h->head_dim;
+        const int hd = (int)h->head_dim, group = (int)(h->hidden / h->kv_dim);
+        const int head = (int)k / hd, c = (int)k - head * hd;
         b = ldcg4i(P.sum + (int64_t)m * P.ntot + P.st->proj[2].noff + (head / group) * h->head_dim + c);
         break;
     }
