@@ -14,13 +14,14 @@
 // Work unit: one 128-row tile of one projection (8 row blocks of the packed
 // layout) over all of K.  Units are claimed from a counter in the scratch,
 // projections of larger K first, so that the units left at the end of the
-// sweep are the small ones.  A stage is a group of four 128-column k tiles
-// (one barrier wait and one commit of the MMA thread per 16 MMAs: measured
-// on B200, the per-stage waits and commits of that single thread, not the
-// MMAs, set the pace with one k tile per stage):
-//   * warp 0 (producer) loads the 8 row blocks x 4 k tiles of codes (16 KB)
-//     with one 3-D TMA and the 4 token blocks (N rows x 128 B each) with one
-//     bulk copy into a ring of L shared-memory stages (as many as fit);
+// sweep are the small ones.  A stage is a group of kGrp (six) 128-column k
+// tiles (one barrier wait and one commit of the MMA thread per 4 kGrp MMAs:
+// measured on B200, the per-stage waits and commits of that single thread,
+// not the MMAs, set the pace with one k tile per stage):
+//   * warp 0 (producer) loads the 8 row blocks x kGrp k tiles of codes (24 KB)
+//     with one 3-D TMA and the kGrp token blocks (N rows x 128 B each) with
+//     one bulk copy into a ring of L shared-memory stages (an even number, as
+//     many as fit);
 //     k tiles past K read as zero codes, which expand to zero weights;
 //   * eight expansion warps (two per TMEM lane quarter, alternating stages)
 //     turn each 16-byte lane slot of the code tile into 16 registers -- the
@@ -28,7 +29,7 @@
 //     consecutive k -- and store them to the stage's A slot in tensor memory
 //     (tcgen05.st 16x256b): column 8s + 2t + h of lane (row) g or g + 8
 //     holds slot s of the word with k = 64h + 16t + 4s .. + 3.  A stage
-//     fills one of kASlots A slots of 4 x 32 columns;
+//     fills one of kASlots A slots of kGrp x 32 columns;
 //   * warp 1 waits only for the expansion of the stage (which itself waited
 //     for the stage's bytes), issues four MMAs of K = 32 per k tile, one per
 //     slot s (columns 8s .. 8s+7), and commits them to the stage's empty
@@ -62,20 +63,21 @@ constexpr int kGrp = kTcGroup;                  // k tiles per stage
 constexpr int kRingTc = 8;                      // unit-info entries
 constexpr int kMaxStagesTc = 8;                 // shared-memory load stages, at most
 constexpr int kThreadsTc = 14 * 32;
-constexpr int kCodeStageBytes = 8 * kGrp * kTileBytes;  // 128 rows x 4 x 128 k = 16 KB
+constexpr int kCodeStageBytes = 8 * kGrp * kTileBytes;  // 128 rows x kGrp x 128 k
 constexpr int kTmemColsTc = 512;
 
 // Tensor-memory plan per token-block width.  32 tokens: one accumulator per
-// buffer (every slot's codes expanded unscaled, c + 1 in {0, 1, 2}) and
-// three A slots, so that the expansion stays further ahead and the epilogue
-// reads one accumulator; 8 or 16 tokens: one accumulator per 2-bit slot
-// (expanded with one AND, scaled by 4^s) and two A slots.  Measured on B200
-// over the 196 projections: 138.3 against 144.4 us at 32 tokens, 117.8
-// against 119.8 us at 16 for the four-accumulator plan.
+// buffer (every slot's codes expanded unscaled, c + 1 in {0, 1, 2}), so that
+// the epilogue reads one accumulator, and three A slots where they fit
+// beside it (with four k tiles per stage), so that the expansion stays
+// further ahead; 8 or 16 tokens: one accumulator per 2-bit slot (expanded
+// with one AND, scaled by 4^s) and two A slots.  Measured on B200 over the
+// 196 projections with four k tiles per stage: 138.3 against 144.4 us at 32
+// tokens, 117.8 against 119.8 us at 16 for the four-accumulator plan.
 template <int NTOK>
 struct AccPlan {
     static constexpr bool kOneD = NTOK == 32;
-    static constexpr int kASlots = kOneD ? 3 : 2;           // A slots of kGrp x 32 columns
+    static constexpr int kASlots = kOneD && 96 * kGrp + 2 * NTOK <= 512 ? 3 : 2;  // A slots of kGrp x 32 columns
     static constexpr int kDCol0 = 32 * kGrp * kASlots;      // the two accumulator buffers
     static constexpr int kDCols = kOneD ? NTOK : 4 * NTOK;  // columns of one buffer
     static_assert(kDCol0 + 2 * kDCols <= 512, "tensor memory");

@@ -249,9 +249,19 @@ int encode_codes_tmap(const uint8_t *packed, int64_t N, int64_t K, int box_rb, i
                       void *out128);
 // k tiles per pipeline stage of the tensor-core decode (tw_decode_tc.cu) and
 // of the weights-in-TMEM GEMM (tw_mid.cu): one barrier wait and one commit
-// of the MMA thread cover that many k tiles.
-constexpr int kTcGroup = 4;
-constexpr int kMidGroup = 2;
+// of the MMA thread cover that many k tiles.  Measured on B200 over the
+// 196 projections: six tiles (K = 1536 is two stages) against four, the
+// tensor-core decode at 9 / 16 / 24 / 32 tokens 113.3 / 117.8 / 129.6 /
+// 136.3 -> 105.9 / 111.7 / 126.7 / 134.3 us; for the weights-in-TMEM GEMM
+// three or four tiles were slower than two (fewer load stages fit).
+#ifndef TW_TC_GROUP
+#define TW_TC_GROUP 6
+#endif
+constexpr int kTcGroup = TW_TC_GROUP;
+#ifndef TW_MID_GROUP
+#define TW_MID_GROUP 2
+#endif
+constexpr int kMidGroup = TW_MID_GROUP;
 
 cudaError_t launch_wait_probe(uint32_t *err, uint64_t timeout_ns, cudaStream_t stream);
 

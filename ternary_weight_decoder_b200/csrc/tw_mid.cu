@@ -119,7 +119,7 @@ __device__ UnitM locate_unit_m(const MidParams &p, const UnitOrder *order, int64
 template <int L>
 __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ MidParams p)
 {
-    static_assert(L >= 2, "load stages");
+    static_assert(L >= 2 && L >= kASlotsM, "load stages");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -384,14 +384,21 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
         const int sh0 = 4 * (t & 1);   // 2 s for i & 1 == 0
         for (uint32_t it = set;; it += 2) {
             const int s = (int)(it % L);
-            if (!mbar_wait(b_full + 8 * s, (it / L) & 1u, p.ctl, abort_flag))
-                break;
-            if (stage_stop[s])
-                break;
-            // A slot it % 4 is free once the MMAs of stage it - 4 have completed.
+            // A slot it % kASlotsM is free once the MMAs of stage it - kASlotsM
+            // have completed.  That wait comes first: those MMAs follow stage
+            // it - L's (kASlotsM <= L), so stage it - L's phase of the load
+            // barrier is complete before this set tests it for stage it.  The
+            // two sets take alternate stages, and with L odd the previous user
+            // of load stage s is the other set: tested first, the barrier
+            // could still be in stage it - L's phase, and the parity test
+            // would pass at once.
             if (it >= (uint32_t)kASlotsM &&
                 !mbar_wait(b_empty + 8 * (int)((it - kASlotsM) % L), ((it - kASlotsM) / L) & 1u, p.ctl,
                            abort_flag))
+                break;
+            if (!mbar_wait(b_full + 8 * s, (it / L) & 1u, p.ctl, abort_flag))
+                break;
+            if (stage_stop[s])
                 break;
             const uint32_t aslot = it % kASlotsM;
             tc_fence_after();
@@ -483,6 +490,13 @@ cudaError_t launch_mid(const MidLaunch &L, uint32_t *err, uint64_t timeout_ns, c
         return launch_mid_l<5>(p, grid, stream);
     if (smem_mid<4>(p.count) <= kLimit)
         return launch_mid_l<4>(p, grid, stream);
+    // (fewer stages only where every A slot has a load stage of its own)
+    if constexpr (kASlotsM <= 3)
+        if (smem_mid<3>(p.count) <= kLimit)
+            return launch_mid_l<3>(p, grid, stream);
+    if constexpr (kASlotsM <= 2)
+        if (smem_mid<2>(p.count) <= kLimit)
+            return launch_mid_l<2>(p, grid, stream);
     return cudaErrorInvalidValue;   // too many projections for the caches
 }
 
