@@ -386,6 +386,23 @@ __device__ __forceinline__ uint32_t quant4c(float4 v, float scale, bool zero, in
            ((uint32_t)(q3 & 0xff) << 24);
 }
 
+// This CTA's share [lo, hi) of n items: [n c / G, n (c + 1) / G).  In
+// 32-bit arithmetic when n G fits (a 64-bit division is a long call on the
+// GPU, and these sit on every stage's path; measured on B200: about 0.3 us
+// per stage for the two of the sum-buffer clearing alone).
+__device__ __forceinline__ void cta_share(int64_t n, int64_t &lo, int64_t &hi)
+{
+    const uint32_t G = gridDim.x, c = blockIdx.x;
+    if (n >= 0 && n * (int64_t)G < ((int64_t)1 << 32)) {
+        const uint32_t n32 = (uint32_t)n;
+        lo = n32 * c / G;
+        hi = n32 * (c + 1) / G;
+    } else {
+        lo = n * c / G;
+        hi = n * (c + 1) / G;
+    }
+}
+
 // Write this CTA's slice of an [mg x width] materialised buffer: element e
 // of the slice has value fn(m, j) for m = e / width, j = e % width (width a
 // multiple of 4; written 4 at a time) -- by threads tid = 0 .. nt - 1 of a
@@ -395,9 +412,12 @@ __device__ __forceinline__ void write_slice(float *dst, int64_t width, int mg, i
                                             F fn)
 {
     const int64_t n4 = (int64_t)mg * width / 4;
-    const int64_t lo = n4 * blockIdx.x / gridDim.x, hi = n4 * (blockIdx.x + 1) / gridDim.x;
+    int64_t lo, hi;
+    cta_share(n4, lo, hi);
+    const bool narrow = n4 < ((int64_t)1 << 31);   // (32-bit index arithmetic)
+    const uint32_t w4 = (uint32_t)(width / 4);
     for (int64_t e = lo + tid; e < hi; e += nt) {
-        const int m = (int)(e / (width / 4));
+        const int m = narrow ? (int)((uint32_t)e / w4) : (int)(e / (width / 4));
         const int64_t j = 4 * (e - (int64_t)m * (width / 4));
         *reinterpret_cast<float4 *>(dst + (int64_t)(m0 + m) * width + j) = fn(m, j);
     }
@@ -411,9 +431,11 @@ __device__ __forceinline__ void write_acc_slice(const Prev &P, int q, int mg, in
         return;
     const int64_t width = pr.N;
     const int64_t n = (int64_t)mg * width;
-    const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
+    int64_t lo, hi;
+    cta_share(n, lo, hi);
+    const bool narrow = n < ((int64_t)1 << 31);
     for (int64_t e = lo + tid; e < hi; e += nt) {
-        const int m = (int)(e / width);
+        const int m = narrow ? (int)((uint32_t)e / (uint32_t)width) : (int)(e / width);
         const int64_t j = e - (int64_t)m * width;
         pr.acc_out[(int64_t)(m0 + m) * width + j] =
             __ldcg(P.sum + (int64_t)m * P.ntot + pr.noff + j) - P.qs[m];
@@ -551,7 +573,8 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
     // ---- clear the first stage's sums, then the first barrier
     {
         const int64_t n = (int64_t)kChainGroup * h->max_ntot;
-        const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
+        int64_t lo, hi;
+        cta_share(n, lo, hi);
         for (int64_t e = lo + threadIdx.x; e < hi; e += kThreadsCh)
             sum_buf(0)[e] = 0;
     }
@@ -599,7 +622,8 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
         auto clear_next = [&]() {
             if (!final_phase && s + 1 < n_stages) {
                 const int64_t n = (int64_t)kChainGroup * sring[(s + 1) & 3].ntot;
-                const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
+                int64_t lo, hi;
+                cta_share(n, lo, hi);
                 int32_t *b = sum_buf(s + 1);
                 for (int64_t e = lo + threadIdx.x; e < hi; e += kThreadsCh)
                     b[e] = 0;
