@@ -13,14 +13,15 @@
 // k_i8_gemm, persistent, one CTA per SM, 128-token x 128-row output tiles:
 //   warp 0     TMA producer: per 128-byte k step one box of xq (128 x 128 B)
 //              and one of wq (128 x 128 B), both 128-byte swizzled, into a
-//              4-stage ring (k past K and rows past M or N read as zero);
+//              ring of 4 or 5 stages (k past K and rows past M or N read as
+//              zero);
 //   warp 1     MMA issuer and TMEM owner: four tcgen05.mma kind::i8 (K = 32
 //              each) per stage into one of two 128-column int32 accumulators;
-//   warps 2-9  epilogue, two per TMEM lane quarter (32 tokens), each taking
-//              half of the tile's columns: per 32 columns, tcgen05.ld,
-//              rescale + bias + ReLU (the tile's bias staged in shared
-//              memory), a 128-byte-swizzled 4 KB staging buffer (three per
-//              warp, in turn), and a TMA store of the 32 x 32 box (clipped
+//   warps 2-   epilogue, 8 or 16 warps (2 or 4 per TMEM lane quarter of 32
+//              tokens), each taking half or a quarter of the tile's columns:
+//              per 32 columns, tcgen05.ld, rescale + bias + ReLU (the tile's
+//              bias staged in shared memory), a 128-byte-swizzled 4 KB
+//              staging buffer, and a TMA store of the 32 x 32 box (clipped
 //              at M and N).  When N is
 //              not a multiple of 4 (the output's row pitch is then not a
 //              multiple of 16 bytes), the warp stores the staged box with
@@ -44,17 +45,31 @@ namespace {
 constexpr int kBM = 128;                       // tokens per tile (MMA M)
 constexpr int kBN = 128;                       // weight rows per tile (MMA N)
 constexpr int kBK = 128;                       // bytes of k per stage
-constexpr int kStages = 3;
 constexpr int kABytes = kBM * kBK;             // 16 KB
 constexpr int kBBytes = kBN * kBK;             // 16 KB
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = (2 + kEpiWarps) * 32;
-constexpr int kEpiBufs = 3;                    // staging buffers per epilogue warp
+constexpr int kEpiBufs = 1;                    // staging buffer per epilogue warp
 constexpr int kBoxBytes = 32 * 32 * 4;         // one 32 x 32 fp32 box
 constexpr int kTmemCols = 2 * kBN;
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiWarps * kEpiBufs * kBoxBytes + 1024 +
-                           kEpiWarps * 64 * 4;
+
+// Launch shapes: EW epilogue warps (8 or 16: EW / 4 per TMEM lane quarter,
+// each taking 16 / EW of the quarter's four 32-column boxes of a tile) and
+// ST load stages of 128 k bytes.  Measured on B200: with one
+// staging buffer per warp, 5 stages beside 8 epilogue warps took the
+// 32768 x 512 -> 2048 layer from 87.8 to 68.0 us (3 stages and 3 buffers
+// before: a K of 4 stages per tile left the load latency exposed) and left
+// 16384 x 256 -> 1024 at 20.6 us; 16 epilogue warps beside 4 stages took
+// that one to 18.7 us (K of 2 stages per tile: the epilogue bounds it) but
+// the other to 77.0 us.
+template <int EW, int ST>
+struct I8Shape {
+    static_assert(EW % 4 == 0 && 16 % EW == 0, "epilogue warps");
+    static constexpr int kEpiWarps = EW, kStages = ST, kBoxesPerWarp = 16 / EW;
+    static constexpr int kThreads = (2 + EW) * 32;
+    static constexpr int kSmemBytes =
+        1024 + ST * kStageBytes + EW * kEpiBufs * kBoxBytes + 1024 + EW * 64 * 4;
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
 constexpr uint64_t kDrainNs = 1000000000ull;
 
 struct alignas(64) I8Params {
@@ -86,8 +101,10 @@ __device__ __forceinline__ void tile_coords(const I8Params &p, int64_t t, int64_
     mi = t - nj * p.tiles_m;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_i8_gemm(const __grid_constant__ I8Params p)
+template <int EW, int ST>
+__global__ void __launch_bounds__(I8Shape<EW, ST>::kThreads, 1) k_i8_gemm(const __grid_constant__ I8Params p)
 {
+    constexpr int kEpiWarps = EW, kStages = ST, kBoxesPerWarp = I8Shape<EW, ST>::kBoxesPerWarp;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -202,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_i8_gemm(const __grid_constant__
         // ------------------------------------------------------ epilogue
         const int quarter = warp & 3;          // TMEM lanes 32q .. 32q + 31
         const int ew = warp - 2;
-        const int half = ew >> 2;              // columns [64 half, 64 half + 64) of the tile
+        const int half = ew >> 2;              // columns [32 B half, 32 B (half + 1)) of the tile, B = kBoxesPerWarp
         const uint32_t stg = stg0 + (uint32_t)(ew * kEpiBufs * kBoxBytes);
         float *stg_f = reinterpret_cast<float *>(gen_base + (stg - base));
         const float sw = __fdiv_rn(__ldg(p.amax_w), 127.f);
@@ -218,10 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_i8_gemm(const __grid_constant__
             int64_t mi, nj;
             tile_coords(p, t, mi, nj);
             const int64_t m = mi * kBM + 32 * quarter + lane;
-            const int64_t n = nj * kBN + 64 * half + lane;
+            const int64_t n = nj * kBN + 32 * kBoxesPerWarp * half + lane;
             amax_n = m < p.M ? __ldg(p.amax_x + m) : 0.f;
             bias_n0 = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.f;
-            bias_n1 = (p.bias && n + 32 < p.N) ? __ldg(p.bias + n + 32) : 0.f;
+            bias_n1 = (kBoxesPerWarp > 1 && p.bias && n + 32 < p.N) ? __ldg(p.bias + n + 32) : 0.f;
         };
         load_scales(blockIdx.x);
         for (int64_t t = blockIdx.x; t < p.tiles; t += G, ++tt) {
@@ -241,12 +258,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_i8_gemm(const __grid_constant__
             if (!mbar_wait(b_tfull + 8 * ab, (uint32_t)((tt / 2) & 1), p.ctl, abort_flag))
                 break;
             tc_fence_after();
-            for (int hc = 0; hc < 2; ++hc) {
-                const int cc = 2 * half + hc;
+            for (int hc = 0; hc < kBoxesPerWarp; ++hc) {
+                const int cc = kBoxesPerWarp * half + hc;
                 const int64_t n0 = nj * kBN + 32 * cc;
                 uint32_t v[32];
                 tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(ab * kBN + 32 * cc), v);
-                if (hc == 1) {
+                if (hc == kBoxesPerWarp - 1) {
                     // the accumulator has been read: release it to the MMA warp
                     tc_fence_before();
                     __syncwarp();
@@ -418,6 +435,19 @@ int i8_shape(const char *fn, int64_t M, int64_t N, int64_t K)
     return TW_OK;
 }
 
+
+template <int EW, int ST>
+cudaError_t launch_i8_shape(const I8Params &p, int grid, cudaStream_t stream)
+{
+    using S = I8Shape<EW, ST>;
+    cudaError_t e = cudaFuncSetAttribute(k_i8_gemm<EW, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         S::kSmemBytes);
+    if (e != cudaSuccess)
+        return e;
+    k_i8_gemm<EW, ST><<<(unsigned)grid, S::kThreads, S::kSmemBytes, stream>>>(p);
+    return cudaGetLastError();
+}
+
 int launch_i8(const int8_t *xq, const float *amax_x, int64_t M, int64_t N, int64_t K,
               const int8_t *wq, const float *amax_w, const float *bias, int relu, float *y,
               int32_t *acc_out, cudaStream_t stream)
@@ -457,13 +487,14 @@ int launch_i8(const int8_t *xq, const float *amax_x, int64_t M, int64_t N, int64
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess)
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_i8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess)
         return record_error(TW_ERR_CUDA, cudaGetErrorString(e));
     const int64_t grid = p.tiles < sms ? p.tiles : sms;
-    k_i8_gemm<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(p);
-    e = cudaGetLastError();
+    // K of at most two stages per tile: the epilogue bounds the layer
+    if (K <= 2 * kBK)
+        e = launch_i8_shape<16, 4>(p, (int)grid, stream);
+    else
+        e = launch_i8_shape<8, 5>(p, (int)grid, stream);
     return e == cudaSuccess ? TW_OK : record_error(TW_ERR_CUDA, cudaGetErrorString(e));
 }
 
