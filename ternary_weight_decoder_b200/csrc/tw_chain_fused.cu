@@ -686,20 +686,17 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
                     red_f[warp * kChainGroup + m] = am[m];
             }
             __syncthreads();
-            if (threadIdx.x < mg) {
-                float a = 0.f;
-                for (int w = 0; w < kNW; ++w)
-                    a = fmaxf(a, red_f[w * kChainGroup + threadIdx.x]);
-                sa_s[threadIdx.x] = __fdiv_rn(a, 127.f);
-                scale_s[threadIdx.x] = a == 0.f ? 0.f : __fdiv_rn(127.f, a);
-            }
-            __syncthreads();
-            // quantise the kept values into shared memory, with sum(q) per token
+            // quantise the kept values into shared memory, with sum(q) per
+            // token; every thread reduces the warps' maxima itself, so no
+            // second barrier precedes the quantisation
 #pragma unroll
             for (int m = 0; m < kRegTokens; ++m) {
                 if (m >= mg)
                     break;
-                const float sc = scale_s[m];
+                float a = 0.f;
+                for (int w = 0; w < kNW; ++w)
+                    a = fmaxf(a, red_f[w * kChainGroup + m]);
+                const float sc = a == 0.f ? 0.f : __fdiv_rn(127.f, a);
                 const bool zero = sc == 0.f;
                 uint32_t *row = reinterpret_cast<uint32_t *>(xbuf + m * p.xstride);
                 int sq = 0;
@@ -716,16 +713,17 @@ __global__ void __launch_bounds__(kThreadsCh, 1) k_chain(const __grid_constant__
                     red_i[warp * kChainGroup + m] = sq;
             }
             __syncthreads();
+            // this stage's scales serve the next prologue's rescale (read
+            // after the grid barrier)
             if (threadIdx.x < mg) {
                 int q = 0;
-                for (int w = 0; w < kNW; ++w)
+                float a = 0.f;
+                for (int w = 0; w < kNW; ++w) {
                     q += red_i[w * kChainGroup + threadIdx.x];
-                qs_s[threadIdx.x] = q;
-            }
-            __syncthreads();
-            if (threadIdx.x < mg) {
-                psa2[(s & 1) * kChainGroup + threadIdx.x] = sa_s[threadIdx.x];
-                pqs2[(s & 1) * kChainGroup + threadIdx.x] = qs_s[threadIdx.x];
+                    a = fmaxf(a, red_f[w * kChainGroup + threadIdx.x]);
+                }
+                psa2[(s & 1) * kChainGroup + threadIdx.x] = __fdiv_rn(a, 127.f);
+                pqs2[(s & 1) * kChainGroup + threadIdx.x] = q;
             }
         } else {
             // per token: amax over the row, then 127/amax (one token at a time
