@@ -125,7 +125,7 @@ int run_prefill_single(const int8_t *xq, const float *amax, const int32_t *qsum,
     r.acc_out = acc_out;
     r.N = N;
     r.K = K;
-    int rc = tw::encode_xq_tmap(xq, M, K, r.tmap_xq);
+    int rc = tw::encode_xq_tmap(xq, M, K, 128, r.tmap_xq);   // the 128-token tiles of the GEMM
     if (!rc)
         rc = tw::encode_codes_tmap(r.packed, N, K, 16, 1, r.tmap_codes);
     if (rc)
@@ -532,7 +532,7 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
             // CUDA driver (-1) a decode table is still encoded for its sizes;
             // the sweep refuses it.
             const bool mid = tw::sweep_on_mid(M);
-            int rc = decode ? 0 : tw::encode_xq_tmap(s.xq, M, s.K, r.tmap_xq);
+            int rc = decode ? 0 : tw::encode_xq_tmap(s.xq, M, s.K, mid ? tw::mid_ntok(M) : 128, r.tmap_xq);
             if (!rc)
                 rc = tw::encode_codes_tmap(r.packed, s.N, s.K, decode || mid ? 8 : 16,
                                            decode ? tw::kTcGroup : mid ? tw::kMidGroup : 1,

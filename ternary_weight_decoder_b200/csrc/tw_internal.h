@@ -226,6 +226,12 @@ int64_t mid_units(int64_t M, int64_t N);
 #define TW_MID_MAX_M 192
 #endif
 inline bool sweep_on_mid(int64_t M) { return M > kDecodeMaxM && M <= TW_MID_MAX_M; }
+// Tokens per unit of the weights-in-TMEM GEMM (the MMA's N side): 128, or
+// 192 above 128 tokens, where two 128-token units would leave the second
+// partly empty (measured on B200 over the 196 projections: 334 / 336 / 345
+// -> 286 / 292 / 339 us at 144 / 160 / 192 tokens; 192-token units lose at
+// 128 tokens and below).
+inline int mid_ntok(int64_t M) { return M <= 128 ? 128 : 192; }
 
 struct PrefillLaunch {
     const DescRecord *table;  // device records (or null: use `single`)
@@ -240,7 +246,7 @@ cudaError_t launch_prefill(const PrefillLaunch &L, uint32_t *err, uint64_t timeo
 int64_t prefill_tiles(int64_t M, int64_t N);
 // Encode the TMA descriptor of xq [M x K] int8 into out128 (128 bytes).
 // Returns 0, -1 when the driver entry point is unavailable, or a CUresult.
-int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, void *out128);
+int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, int box_m, void *out128);
 // Encode the TMA descriptor of the packed codes of an [N x K] matrix, seen as
 // [ceil(N/16)] x [K/128] tiles of 128 32-bit words (one box = box_rb row
 // blocks x box_kt consecutive k tiles; row blocks and k tiles past the

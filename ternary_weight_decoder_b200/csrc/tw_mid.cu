@@ -1,7 +1,8 @@
 // tw_mid.cu — ternary GEMM for more than 32 tokens with the weights held
 // in tensor memory: the 128-row side of tcgen05.mma kind::i8 is a tile of
 // ternary codes expanded to int8 {0, 1, 2} (= code + 1) straight into TMEM,
-// and the N side is up to 128 int8 token rows loaded by TMA from xq.
+// and the N side is a tile of 128 (192 above 128 tokens) int8 token rows
+// loaded by TMA from xq.
 //
 // What it computes, per projection (per-tensor ternary weights, s =
 // 1/mean|W|: "VibeVoice-ASR-BitNet-ONNX" model page, Quantization table; the
@@ -16,12 +17,12 @@
 // read once by the expansion or the MMAs, against 48 KB of operand reads
 // plus a 32 KB expanded tile when the weights are the shared-memory operand.
 //
-// Work unit: one 128-row tile of one projection times one 128-token tile,
-// over all of K; units are claimed from a counter, projections of larger K
+// Work unit: one 128-row tile of one projection times one token tile of
+// 128 tokens (192 when M > 128: fewer, fuller units), over all of K; units are claimed from a counter, projections of larger K
 // first.  A stage is a pair of 128-column k tiles (one barrier wait and one
 // commit of the MMA thread per 8 MMAs):
 //   * warp 0 loads the 8 row blocks x 2 k tiles of codes (one 3-D TMA box,
-//     k tiles past K read as zero codes) and the two 128 x 128 B token tiles
+//     k tiles past K read as zero codes) and the two NT x 128 B token tiles
 //     (2-D TMA boxes of xq, 128-byte swizzled, tokens past M read as zero)
 //     into a ring of L shared-memory stages;
 //   * eight expansion warps (two sets of four, one warp per TMEM lane
@@ -29,10 +30,11 @@
 //     tile into 16 registers holding code + 1 for 4 consecutive k each, in
 //     the natural k order of the MMA's K (each register's 16 source bits
 //     come from the word of lane 2(u & 1) + t/2 of the row's quad, fetched
-//     with a shuffle), and store them to one of 4 TMEM A slots of 2 x 32
-//     columns (tcgen05.st 16x256b: column c of a k tile holds k = 4c .. 4c+3);
+//     with a shuffle), and store them to one of the TMEM A slots of 2 x 32
+//     columns (4 for 128-token units, 2 for 192; tcgen05.st 16x256b: column c
+//     of a k tile holds k = 4c .. 4c+3);
 //   * warp 1 issues four MMAs of K = 32 per k tile into the unit's
-//     accumulator (N = 128 columns, one of two) and commits them to the
+//     accumulator (N = NT columns, one of two) and commits them to the
 //     stage's empty barrier, which frees the stage and, four stages later,
 //     the A slot;
 //   * four epilogue warps (one per lane quarter: 32 weight rows each) read
@@ -52,17 +54,29 @@
 namespace tw {
 namespace {
 
-constexpr int kNTok = 128;                       // tokens per unit (MMA N)
 constexpr int kGrpM = kMidGroup;                 // k tiles per stage
-constexpr int kASlotsM = 8 / kGrpM;              // A slots of kGrpM x 32 columns
 constexpr int kRingM = 8;                        // unit-info entries
 constexpr int kThreadsM = 14 * 32;
 constexpr int kCodeBytesM = 8 * kGrpM * kTileBytes;   // 128 rows x 2 x 128 k = 8 KB
-constexpr int kTokBytesM = kNTok * 128;           // 16 KB per k tile
-constexpr int kStageM = kCodeBytesM + kGrpM * kTokBytesM;
 constexpr int kTmemColsM = 512;
-constexpr int kDCol0M = 256;                     // two accumulators after 8 A slots
 constexpr int kMiscM = 2048;
+
+// The shape of a unit of NT tokens (the MMA's N side, 128 or 192): the
+// tensor memory holds the two accumulators of NT columns after the A slots,
+// which take the rest (8 slots of one k-tile pair for 128 tokens, 2 for
+// 192).
+template <int NT>
+struct MidShape {
+    static constexpr int kNTok = NT;
+    static constexpr int kASlots = (kTmemColsM - 2 * NT) / (32 * kGrpM);   // A slots of kGrpM x 32 columns
+    static constexpr int kTokBytes = NT * 128;                               // per k tile
+    static constexpr int kStage = kCodeBytesM + kGrpM * kTokBytes;
+    static constexpr int kDCol0 = 32 * kGrpM * kASlots;                      // the accumulators
+    // int8 x int8 -> int32, K-major, M = 128, N = NT.
+    static constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NT >> 3) << 17) |
+                                       ((128u >> 4) << 24);
+    static_assert(NT % 32 == 0 && NT <= 256 && kASlots >= 2, "unit shape");
+};
 constexpr uint64_t kDrainNsM = 1000000000ull;
 
 struct UnitM {
@@ -85,22 +99,18 @@ struct MidParams {
     const UnitOrder *order;   // projections by K, descending, with their first unit
     int count;
     int M;
-    int tiles_m;              // token tiles of 128
+    int tiles_m;              // token tiles of the unit width
     int64_t total_units;
     uint32_t *ctr;            // [0] claim counter, [1] finished blocks
     WaitCtl ctl;
 };
 
 constexpr int kBoxM = 32 * 32 * 4;               // one epilogue warp's staging box
-template <int L>
+template <int NT, int L>
 constexpr int smem_mid(int count)
 {
-    return 1024 + L * kStageM + 4 * kBoxM + kMiscM + (16 + (int)sizeof(ProjM)) * count;
+    return 1024 + L * MidShape<NT>::kStage + 4 * kBoxM + kMiscM + (16 + (int)sizeof(ProjM)) * count;
 }
-
-// int8 x int8 -> int32, K-major, M = 128, N = 128.
-constexpr uint32_t kIdescMid = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kNTok >> 3) << 17) |
-                               ((128u >> 4) << 24);
 
 __device__ UnitM locate_unit_m(const MidParams &p, const UnitOrder *order, int64_t uid)
 {
@@ -116,9 +126,13 @@ __device__ UnitM locate_unit_m(const MidParams &p, const UnitOrder *order, int64
     return UnitM{order[lo].d, local / p.tiles_m, local % p.tiles_m, 1};
 }
 
-template <int L>
+template <int NT, int L>
 __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ MidParams p)
 {
+    using S = MidShape<NT>;
+    constexpr int kNTok = S::kNTok, kASlotsM = S::kASlots, kTokBytesM = S::kTokBytes;
+    constexpr int kStageM = S::kStage, kDCol0M = S::kDCol0;
+    constexpr uint32_t kIdescMid = S::kIdesc;
     static_assert(L >= 2 && L >= kASlotsM, "load stages");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -331,9 +345,14 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
                 if (32 * c >= nvalid)
                     continue;   // (uniform across the warp)
                 // (selected, not indexed: the arrays stay in registers)
-                static_assert(kNTok / 32 == 4, "token groups");
-                const float sa_c = c == 0 ? sa_l[0] : c == 1 ? sa_l[1] : c == 2 ? sa_l[2] : sa_l[3];
-                const int qs_c = c == 0 ? qs_l[0] : c == 1 ? qs_l[1] : c == 2 ? qs_l[2] : qs_l[3];
+                float sa_c = sa_l[0];
+                int qs_c = qs_l[0];
+#pragma unroll
+                for (int i = 1; i < kNTok / 32; ++i)
+                    if (c == i) {
+                        sa_c = sa_l[i];
+                        qs_c = qs_l[i];
+                    }
                 for (int pass = 0; pass < (pr.acc_out ? 2 : 1); ++pass) {
                     // box[n][lane] = token 32c + n of this lane's row
 #pragma unroll
@@ -446,22 +465,42 @@ __global__ void __launch_bounds__(kThreadsM, 1) k_mid(const __grid_constant__ Mi
     }
 }
 
-template <int L>
+template <int NT, int L>
 cudaError_t launch_mid_l(const MidParams &p, int grid, cudaStream_t stream)
 {
-    const int smem = smem_mid<L>(p.count);
-    cudaError_t e = cudaFuncSetAttribute(k_mid<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = smem_mid<NT, L>(p.count);
+    cudaError_t e = cudaFuncSetAttribute(k_mid<NT, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return e;
-    k_mid<L><<<(unsigned)grid, kThreadsM, smem, stream>>>(p);
+    k_mid<NT, L><<<(unsigned)grid, kThreadsM, smem, stream>>>(p);
     return cudaGetLastError();
+}
+
+// The deepest ring of load stages that fits beside the caches (fewer stages
+// only where every A slot has a load stage of its own).
+template <int NT>
+cudaError_t launch_mid_nt(const MidParams &p, int grid, cudaStream_t stream)
+{
+    constexpr int kLimit = 227 * 1024, kA = MidShape<NT>::kASlots;
+    if (smem_mid<NT, 5>(p.count) <= kLimit)
+        return launch_mid_l<NT, 5>(p, grid, stream);
+    if (smem_mid<NT, 4>(p.count) <= kLimit)
+        return launch_mid_l<NT, 4>(p, grid, stream);
+    if constexpr (kA <= 3)
+        if (smem_mid<NT, 3>(p.count) <= kLimit)
+            return launch_mid_l<NT, 3>(p, grid, stream);
+    if constexpr (kA <= 2)
+        if (smem_mid<NT, 2>(p.count) <= kLimit)
+            return launch_mid_l<NT, 2>(p, grid, stream);
+    return cudaErrorInvalidValue;   // too many projections for the caches
 }
 
 }  // namespace
 
 int64_t mid_units(int64_t M, int64_t N)
 {
-    return ((N + 127) / 128) * ((M + kNTok - 1) / kNTok);
+    const int nt = mid_ntok(M);
+    return ((N + 127) / 128) * ((M + nt - 1) / nt);
 }
 
 cudaError_t launch_mid(const MidLaunch &L, uint32_t *err, uint64_t timeout_ns, cudaStream_t stream)
@@ -478,26 +517,15 @@ cudaError_t launch_mid(const MidLaunch &L, uint32_t *err, uint64_t timeout_ns, c
     p.order = L.order;
     p.count = L.count;
     p.M = (int)L.M;
-    p.tiles_m = (int)((L.M + kNTok - 1) / kNTok);
+    const int nt = mid_ntok(L.M);
+    p.tiles_m = (int)((L.M + nt - 1) / nt);
     p.total_units = L.total_units;
     p.ctr = L.ctr;
     p.ctl.err = err;
     p.ctl.timeout_ns = timeout_ns;
     const int64_t grid64 = L.total_units < sms ? L.total_units : sms;
     const int grid = (int)(grid64 < 1 ? 1 : grid64);
-    constexpr int kLimit = 227 * 1024;
-    if (smem_mid<5>(p.count) <= kLimit)
-        return launch_mid_l<5>(p, grid, stream);
-    if (smem_mid<4>(p.count) <= kLimit)
-        return launch_mid_l<4>(p, grid, stream);
-    // (fewer stages only where every A slot has a load stage of its own)
-    if constexpr (kASlotsM <= 3)
-        if (smem_mid<3>(p.count) <= kLimit)
-            return launch_mid_l<3>(p, grid, stream);
-    if constexpr (kASlotsM <= 2)
-        if (smem_mid<2>(p.count) <= kLimit)
-            return launch_mid_l<2>(p, grid, stream);
-    return cudaErrorInvalidValue;   // too many projections for the caches
+    return nt == 192 ? launch_mid_nt<192>(p, grid, stream) : launch_mid_nt<128>(p, grid, stream);
 }
 
 }  // namespace tw

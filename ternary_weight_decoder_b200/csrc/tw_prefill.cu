@@ -400,7 +400,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, void *out128)
+int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, int box_m, void *out128)
 {
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
@@ -416,7 +416,7 @@ int encode_xq_tmap(const int8_t *xq, int64_t M, int64_t K, void *out128)
     memset(&m, 0, sizeof(m));
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)K};
-    const cuuint32_t box[2] = {kBK, kBM};
+    const cuuint32_t box[2] = {kBK, (cuuint32_t)box_m};   // 128 k bytes x box_m tokens
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(xq), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
