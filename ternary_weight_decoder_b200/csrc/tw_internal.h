@@ -226,12 +226,13 @@ int64_t mid_units(int64_t M, int64_t N);
 #define TW_MID_MAX_M 192
 #endif
 inline bool sweep_on_mid(int64_t M) { return M > kDecodeMaxM && M <= TW_MID_MAX_M; }
-// Tokens per unit of the weights-in-TMEM GEMM (the MMA's N side): 128, or
-// 192 above 128 tokens, where two 128-token units would leave the second
-// partly empty (measured on B200 over the 196 projections: 334 / 336 / 345
-// -> 286 / 292 / 339 us at 144 / 160 / 192 tokens; 192-token units lose at
-// 128 tokens and below).
-inline int mid_ntok(int64_t M) { return M <= 128 ? 128 : 192; }
+// Tokens per unit of the weights-in-TMEM GEMM (the MMA's N side): the
+// narrowest of 64, 96, 128 and 192 that holds M, so that no unit is mostly
+// empty (measured on B200 over the 196 projections against 128-token units
+// throughout: 196.5 / 182.4 -> 159.2 / 162.4 us at 33 / 64 tokens, 188.2 /
+// 191.5 -> 173.0 / 176.3 at 80 / 96, 334 / 336 / 345 -> 286 / 292 / 339 at
+// 144 / 160 / 192).
+inline int mid_ntok(int64_t M) { return M <= 64 ? 64 : M <= 96 ? 96 : M <= 128 ? 128 : 192; }
 
 struct PrefillLaunch {
     const DescRecord *table;  // device records (or null: use `single`)

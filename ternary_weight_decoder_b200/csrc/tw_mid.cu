@@ -1,7 +1,7 @@
 // tw_mid.cu — ternary GEMM for more than 32 tokens with the weights held
 // in tensor memory: the 128-row side of tcgen05.mma kind::i8 is a tile of
 // ternary codes expanded to int8 {0, 1, 2} (= code + 1) straight into TMEM,
-// and the N side is a tile of 128 (192 above 128 tokens) int8 token rows
+// and the N side is a tile of 64, 96, 128 or 192 int8 token rows (by M)
 // loaded by TMA from xq.
 //
 // What it computes, per projection (per-tensor ternary weights, s =
@@ -17,8 +17,8 @@
 // read once by the expansion or the MMAs, against 48 KB of operand reads
 // plus a 32 KB expanded tile when the weights are the shared-memory operand.
 //
-// Work unit: one 128-row tile of one projection times one token tile of
-// 128 tokens (192 when M > 128: fewer, fuller units), over all of K; units are claimed from a counter, projections of larger K
+// Work unit: one 128-row tile of one projection times one token tile of NT
+// tokens (NT = 64, 96, 128 or 192 by M: fewer, fuller units), over all of K; units are claimed from a counter, projections of larger K
 // first.  A stage is a pair of 128-column k tiles (one barrier wait and one
 // commit of the MMA thread per 8 MMAs):
 //   * warp 0 loads the 8 row blocks x 2 k tiles of codes (one 3-D TMA box,
@@ -31,7 +31,7 @@
 //     the natural k order of the MMA's K (each register's 16 source bits
 //     come from the word of lane 2(u & 1) + t/2 of the row's quad, fetched
 //     with a shuffle), and store them to one of the TMEM A slots of 2 x 32
-//     columns (4 for 128-token units, 2 for 192; tcgen05.st 16x256b: column c
+//     columns (4 up to 128-token units, 2 for 192; tcgen05.st 16x256b: column c
 //     of a k tile holds k = 4c .. 4c+3);
 //   * warp 1 issues four MMAs of K = 32 per k tile into the unit's
 //     accumulator (N = NT columns, one of two) and commits them to the
@@ -61,14 +61,15 @@ constexpr int kCodeBytesM = 8 * kGrpM * kTileBytes;   // 128 rows x 2 x 128 k = 
 constexpr int kTmemColsM = 512;
 constexpr int kMiscM = 2048;
 
-// The shape of a unit of NT tokens (the MMA's N side, 128 or 192): the
-// tensor memory holds the two accumulators of NT columns after the A slots,
-// which take the rest (8 slots of one k-tile pair for 128 tokens, 2 for
-// 192).
+// The shape of a unit of NT tokens (the MMA's N side: 64, 96, 128 or 192):
+// the tensor memory holds the two accumulators of NT columns after the A
+// slots, which take the rest, at most four (4 slots of a k-tile pair for up
+// to 128 tokens, 2 for 192).
 template <int NT>
 struct MidShape {
     static constexpr int kNTok = NT;
-    static constexpr int kASlots = (kTmemColsM - 2 * NT) / (32 * kGrpM);   // A slots of kGrpM x 32 columns
+    static constexpr int kFit = (kTmemColsM - 2 * NT) / (32 * kGrpM);
+    static constexpr int kASlots = kFit < 4 ? kFit : 4;                     // A slots of kGrpM x 32 columns
     static constexpr int kTokBytes = NT * 128;                               // per k tile
     static constexpr int kStage = kCodeBytesM + kGrpM * kTokBytes;
     static constexpr int kDCol0 = 32 * kGrpM * kASlots;                      // the accumulators
@@ -525,7 +526,12 @@ cudaError_t launch_mid(const MidLaunch &L, uint32_t *err, uint64_t timeout_ns, c
     p.ctl.timeout_ns = timeout_ns;
     const int64_t grid64 = L.total_units < sms ? L.total_units : sms;
     const int grid = (int)(grid64 < 1 ? 1 : grid64);
-    return nt == 192 ? launch_mid_nt<192>(p, grid, stream) : launch_mid_nt<128>(p, grid, stream);
+    switch (nt) {
+    case 64: return launch_mid_nt<64>(p, grid, stream);
+    case 96: return launch_mid_nt<96>(p, grid, stream);
+    case 192: return launch_mid_nt<192>(p, grid, stream);
+    default: return launch_mid_nt<128>(p, grid, stream);
+    }
 }
 
 }  // namespace tw

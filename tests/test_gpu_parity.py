@@ -408,13 +408,14 @@ def test_argument_errors(dev, api):
     assert not y.cpu().numpy().any()
 
 
-@pytest.mark.parametrize("M", [33, 64, 127, 128, 129, 191, 192, 193, 255, 300])
+@pytest.mark.parametrize("M", [33, 64, 65, 96, 97, 127, 128, 129, 191, 192, 193, 255, 300])
 def test_sweep_mid_m(dev, api, M):
     """More than 32 tokens (the weights-in-tensor-memory kernel up to 192,
-    the expanded-weights kernel from 193, both sides of the switch): every
-    token-tile tail, projections whose N is not a multiple of 128 (the last
-    128-row unit partial), several K, twice in a row (the unit counters are
-    left zero for the next call)."""
+    with units of 64, 96, 128 or 192 tokens by M and both sides of each
+    width switch; the expanded-weights kernel from 193): every token-tile
+    tail, projections whose N is not a multiple of 128 (the last 128-row
+    unit partial), several K, twice in a row (the unit counters are left
+    zero for the next call)."""
     import torch
     shapes = [(200, 256), (128, 1536), (17, 384), (385, 640), (256, 2048), (1, 128)]
     descs, keep = [], []
