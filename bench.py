@@ -20,7 +20,10 @@ benchmark definition, measured in the same run on the same weights:
   4. the 196-projection sweep at M = 4, 8, 16, 32 (fraction of HBM);
   5. the 196-projection prefill sweep at M = 256, 1024, 4096 on int8
      activations quantised beforehand (fraction of the int8 tensor peak);
-  and the decoder-layer chain (28 dependent layers at M = 1).
+  and the 196-projection sweep at M = 64, 128, 192 (more than 32 tokens:
+  the default weights-in-TMEM GEMM against the expanded-weights GEMM on the
+  same descriptors), the I8_S int8 linear layer with bias and ReLU, and the
+  decoder-layer chain (28 dependent layers at M = 1).
 Each decode/prefill entry also carries the oracle timed on the host's cores
 on a bounded sample (labelled, extrapolated by weight count and tokens).
 
@@ -53,6 +56,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 DTYPE = "int8xternary->int32, f32 in/out"
 DECODE_MS = (4, 8, 16, 32)
 PREFILL_MS = (256, 1024, 4096)
+MID_MS = (64, 128, 192)          # more than 32 tokens, below the expanded-weights crossover
 L2_FLUSH_BYTES = 256 << 20   # > 2 x the 126 MB L2
 PREFILL_DISTINCT_ROWS = 256  # distinct generated token rows per projection (tiled up to M)
 # I8_S encoder layer shapes (tokens M, channels K -> N = 4K): activations
@@ -72,7 +76,7 @@ def parse(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="headline only (no configs object)")
-    ap.add_argument("--configs", default="1,2,4,5,i8,chain",
+    ap.add_argument("--configs", default="1,2,4,5,mid,i8,chain",
                     help="comma list of the extra workloads to measure")
     ap.add_argument("--chain", action="store_true",
                     help="time the dependent decoder-layer chain instead of the sweep")
@@ -810,6 +814,42 @@ def measure_configs(args, api, torch, dev, rank, shapes, weights, descs_m1, want
                                              layers=args.layers)
             out[f"5_prefill_sweep_196x_M{M}"] = e
             del table, descs
+            torch.cuda.empty_cache()
+
+    if "mid" in want:
+        # 33..192 tokens: the default (weights expanded into tensor memory)
+        # against the expanded-weights GEMM on the same descriptors
+        for M in MID_MS:
+            descs = prefill_inputs(api, torch, dev, shapes, weights, M, rank)
+            e = {"M": M, "inputs": f"{min(M, PREFILL_DISTINCT_ROWS)} distinct seeded token rows "
+                                   f"per projection, quantised before the timed region"}
+            ops = sweep_ops(shapes, M)
+            _, codes, _ = sweep_bytes(shapes, M)
+            nbytes = codes + sum(M * K + M * N * 4 for (_, _, _, N, K) in shapes)
+            for gemm, name in (("auto", "tmem_weights"), ("expanded", "expanded_weights")):
+                table = api.SweepTable(descs, M, device=dev, gemm=gemm)
+                for _ in range(cwarm):
+                    api.decoder_projection_sweep(table)
+                api.check()
+                ms, per = timed_steps(torch, stream, lambda: api.decoder_projection_sweep(table),
+                                      psteps, barrier)
+                api.check()
+                step_s = ms / psteps / 1e3
+                e[name] = {"tokens_per_s": M / step_s, "us_per_step": step_s * 1e6,
+                           "step_times": dist_summary(per),
+                           "achieved_tops": ops / step_s / 1e12,
+                           "frac_int8": ops / step_s / 1e12 / int8_peak,
+                           "achieved_gbs": nbytes / step_s / 1e9,
+                           "frac_hbm": nbytes / step_s / 1e9 / hbm,
+                           "launches_per_step": table.launches}
+                del table
+            e["default"] = "tmem_weights"
+            e["speedup_vs_expanded"] = (e["expanded_weights"]["us_per_step"]
+                                        / e["tmem_weights"]["us_per_step"])
+            e["int8_ops"], e["algorithmic_bytes"] = ops, nbytes
+            e["traffic"] = profiled_traffic("tw_mid.cu", M, args.layers)
+            out[f"f2_mid_sweep_196x_M{M}"] = e
+            del descs
             torch.cuda.empty_cache()
 
     if "i8" in want:

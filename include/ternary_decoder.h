@@ -220,6 +220,25 @@ TW_API size_t tw_sweep_table_bytes(int count);
 TW_API int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M,
                           void *table, size_t table_bytes);
 
+/* The GEMM that a sweep of more than 32 tokens runs. */
+#define TW_SWEEP_GEMM_AUTO 0     /* by M: weights expanded into tensor memory */
+                                 /* for 33..192 tokens, into shared memory    */
+                                 /* above (the measured crossover)            */
+#define TW_SWEEP_GEMM_EXPANDED 1 /* weights expanded into shared memory for   */
+                                 /* every M > 32                              */
+
+/*
+ * HOST-ONLY.  tw_sweep_table_encode with the GEMM of a sweep of more than
+ * 32 tokens chosen by the caller: TW_SWEEP_GEMM_AUTO (what
+ * tw_sweep_table_encode does) or TW_SWEEP_GEMM_EXPANDED, which runs the
+ * expanded-weights GEMM at 33..192 tokens too (to time the two kernels
+ * against each other on the caller's own shapes).  Both give the same bits:
+ * the int32 sums are exact and the rescale is the same expression.  For
+ * M <= 32 the choice is ignored.  Any other value: TW_ERR_SHAPE.
+ */
+TW_API int tw_sweep_table_encode_gemm(const tw_proj_desc *descs, int count, int64_t M,
+                               int gemm, void *table, size_t table_bytes);
+
 /* Scratch needed by tw_decoder_projection_sweep for an encoded HOST table.
  * For decode (M <= 32) it holds 256 bytes of work counters, then the
  * quantised rows of every projection (room for 8, 16 or 32 token rows of K
@@ -236,8 +255,9 @@ TW_API size_t tw_sweep_workspace_bytes(const void *table_host);
  * widest projection does not fit shared memory and the tokens are split
  * into groups -- and for 8 < M <= 32 one launch of the tensor-core decode
  * kernel.  33..192 tokens: one persistent tensor-core launch with the
- * weights in tensor memory (units of 128 weight rows x 128 tokens, claimed
- * from the counters in the workspace); more tokens: one persistent
+ * weights in tensor memory (units of 128 weight rows x 64, 96, 128 or 192
+ * tokens, the narrowest that holds M, claimed from the counters in the
+ * workspace); more tokens (or TW_SWEEP_GEMM_EXPANDED): one persistent
  * tensor-core launch with the weights expanded in shared memory (output
  * tiles of 128 tokens x 256 weight rows dealt out round robin).  Either is
  * preceded by one quantisation launch when some descriptor gives x.

@@ -62,6 +62,9 @@ tw_ternary_linear_q = _sig("tw_ternary_linear_q", _int,
                            [_p, _p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p, _sz, _p])
 tw_sweep_table_bytes = _sig("tw_sweep_table_bytes", _sz, [_int])
 tw_sweep_table_encode = _sig("tw_sweep_table_encode", _int, [_p, _int, _i64, _p, _sz])
+tw_sweep_table_encode_gemm = _sig("tw_sweep_table_encode_gemm", _int,
+                                  [_p, _int, _i64, _int, _p, _sz])
+SWEEP_GEMM = {"auto": 0, "expanded": 1}   # TW_SWEEP_GEMM_AUTO, TW_SWEEP_GEMM_EXPANDED
 tw_sweep_workspace_bytes = _sig("tw_sweep_workspace_bytes", _sz, [_p])
 tw_decoder_projection_sweep = _sig("tw_decoder_projection_sweep", _int, [_p, _p, _p, _sz, _p])
 tw_sweep_launches = _sig("tw_sweep_launches", _int, [_p])
@@ -229,9 +232,13 @@ class SweepTable:
     """An encoded sweep over many projections: the host bytes written by
     ``tw_sweep_table_encode`` and their device copy.  The table holds
     references to the tensors its descriptors name (it stores their
-    addresses), so they stay allocated for as long as the table does."""
+    addresses), so they stay allocated for as long as the table does.
+    ``gemm`` picks the GEMM of a sweep of more than 32 tokens: "auto" (by M)
+    or "expanded" (the expanded-weights kernel at every M > 32;
+    ``tw_sweep_table_encode_gemm``)."""
 
-    def __init__(self, descs: Sequence[dict], M: int, device=None, workspace: bool = True):
+    def __init__(self, descs: Sequence[dict], M: int, device=None, workspace: bool = True,
+                 gemm: str = "auto"):
         n = len(descs)
         arr = (ProjDesc * n)()
         for i, d in enumerate(descs):
@@ -242,8 +249,8 @@ class SweepTable:
         nbytes = int(tw_sweep_table_bytes(n))
         self.host = torch.empty(nbytes, dtype=torch.uint8).pin_memory() \
             if torch.cuda.is_available() else torch.empty(nbytes, dtype=torch.uint8)
-        _raise(tw_sweep_table_encode(arr, n, M, _ptr(self.host), nbytes))
-        self.count, self.M = n, M
+        _raise(tw_sweep_table_encode_gemm(arr, n, M, SWEEP_GEMM[gemm], _ptr(self.host), nbytes))
+        self.count, self.M, self.gemm = n, M, gemm
         self.descs = [dict(d) for d in descs]   # owns what the records point at
         self.device = None
         if device is not None:

@@ -476,9 +476,17 @@ size_t tw_sweep_table_bytes(int count)
 int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void *table,
                           size_t table_bytes)
 {
+    return tw_sweep_table_encode_gemm(descs, count, M, TW_SWEEP_GEMM_AUTO, table, table_bytes);
+}
+
+int tw_sweep_table_encode_gemm(const tw_proj_desc *descs, int count, int64_t M, int gemm,
+                               void *table, size_t table_bytes)
+{
     t_last_error[0] = 0;
     if (!descs || !table)
         return fail(TW_ERR_NULL, "tw_sweep_table_encode: descs and table are required");
+    if (gemm != TW_SWEEP_GEMM_AUTO && gemm != TW_SWEEP_GEMM_EXPANDED)
+        return fail(TW_ERR_SHAPE, "gemm=%d is not a TW_SWEEP_GEMM_* value", gemm);
     if (count < 1)
         return fail(TW_ERR_SHAPE, "count=%d must be >= 1", count);
     if (table_bytes < tw_sweep_table_bytes(count))
@@ -487,6 +495,7 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
     if (M < 1 || M > (1 << 24))
         return fail(TW_ERR_SHAPE, "M=%lld out of range", (long long)M);
     const bool decode = M <= tw::kDecodeMaxM;
+    const bool mid = gemm == TW_SWEEP_GEMM_AUTO && tw::sweep_on_mid(M);
     auto *hdr = static_cast<tw::TableHeader *>(table);
     auto *recs = reinterpret_cast<tw::DescRecord *>(hdr + 1);
     memset(table, 0, tw_sweep_table_bytes(count));
@@ -531,7 +540,6 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
             // GEMM) or 256 rows x 1 k tile (expanded-weights GEMM).  Without a
             // CUDA driver (-1) a decode table is still encoded for its sizes;
             // the sweep refuses it.
-            const bool mid = tw::sweep_on_mid(M);
             int rc = decode ? 0 : tw::encode_xq_tmap(s.xq, M, s.K, mid ? tw::mid_ntok(M) : 128, r.tmap_xq);
             if (!rc)
                 rc = tw::encode_codes_tmap(r.packed, s.N, s.K, decode || mid ? 8 : 16,
@@ -581,8 +589,9 @@ int tw_sweep_table_encode(const tw_proj_desc *descs, int count, int64_t M, void 
     hdr->total_ptiles = ptiles;
     // decode: counters, rows and scales; more tokens: the unit counters of the
     // weights-in-TMEM kernel
-    hdr->ws_bytes = decode ? ws_off + 256 * (int64_t)count : (tw::sweep_on_mid(M) ? tw::kWsCtrBytes : 0);
-    hdr->max_K = max_K;
+    hdr->ws_bytes = decode ? ws_off + 256 * (int64_t)count : (mid ? tw::kWsCtrBytes : 0);
+    hdr->max_K = (int32_t)max_K;
+    hdr->gemm = decode ? TW_SWEEP_GEMM_AUTO : gemm;
     hdr->total_cost = cost;
     return TW_OK;
 }
@@ -597,6 +606,12 @@ size_t tw_sweep_workspace_bytes(const void *table_host)
 
 // Whether a sweep of more than 32 tokens quantises some descriptor's fp32 x
 // itself (first launch) before the GEMM.
+// Whether a host table of more than 32 tokens runs the weights-in-TMEM GEMM.
+static bool table_on_mid(const tw::TableHeader *hdr)
+{
+    return hdr->gemm == TW_SWEEP_GEMM_AUTO && tw::sweep_on_mid(hdr->M);
+}
+
 static bool sweep_quantises_x(const tw::TableHeader *hdr)
 {
     if (hdr->M <= tw::kDecodeMaxM)
@@ -632,7 +647,7 @@ int tw_decoder_projection_sweep(const void *table_host, const void *table_dev, v
     uint32_t *err = nullptr;
     if (int rc = err_word(&err))
         return rc;
-    if (tw::sweep_on_mid(hdr->M)) {
+    if (table_on_mid(hdr)) {
         if (ws_bytes < (size_t)hdr->ws_bytes || !ws)
             return fail(TW_ERR_BUFSIZE, "sweep workspace %zu < %lld bytes", ws_bytes,
                         (long long)hdr->ws_bytes);

@@ -48,7 +48,8 @@ struct alignas(64) TableHeader {
     int64_t total_rb;
     int64_t total_units; // decode: 128-row units of the tensor-core sweep
     int64_t total_ptiles;
-    int64_t max_K;
+    int32_t max_K;       // K <= 2^24
+    int32_t gemm;        // more than 32 tokens: the TW_SWEEP_GEMM_* the table was encoded for
     int64_t total_cost;  // decode: cost units of the sweep
     int64_t ws_bytes;    // decode: scratch (counter, ready flags, int8 rows, scales)
 };

@@ -69,8 +69,8 @@ REC = np.dtype([("x", "<u8"), ("xq", "<u8"), ("amax", "<u8"), ("qsum", "<u8"),
                 ("tmap_ok", "<i8"),
                 ("tmap", "u1", 128), ("tmap_codes", "u1", 128)])
 HDR = np.dtype([("magic", "<u4"), ("count", "<i4"), ("M", "<i8"), ("total_rb", "<i8"),
-                ("total_units", "<i8"), ("total_ptiles", "<i8"), ("max_K", "<i8"),
-                ("total_cost", "<i8"), ("ws_bytes", "<i8")])
+                ("total_units", "<i8"), ("total_ptiles", "<i8"), ("max_K", "<i4"),
+                ("gemm", "<i4"), ("total_cost", "<i8"), ("ws_bytes", "<i8")])
 
 
 def test_table_encode_prefix_sums(lib):
@@ -126,6 +126,29 @@ def test_table_encode_rejects(lib, bad, status):
     buf = np.zeros(n, np.uint8)
     assert api.tw_sweep_table_encode(arr, 2, 4, buf.ctypes.data, n) == status
     assert api.tw_last_error()
+
+
+def test_table_encode_gemm_choice(lib):
+    """The GEMM choice: only TW_SWEEP_GEMM_AUTO (0) and _EXPANDED (1) are
+    accepted, before any descriptor is read; a decode table ignores it and
+    encodes the same bytes as tw_sweep_table_encode."""
+    from ternary_weight_decoder_b200 import api
+    shapes = [(1536, 1536), (17, 256)]
+    arr = _descs(shapes)
+    n = api.tw_sweep_table_bytes(len(shapes))
+    for bad in (-1, 2, 7):
+        buf = np.zeros(n, np.uint8)
+        assert api.tw_sweep_table_encode_gemm(arr, 2, 1, bad, buf.ctypes.data, n) == 2
+        assert b"gemm" in api.tw_last_error()
+        assert not buf.any()
+    ref = np.zeros(n, np.uint8)
+    assert api.tw_sweep_table_encode(arr, 2, 4, ref.ctypes.data, n) == 0
+    for gemm in (0, 1):
+        buf = np.zeros(n, np.uint8)
+        assert api.tw_sweep_table_encode_gemm(arr, 2, 4, gemm, buf.ctypes.data, n) == 0
+        assert (buf == ref).all()
+        assert buf[:64].view(HDR)[0]["gemm"] == 0
+    assert api.SWEEP_GEMM == {"auto": 0, "expanded": 1}
 
 
 def test_table_encode_rejects_small_buffer_and_count(lib):

@@ -86,4 +86,4 @@ def test_dist_summary_and_cpu_info():
 def test_bench_arguments_default_to_one_gpu():
     a = bench.parse([])
     assert a.gpus == 1 and a.m == 1 and a.layers == 28 and a.warmup >= 3
-    assert set(a.configs.split(",")) == {"1", "2", "4", "5", "i8", "chain"}
+    assert set(a.configs.split(",")) == {"1", "2", "4", "5", "mid", "i8", "chain"}

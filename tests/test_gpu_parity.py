@@ -441,3 +441,35 @@ def test_sweep_mid_m(dev, api, M):
         for d in descs:
             d["y"].fill_(float("nan"))
             d["acc_out"].fill_(int(POISON_I32))
+
+
+@pytest.mark.parametrize("M", [33, 100, 192])
+def test_sweep_gemm_choice(dev, api, M):
+    """A table encoded for the expanded-weights GEMM (TW_SWEEP_GEMM_EXPANDED)
+    at token counts where the default runs the weights-in-TMEM GEMM: the
+    oracle's sums and outputs, and the same bytes as the default table."""
+    import torch
+    shapes = [(200, 256), (128, 1536), (17, 384), (385, 640)]
+    descs, keep = [], []
+    for i, (N, K) in enumerate(shapes):
+        W = _weights(N, K, 7100 + 10 * M + i)
+        x = _acts(M, K, 7200 + 10 * M + i)
+        packed, _, wscale = G.ternarize_gpu(W, dev)
+        xq, amax, qsum = api.quantize_act(G.to_dev(x, dev))
+        descs.append(dict(xq=xq, amax=amax, qsum=qsum, packed=packed, wscale=wscale, N=N, K=K))
+        keep.append((W, x))
+    outs = {}
+    for gemm in ("expanded", "auto"):
+        ds = [dict(d, y=torch.full((M, d["N"]), float("nan"), dtype=torch.float32, device=dev),
+                   acc_out=torch.full((M, d["N"]), int(POISON_I32), dtype=torch.int32,
+                                      device=dev)) for d in descs]
+        table = api.SweepTable(ds, M, device=dev, gemm=gemm)
+        api.decoder_projection_sweep(table)
+        api.check()
+        outs[gemm] = [(d["y"].cpu().numpy(), d["acc_out"].cpu().numpy()) for d in ds]
+    for (ye, ae), (ya, aa), (W, x), (N, K) in zip(outs["expanded"], outs["auto"], keep, shapes):
+        codes, mean = orc.ternarize(W)
+        ref = orc.ternary_linear(x, codes, mean)
+        assert (ae == ref["acc"]).all(), (M, N, K)
+        G.assert_y_close(ye, ref["y"], f"expanded M={M} N={N} K={K}")
+        assert (ae == aa).all() and (ye.view(np.uint32) == ya.view(np.uint32)).all(), (M, N, K)
