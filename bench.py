@@ -848,6 +848,9 @@ def measure_configs(args, api, torch, dev, rank, shapes, weights, descs_m1, want
                                         / e["tmem_weights"]["us_per_step"])
             e["int8_ops"], e["algorithmic_bytes"] = ops, nbytes
             e["traffic"] = profiled_traffic("tw_mid.cu", M, args.layers)
+            if cpu_ok:
+                e["oracle"] = _oracle_sample(M, rows_cap=64, token_cap=M, budget_s=2.5,
+                                             layers=args.layers)
             out[f"f2_mid_sweep_196x_M{M}"] = e
             del descs
             torch.cuda.empty_cache()
