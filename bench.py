@@ -13,7 +13,8 @@ The same JSON line carries a ``configs`` object with every workload of the
 benchmark definition, measured in the same run on the same weights:
 
   1. one 1536x1536 GEMV at M = 1 (x without outliers), L2 flushed before
-     every call: us per call, median and p10/p90;
+     every call: us per call, median and p10/p90; and back to back over a
+     rotating pool of distinct matrices whose codes exceed twice the L2;
   2. one decoder layer's 7 projections at M = 1 as one sweep call, L2
      flushed before every call: us per matrix;
   3. the headline (196 projections, M = 1);
@@ -409,6 +410,26 @@ def cold_calls(torch, stream, fn, n, flush, batch=32, sleep_cycles=40_000_000):
     return per
 
 
+def pool_calls(torch, stream, fns, batch=64, sleep_cycles=40_000_000):
+    """Device time of each call in `fns`, run back to back in batches; a spin
+    kernel at the head of every batch lets the host queue the whole batch,
+    so an event after each call brackets device work only.  Returns
+    per-call ms (the first call of each batch is not timed)."""
+    per = []
+    for b0 in range(0, len(fns), batch):
+        chunk = fns[b0:b0 + batch]
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(chunk))]
+        torch.cuda._sleep(sleep_cycles)
+        chunk[0]()
+        evs[0].record(stream)
+        for fn, ev in zip(chunk[1:], evs[1:]):
+            fn()
+            ev.record(stream)
+        torch.cuda.synchronize()
+        per += [evs[i - 1].elapsed_time(evs[i]) for i in range(1, len(chunk))]
+    return per
+
+
 CHAIN_METRIC = "decoder-layer chain tokens/s (28 dependent layers; % of HBM roofline)"
 CHAIN_DIMS = (1536, 256, 128, 8960)   # hidden, kv_dim, head_dim, inter (Qwen2.5-1.5B)
 
@@ -740,6 +761,36 @@ def measure_configs(args, api, torch, dev, rank, shapes, weights, descs_m1, want
             "frac_hbm_at_median": nbytes / (s["median_us"] * 1e-6) / 1e9 / hbm,
             "launches_per_call": 2, "l2": "flushed (256 MB written) before every call",
             "note": "launch-latency bound: the 0.6 MB of work is 0.09 us of HBM time"}
+        # A rotating pool of distinct seeded 1536^2 matrices whose codes
+        # exceed twice the L2, called back to back: each call's matrix was
+        # last read a whole pool earlier, so it streams from HBM.
+        pool_n = -(-L2_FLUSH_BYTES // (N * K // 4))
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(20261202 + rank)
+        pool = []
+        for _ in range(pool_n):
+            Wi = torch.randn((N, K), generator=gen, device=dev).mul_(0.02)
+            pk, _, wsc = api.ternarize_pack(Wi)
+            pool.append((pk, wsc))
+            del Wi
+        api.check()
+
+        def call(i):
+            return lambda: api.ternary_linear(x, pool[i][0], pool[i][1], N, y=y, ws=ws)
+        fns = [call(i % pool_n) for i in range(2 * pool_n)]
+        for f in fns[:pool_n]:
+            f()
+        api.check()
+        per = pool_calls(torch, stream, fns)
+        api.check()
+        s = dist_summary(per)
+        out["1_gemv_1536x1536_M1"]["rotating_pool"] = {
+            "us_per_call": s, "matrices": pool_n, "pool_code_bytes": pool_n * (N * K // 4),
+            "gbs_at_median": nbytes / (s["median_us"] * 1e-6) / 1e9,
+            "frac_hbm_at_median": nbytes / (s["median_us"] * 1e-6) / 1e9 / hbm,
+            "note": "calls back to back over distinct W ~ N(0, 0.02^2) (device-seeded), "
+                    "codes of the pool > 2 x L2; one x and one y"}
+        del pool, fns
         if cpu_ok:
             out["1_gemv_1536x1536_M1"]["oracle"] = _oracle_call_us([(0, 0)], 1, 2.0)
 
